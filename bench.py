@@ -1,0 +1,417 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 LLM.int8() linear layer (one JSON line on stdout).
+
+A step is one llmint8_matmul call: the whole hot path (outlier detection, row
+quantisation, outlier tiles, int8 tcgen05 GEMM with the fused dequantisation /
+outlier product / fp16 store) on one batch of seeded synthetic input already
+resident in HBM. The metric is effective TOPS = 2*s*h*o / step time.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                  [--impl ours|reference]
+
+Timing: W untimed warm-up steps; then exactly K steps between a barrier +
+synchronize on both sides, each step timed with CUDA events on the launching
+stream. The L2 cache (126 MB) is flushed by writing a 512 MB buffer before
+every timed step (outside the step's events), because the default workload's
+inputs fit in L2. Multi-GPU (torchrun): independent replicas on every rank
+(the layer has no exchange step), time = max over ranks, value = total work of
+all ranks / that time.
+
+--impl reference times the CPU oracle (plain C, OpenMP) on the host cores,
+on a bounded row sample of the same workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from mixed_precision_int8_b200 import workloads  # noqa: E402
+
+METRIC = "LLM.int8() matmul effective TOPS"
+UNIT = "TOPS"
+DEFAULT_WORKLOAD = "opt6.7b_attn_prefill"
+FLUSH_BYTES = 512 << 20
+KERNEL_SOURCES = ["mixed_precision_int8_b200/csrc/gemm_sm100.cuh",
+                  "mixed_precision_int8_b200/csrc/decode_sm100.cuh",
+                  "mixed_precision_int8_b200/csrc/quant_kernels.cuh",
+                  "mixed_precision_int8_b200/csrc/ptx_sm100.cuh",
+                  "mixed_precision_int8_b200/csrc/llmint8_api.cu"]
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
+            "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def recorded_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernels are
+    unchanged since it was taken."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(workload, {}).get(kernel)
+    if not e or e.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML in a thread."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown",
+               0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap",
+               0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle",
+               0x2: "applications_clocks_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.002):
+        self.samples = []
+        self.ok = False
+        self.period = period_s
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(
+                self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._t is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self, t0: float, t1: float):
+        if not self.ok or not self.samples:
+            return None
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        use = inside if inside else self.samples
+        mhz = statistics.median(s[1] for s in use)
+        bits = 0
+        for s in use:
+            bits |= s[2]
+        reasons = sorted(n for b, n in self.REASONS.items()
+                         if bits & b and n != "gpu_idle")
+        return {"sm_mhz": mhz, "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(inside),
+                "window": "timed region" if inside else "whole run"}
+
+
+# ------------------------------------------------------------ CPU oracle
+
+def cpu_oracle_run(wl, X, Wq, aw, budget_s: float, max_rows: int = None):
+    """Time the oracle on a row sample sized to ~budget_s seconds."""
+    import oracle
+    rng = np.random.default_rng(123)
+    probe_rows = np.sort(rng.choice(wl.s, size=min(wl.s, 2), replace=False))
+    t = time.perf_counter()
+    oracle.matmul(X, Wq, aw, wl.alpha, rows=probe_rows)
+    dt = max(time.perf_counter() - t, 1e-4) / len(probe_rows)
+    n = int(max(1, min(wl.s, budget_s / dt)))
+    if max_rows:
+        n = min(n, max_rows)
+    rows = np.sort(rng.choice(wl.s, size=n, replace=False))
+    t = time.perf_counter()
+    oracle.matmul(X, Wq, aw, wl.alpha, rows=rows)
+    el = time.perf_counter() - t
+    tops = 2.0 * n * wl.h * wl.o / el / 1e12
+    return {"value": tops, "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{n} of {wl.s} rows x all {wl.o} columns of "
+                      f"{wl.name} (outlier set over all rows), {el:.1f} s"}
+
+
+# ---------------------------------------------------------------- ranks
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if _cuda_ok() else "gloo"
+        dist.init_process_group(backend=backend,
+                                timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def _cuda_ok():
+    import torch
+    return torch.cuda.is_available()
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64,
+                     device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def finish(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------- our path
+
+def run_ours(args, world, rank, local):
+    import torch
+    from mixed_precision_int8_b200 import binding, build
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    build.build()
+    binding.load_library()
+    wl, X, cols, W = workloads.make_inputs(args.workload)
+    s, h, o = wl.s, wl.h, wl.o
+    Xd = torch.from_numpy(X).to(dev)
+    Wd = torch.from_numpy(W).to(dev)
+    pw = binding.llmint8_prepare_weight(Wd)
+    torch.cuda.synchronize()
+    del Wd
+    out = torch.empty((s, o), dtype=torch.float16, device=dev)
+    ws = binding.Workspace(s, h, o, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    K, Wm = args.steps, args.warmup
+
+    def step(ev=None):
+        binding.llmint8_matmul(Xd, pw, wl.alpha, out=out, workspace=ws,
+                               events=ev)
+
+    for _ in range(Wm):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    launches_per_step = binding.llmint8_matmul.last_launches
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    g0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    g1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    clocks = ClockSampler(local) if rank == 0 else None
+    if clocks:
+        clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    t_wall0 = time.perf_counter()
+    for k in range(K):
+        flush.fill_(k & 0xFF)
+        starts[k].record(stream)
+        step((g0[k], g1[k]))
+        stops[k].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    t_wall1 = time.perf_counter()
+    if clocks:
+        clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, stops)]
+    gemm_ms = [a.elapsed_time(b) for a, b in zip(g0, g1)]
+    ms_per_step = max_over_ranks(sum(step_ms) / K, world, dev)
+    gemm_ms_avg = sum(gemm_ms) / K
+    status_bits = binding.llmint8_read_device_status(ws)
+
+    # end to end through the host-buffer entry point
+    Xh = torch.from_numpy(X).pin_memory()
+    outh = torch.empty((s, o), dtype=torch.float16).pin_memory()
+    wsh = binding.Workspace(s, h, o, device=dev, host=True)
+    for _ in range(max(1, Wm)):
+        binding.llmint8_matmul_host(Xh, pw, wl.alpha, outh, wsh)
+    e_ms = []
+    barrier(world)
+    torch.cuda.synchronize()
+    for k in range(K):
+        flush.fill_(k & 0xFF)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        binding.llmint8_matmul_host(Xh, pw, wl.alpha, outh, wsh)
+        b.record(stream)
+        b.synchronize()
+        e_ms.append(a.elapsed_time(b))
+    barrier(world)
+    e2e_ms = max_over_ranks(sum(e_ms) / K, world, dev)
+
+    ops = 2.0 * s * h * o
+    value = world * ops / (ms_per_step * 1e-3) / 1e12
+    e2e_value = world * ops / (e2e_ms * 1e-3) / 1e12
+    peaks = measured_peaks()
+    decode = s <= binding.llmint8_decode_max_rows()
+    if decode:
+        kernel = "k_decode_i8"
+        algo_bytes = h * o + 16 * h  # int8 weight + padded int8 rows
+        achieved = algo_bytes / (gemm_ms_avg * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                "kernel": kernel,
+                "peak_source": f"hbm_gbs ({peaks['source']})"}
+    else:
+        kernel = "k_gemm_i8_fused"
+        peak = 2.0 * peaks["bf16_tflops"]
+        achieved = ops / (gemm_ms_avg * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "kernel": kernel,
+                "peak_source": "bf16_tflops x 2 (nominal int8/bf16 dense "
+                               f"ratio 4.5/2.25), {peaks['source']}"}
+    roof["traffic"] = recorded_traffic(wl.name, kernel)
+    roof["kernel_ms"] = gemm_ms_avg
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": Wm, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "i8", "data": "synthetic (seeded, OPT-shaped outliers)",
+        "config": {"workload": wl.name, "s": s, "h": h, "o": o,
+                   "alpha": wl.alpha, "outlier_cols": int(len(cols)),
+                   "parallelism": f"replicas x{world}" if world > 1 else "single",
+                   "l2": "flushed (512 MB write) before every timed step"},
+        "e2e": {"value": e2e_value, "unit": UNIT,
+                "h2d_bytes_per_step": 2 * s * h,
+                "d2h_bytes_per_step": 2 * s * o},
+        "gpu_launches": launches_per_step * K,
+        "roofline": roof,
+        "device_status": status_bits,
+    }
+    if clocks:
+        line["clocks"] = clocks.summary(t_wall0, t_wall1)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        Wq = pw.wq.cpu().numpy()
+        aw = pw.aw.cpu().numpy()
+        line["cpu_baseline"] = cpu_oracle_run(wl, X, Wq, aw, args.cpu_seconds)
+    return line
+
+
+# ------------------------------------------------------ reference (oracle)
+
+def run_reference(args, world, rank, local):
+    if rank != 0:
+        return None
+    import oracle
+    wl, X, cols, W = workloads.make_inputs(args.workload)
+    Wq, aw = oracle.prepare_weight(W)
+    per_step = max(0.2, args.cpu_seconds / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_oracle_run(wl, X, Wq, aw, per_step)
+    vals, samples = [], []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        r = cpu_oracle_run(wl, X, Wq, aw, per_step)
+        vals.append(r["value"])
+        samples.append(r["sample"])
+    el = time.perf_counter() - t0
+    value = statistics.mean(vals)
+    ms = 2.0 * wl.s * wl.h * wl.o / (value * 1e12) * 1e3
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "i8 codes, fp64 accumulation",
+        "data": "synthetic (seeded, OPT-shaped outliers)",
+        "config": {"workload": wl.name, "s": wl.s, "h": wl.h, "o": wl.o,
+                   "alpha": wl.alpha, "parallelism": "single"},
+        "cpu_baseline": {"value": value, "unit": UNIT,
+                         "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": f"per step: {samples[-1]}; "
+                                   f"{args.steps} steps in {el:.1f} s"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=list(workloads.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        # rank 0 alone times the CPU oracle; other ranks exit without work
+        if int(os.environ.get("RANK", "0")) != 0:
+            return
+        line = run_reference(args, 1, 0, 0)
+        line["n_gpus"] = int(os.environ.get("WORLD_SIZE", "1"))
+        print(json.dumps(line), flush=True)
+        return
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        line = run_ours(args, world, rank, local)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        finish(world)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,210 @@
+/*
+ * llmint8.h — C ABI of the B200 (sm_100a) LLM.int8() linear-layer library.
+ *
+ * The library computes C = X.W for a transformer linear layer the way the
+ * LLM.int8() method does it:
+ *
+ *   Step 1  outlier detection: O = { j : some row i has |X[i][j]| >= alpha }
+ *   Step 2  decomposition: X^O = X[:, O] and W^O = W[O, :] (fp16);
+ *           the rest of X and W goes to the int8 path
+ *   Step 3  fp16 outlier product X^O . W^O (fp32 accumulation)
+ *   Step 4  vector-wise absmax quantisation: one scale per row of X (over the
+ *           non-outlier columns), one per column of W; int8 x int8 product
+ *           accumulated in int32; dequantised by the outer product of the
+ *           scales (divided by 127*127)
+ *   Step 5  sum of the two parts, stored once as fp16.
+ *
+ * Sources: "LLM.int8(): 8-bit Matrix Multiplication for Transformers at Scale"
+ * (paper-graph-ui summary), section "The Full LLM.int8() Algorithm", Steps 1-5,
+ * and sections "Vector-wise Quantization" and "Mixed-Precision Decomposition";
+ * "tm_llm_int8" (aicassindra.com), sections "Absmax INT8 quantization from
+ * first principles" and "The mixed-precision decomposition";
+ * "LLM.int8() 完全拆解" (pinghaoyang.com.cn), sections "第一件武器：向量级量化"
+ * and "第二件武器：混合精度分解".
+ *
+ * Conventions for every entry point:
+ *  - Half-precision tensors are IEEE binary16, passed as uint16_t bit
+ *    patterns. All tensors are dense and row-major unless stated.
+ *  - Pointers named *_dev are device pointers of the current CUDA device,
+ *    owned by the caller; the library never allocates or frees device memory
+ *    (scratch space comes from the caller's workspace).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream). Calls are asynchronous: LLMINT8_OK means "validated and
+ *    enqueued", except where a function says it synchronises.
+ *  - Arguments are validated on the host before anything is enqueued; on an
+ *    error return nothing has been enqueued and no output was touched.
+ *  - Shape rules: 16 <= h <= 133144 and h % 16 == 0 (16-byte TMA row
+ *    strides for int8; 127*127*h must fit int32); o >= 16 and o % 16 == 0;
+ *    s >= 0 (s == 0 is a no-op that returns LLMINT8_OK). Device pointers to
+ *    fp16/int8 tensors must be 16-byte aligned; the workspace 256-byte aligned.
+ *  - alpha must be >= 0 (and not NaN); alpha = +inf switches the
+ *    decomposition off (pure vector-wise int8). The comparison is |x| >= alpha.
+ *  - Rounding of int8 codes: q = round-half-away-from-zero(fp32(127*x) / a)
+ *    with one IEEE fp32 division; a == 0 gives q == 0.
+ *  - The kernels contain only bounded waits. If one runs out (it should not),
+ *    the kernel records a bit in the workspace's status word and returns;
+ *    llmint8_read_device_status() reports and clears it.
+ *  - Only sm_100 devices are supported; other devices give
+ *    LLMINT8_ERR_UNSUPPORTED. There is no CPU fallback.
+ */
+#ifndef LLMINT8_H_
+#define LLMINT8_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LLMINT8_API __attribute__((visibility("default")))
+#else
+#define LLMINT8_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LLMINT8_OK = 0,
+    LLMINT8_ERR_NULL = -1,          /* a required pointer is NULL */
+    LLMINT8_ERR_SHAPE = -2,         /* a size breaks the shape rules */
+    LLMINT8_ERR_ALIGN = -3,         /* a pointer breaks the alignment rules */
+    LLMINT8_ERR_WORKSPACE = -4,     /* workspace smaller than required */
+    LLMINT8_ERR_CUDA = -5,          /* a CUDA runtime/driver call failed */
+    LLMINT8_ERR_DEVICE_STATUS = -6, /* a kernel flagged an anomaly */
+    LLMINT8_ERR_ARG = -7,           /* a scalar argument is invalid */
+    LLMINT8_ERR_UNSUPPORTED = -8    /* current device is not sm_100 */
+} llmint8_status;
+
+/* Bits of the device status word (llmint8_read_device_status). */
+#define LLMINT8_DEV_TIMEOUT_PRODUCER 0x1  /* TMA producer gave up waiting */
+#define LLMINT8_DEV_TIMEOUT_MMA 0x2       /* MMA issuer gave up waiting */
+#define LLMINT8_DEV_TIMEOUT_EPILOGUE 0x4  /* epilogue gave up waiting */
+#define LLMINT8_DEV_TIMEOUT_DRAIN 0x8     /* drain after an abort timed out */
+
+/* A prepared (offline-quantised) weight. Buffers are caller-owned device
+ * memory: wq_dev is int8 [o][h] (the reduction index k contiguous, i.e. the
+ * transpose of W), aw_dev is fp32 [o] holding each column's absmax (an exact
+ * binary16 value). */
+typedef struct {
+    int64_t h;
+    int64_t o;
+    int8_t *wq_dev;
+    float *aw_dev;
+} llmint8_weight;
+
+/* Optional extras for llmint8_matmul_ex (all fields may be zero/NULL).
+ *  gemm_event_start/stop: cudaEvent_t (as void*) recorded on `stream`
+ *      immediately before and after the int8 GEMM kernel launch, for timing
+ *      the dominant kernel from the caller.
+ *  ci_dev: if non-NULL, int32 [s][o] receives the exact int32 accumulators
+ *      of Step 4 (testing; costs an extra 4*s*o bytes of stores).
+ *  path: 0 = automatic, 1 = force the prefill GEMM kernel, 2 = force the
+ *      decode (s <= 16) kernel; 2 with s > 16 is LLMINT8_ERR_ARG.
+ *  launches (out): number of kernels this call enqueued. */
+typedef struct {
+    void *gemm_event_start;
+    void *gemm_event_stop;
+    int32_t *ci_dev;
+    int32_t path;
+    int32_t launches;
+} llmint8_matmul_opts;
+
+/* Human-readable name of a status code (static storage). */
+LLMINT8_API const char *llmint8_status_string(llmint8_status st);
+
+/* Bytes of device workspace llmint8_matmul needs for an [s,h] x [h,o]
+ * problem. Sized for the worst case |O| = h, so any alpha fits:
+ * about s*h (int8 codes) + 2*s*h (fp16 outlier columns of X) + 2*h*o (fp16
+ * outlier rows of W) + 4*16*o (decode accumulators) + O(h + s). */
+LLMINT8_API size_t llmint8_workspace_size(int64_t s, int64_t h, int64_t o);
+
+/* Clears the workspace's status block (its first 256 bytes). Call once on a
+ * new workspace before its first llmint8_matmul; asynchronous on `stream`. */
+LLMINT8_API llmint8_status llmint8_workspace_init(void *ws_dev, size_t ws_bytes, void *stream);
+
+/* Workspace for llmint8_matmul_host: llmint8_workspace_size plus staging
+ * for the device copies of X (2*s*h bytes) and of C (2*s*o bytes). */
+LLMINT8_API size_t llmint8_workspace_size_host(int64_t s, int64_t h, int64_t o);
+
+/* Offline weight preparation ("The Full LLM.int8() Algorithm", Step 1 remark
+ * that W's part is fixed at model-load time, and section "Why vector-wise
+ * rather than row-wise": column constants precomputed once):
+ *   aw[j]    = max_k |W[k][j]|            over all h rows
+ *   wq[j][k] = q(W[k][j], aw[j])           (see rounding rule above)
+ * W_dev is fp16 [h][o]. out->h, out->o must equal h, o and out->wq_dev /
+ * out->aw_dev must point at caller buffers of o*h and o elements. */
+LLMINT8_API llmint8_status llmint8_prepare_weight(const uint16_t *W_dev, int64_t h,
+                                      int64_t o, llmint8_weight *out,
+                                      void *stream);
+
+/* Steps 1 and 4 (activation side) on their own, for testing:
+ *   flags_dev[j]  = 1 if column j is an outlier column, else 0   (u8 [h])
+ *   idx_dev[0..n) = outlier columns in ascending order           (i32 [h])
+ *   *n_outliers_dev = n                                          (i32 scalar)
+ *   ax_dev[i]     = max over non-outlier j of |X[i][j]| (0 if none) (f32 [s])
+ *   Xq_dev[i][j]  = q(X[i][j], ax[i]) for non-outlier j, else 0  (i8 [s][h])
+ * X_dev is fp16 [s][h]. scratch_dev must hold
+ * llmint8_quantize_rows_scratch_size(h) bytes (256-byte aligned). */
+LLMINT8_API size_t llmint8_quantize_rows_scratch_size(int64_t h);
+LLMINT8_API llmint8_status llmint8_quantize_rows(const uint16_t *X_dev, int64_t s,
+                                     int64_t h, float alpha, int8_t *Xq_dev,
+                                     float *ax_dev, uint8_t *flags_dev,
+                                     int32_t *idx_dev, int32_t *n_outliers_dev,
+                                     void *scratch_dev, size_t scratch_bytes,
+                                     void *stream);
+
+/* The whole layer, Steps 1-5: out_dev (fp16 [s][o]) = LLM.int8()(X_dev, w).
+ *   out[i][j] = fp16( Ci[i][j] * ax[i] * aw[j] / (127*127)
+ *                     + sum_{t in O} X[i][t] * WO[t][j] )
+ * where WO[t][j] = fp16( fp32(fp32(wq[j][t]) * aw[j]) / 127 ) is the fp16
+ * outlier row of W recovered from the int8 weight (the prepared weight is
+ * the only copy of W the library holds). Ci is exact; the fp16 outlier
+ * product and the dequantisation use fp32 arithmetic. ws_dev must hold
+ * llmint8_workspace_size(s, h, o) bytes; it may be reused across calls on
+ * the same stream, not shared by calls that can overlap. |O| stays on the
+ * device: the call never synchronises. */
+LLMINT8_API llmint8_status llmint8_matmul(const uint16_t *X_dev, int64_t s,
+                              const llmint8_weight *w, float alpha,
+                              uint16_t *out_dev, void *ws_dev, size_t ws_bytes,
+                              void *stream);
+
+/* llmint8_matmul with the extras of llmint8_matmul_opts (opts may be NULL). */
+LLMINT8_API llmint8_status llmint8_matmul_ex(const uint16_t *X_dev, int64_t s,
+                                 const llmint8_weight *w, float alpha,
+                                 uint16_t *out_dev, void *ws_dev,
+                                 size_t ws_bytes, llmint8_matmul_opts *opts,
+                                 void *stream);
+
+/* End-to-end form with HOST buffers: copies X_host (fp16 [s][h], ideally
+ * pinned) into the workspace, runs llmint8_matmul, copies C back into
+ * out_host (fp16 [s][o]) and synchronises `stream` before returning.
+ * ws_dev must hold llmint8_workspace_size_host(s, h, o) bytes. */
+LLMINT8_API llmint8_status llmint8_matmul_host(const uint16_t *X_host, int64_t s,
+                                   const llmint8_weight *w, float alpha,
+                                   uint16_t *out_host, void *ws_dev,
+                                   size_t ws_bytes, void *stream);
+
+/* The fp16 outlier tiles of the last llmint8_matmul on this workspace:
+ * copies n_outliers (to *n_out_host), XO (fp16 [s][n], to XO_host if
+ * non-NULL) and WO (fp16 [n][o], to WO_host if non-NULL) from the workspace
+ * to host memory sized for n = h. Synchronises `stream`. Testing aid. */
+LLMINT8_API llmint8_status llmint8_read_outlier_tiles(const void *ws_dev, size_t ws_bytes,
+                                          int64_t s, int64_t h, int64_t o,
+                                          int32_t *n_out_host,
+                                          uint16_t *XO_host, uint16_t *WO_host,
+                                          void *stream);
+
+/* Reads and clears the device status word kept in a matmul workspace;
+ * synchronises `stream`. Returns LLMINT8_ERR_DEVICE_STATUS if any bit was
+ * set (bits also stored in *bits_out when non-NULL), else LLMINT8_OK. */
+LLMINT8_API llmint8_status llmint8_read_device_status(void *ws_dev, size_t ws_bytes,
+                                          int32_t *bits_out, void *stream);
+
+/* Largest s the decode kernel accepts. */
+LLMINT8_API int64_t llmint8_decode_max_rows(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LLMINT8_H_ */

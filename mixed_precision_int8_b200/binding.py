@@ -1,0 +1,262 @@
+"""ctypes binding of libllmint8.so (the C ABI in include/llmint8.h).
+
+Argument marshalling only: every step of the layer runs in the library's
+CUDA kernels. PyTorch provides device memory and streams. The functions keep
+the C names; tensors are passed as device pointers, the stream as the current
+torch stream. If the library is missing, loading fails loudly: there is no
+CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libllmint8.so")
+
+OK = 0
+STATUS_NAMES = {0: "OK", -1: "ERR_NULL", -2: "ERR_SHAPE", -3: "ERR_ALIGN",
+                -4: "ERR_WORKSPACE", -5: "ERR_CUDA", -6: "ERR_DEVICE_STATUS",
+                -7: "ERR_ARG", -8: "ERR_UNSUPPORTED"}
+
+_c_i64, _c_i32, _c_f32 = ctypes.c_int64, ctypes.c_int32, ctypes.c_float
+_vp, _sz = ctypes.c_void_p, ctypes.c_size_t
+
+
+class llmint8_weight(ctypes.Structure):
+    _fields_ = [("h", _c_i64), ("o", _c_i64), ("wq_dev", _vp), ("aw_dev", _vp)]
+
+
+class llmint8_matmul_opts(ctypes.Structure):
+    _fields_ = [("gemm_event_start", _vp), ("gemm_event_stop", _vp),
+                ("ci_dev", _vp), ("path", _c_i32), ("launches", _c_i32)]
+
+
+class Llmint8Error(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        self.code = code
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(code, code)}"
+                         f" ({status_string(code) if _lib is not None else ''})")
+
+
+_lib = None
+
+
+def load_library():
+    """Load libllmint8.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} not found: build it with `python -m "
+            "mixed_precision_int8_b200.build` (or __graft_entry__.build())")
+    lib = ctypes.CDLL(LIB_PATH)
+    sig = {
+        "llmint8_status_string": ([_c_i32], ctypes.c_char_p),
+        "llmint8_workspace_size": ([_c_i64, _c_i64, _c_i64], _sz),
+        "llmint8_workspace_size_host": ([_c_i64, _c_i64, _c_i64], _sz),
+        "llmint8_workspace_init": ([_vp, _sz, _vp], _c_i32),
+        "llmint8_prepare_weight": ([_vp, _c_i64, _c_i64,
+                                    ctypes.POINTER(llmint8_weight), _vp], _c_i32),
+        "llmint8_quantize_rows_scratch_size": ([_c_i64], _sz),
+        "llmint8_quantize_rows": ([_vp, _c_i64, _c_i64, _c_f32, _vp, _vp, _vp,
+                                   _vp, _vp, _vp, _sz, _vp], _c_i32),
+        "llmint8_matmul": ([_vp, _c_i64, ctypes.POINTER(llmint8_weight), _c_f32,
+                            _vp, _vp, _sz, _vp], _c_i32),
+        "llmint8_matmul_ex": ([_vp, _c_i64, ctypes.POINTER(llmint8_weight),
+                               _c_f32, _vp, _vp, _sz,
+                               ctypes.POINTER(llmint8_matmul_opts), _vp], _c_i32),
+        "llmint8_matmul_host": ([_vp, _c_i64, ctypes.POINTER(llmint8_weight),
+                                 _c_f32, _vp, _vp, _sz, _vp], _c_i32),
+        "llmint8_read_outlier_tiles": ([_vp, _sz, _c_i64, _c_i64, _c_i64, _vp,
+                                        _vp, _vp, _vp], _c_i32),
+        "llmint8_read_device_status": ([_vp, _sz, _vp, _vp], _c_i32),
+        "llmint8_decode_max_rows": ([], _c_i64),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = lib
+    return lib
+
+
+EXPORTED = ("llmint8_status_string", "llmint8_workspace_size",
+            "llmint8_workspace_size_host", "llmint8_workspace_init",
+            "llmint8_prepare_weight", "llmint8_quantize_rows_scratch_size",
+            "llmint8_quantize_rows", "llmint8_matmul", "llmint8_matmul_ex",
+            "llmint8_matmul_host", "llmint8_read_outlier_tiles",
+            "llmint8_read_device_status", "llmint8_decode_max_rows")
+
+
+def status_string(code: int) -> str:
+    return load_library().llmint8_status_string(code).decode()
+
+
+def _check(fn: str, code: int):
+    if code != OK:
+        raise Llmint8Error(fn, code)
+
+
+def _stream(stream: Optional[torch.cuda.Stream] = None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _f16_dev(t: torch.Tensor, name: str):
+    if t.dtype != torch.float16 or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA float16 tensor")
+
+
+class PreparedWeight:
+    """Device buffers of a prepared weight: wq int8 [o,h], aw float32 [o]."""
+
+    def __init__(self, wq: torch.Tensor, aw: torch.Tensor):
+        self.wq = wq
+        self.aw = aw
+        self.o, self.h = wq.shape
+        self.c = llmint8_weight(self.h, self.o, wq.data_ptr(), aw.data_ptr())
+
+
+class Workspace:
+    """A caller-owned device workspace (torch uint8 buffer) for one stream."""
+
+    def __init__(self, s: int, h: int, o: int, device=None, host: bool = False):
+        lib = load_library()
+        size_fn = (lib.llmint8_workspace_size_host if host
+                   else lib.llmint8_workspace_size)
+        self.nbytes = int(size_fn(s, h, o))
+        self.buf = torch.empty(self.nbytes, dtype=torch.uint8,
+                               device=device or "cuda")
+        self.s, self.h, self.o = s, h, o
+        _check("llmint8_workspace_init",
+               lib.llmint8_workspace_init(_ptr(self.buf), self.nbytes, _stream()))
+
+
+def llmint8_workspace_size(s: int, h: int, o: int) -> int:
+    return int(load_library().llmint8_workspace_size(s, h, o))
+
+
+def llmint8_decode_max_rows() -> int:
+    return int(load_library().llmint8_decode_max_rows())
+
+
+def llmint8_prepare_weight(W: torch.Tensor, stream=None) -> PreparedWeight:
+    """W fp16 [h,o] on the GPU -> PreparedWeight (int8 [o,h] codes + scales)."""
+    _f16_dev(W, "W")
+    h, o = W.shape
+    wq = torch.empty((o, h), dtype=torch.int8, device=W.device)
+    aw = torch.empty((o,), dtype=torch.float32, device=W.device)
+    pw = PreparedWeight(wq, aw)
+    _check("llmint8_prepare_weight", load_library().llmint8_prepare_weight(
+        _ptr(W), h, o, ctypes.byref(pw.c), _stream(stream)))
+    return pw
+
+
+def llmint8_quantize_rows(X: torch.Tensor, alpha: float = 6.0, stream=None):
+    """Steps 1 and 4 (activation side) -> (Xq, ax, flags, idx, n_outliers).
+
+    n_outliers is a 1-element device tensor (it is never read back here);
+    idx holds valid entries in its first n_outliers slots.
+    """
+    _f16_dev(X, "X")
+    s, h = X.shape
+    dev = X.device
+    lib = load_library()
+    Xq = torch.empty((s, h), dtype=torch.int8, device=dev)
+    ax = torch.empty((s,), dtype=torch.float32, device=dev)
+    flags = torch.empty((h,), dtype=torch.uint8, device=dev)
+    idx = torch.empty((h,), dtype=torch.int32, device=dev)
+    n = torch.empty((1,), dtype=torch.int32, device=dev)
+    nb = int(lib.llmint8_quantize_rows_scratch_size(h))
+    scratch = torch.empty(max(nb, 256), dtype=torch.uint8, device=dev)
+    _check("llmint8_quantize_rows", lib.llmint8_quantize_rows(
+        _ptr(X), s, h, float(alpha), _ptr(Xq), _ptr(ax), _ptr(flags), _ptr(idx),
+        _ptr(n), _ptr(scratch), nb, _stream(stream)))
+    return Xq, ax, flags, idx, n
+
+
+def llmint8_matmul(X: torch.Tensor, w: PreparedWeight, alpha: float = 6.0,
+                   out: Optional[torch.Tensor] = None,
+                   workspace: Optional[Workspace] = None,
+                   ci: Optional[torch.Tensor] = None, path: int = 0,
+                   events=None, stream=None) -> torch.Tensor:
+    """C = LLM.int8()(X, W): X fp16 [s,h] on the GPU -> fp16 [s,o].
+
+    ci (optional, int32 [s,o]) receives the exact int32 accumulators; path
+    forces the prefill (1) or decode (2) kernel; events = (start, stop)
+    torch.cuda.Event pair recorded around the GEMM kernel.
+    """
+    _f16_dev(X, "X")
+    s, h = X.shape
+    if h != w.h:
+        raise ValueError(f"X has h={h}, weight has h={w.h}")
+    if out is None:
+        out = torch.empty((s, w.o), dtype=torch.float16, device=X.device)
+    if workspace is None:
+        workspace = Workspace(s, h, w.o, device=X.device)
+    opts = llmint8_matmul_opts()
+    opts.path = int(path)
+    if ci is not None:
+        if ci.dtype != torch.int32 or ci.shape != (s, w.o):
+            raise ValueError("ci must be int32 [s,o]")
+        opts.ci_dev = ci.data_ptr()
+    if events is not None:
+        opts.gemm_event_start = events[0].cuda_event
+        opts.gemm_event_stop = events[1].cuda_event
+    _check("llmint8_matmul_ex", load_library().llmint8_matmul_ex(
+        _ptr(X), s, ctypes.byref(w.c), float(alpha), _ptr(out),
+        _ptr(workspace.buf), workspace.nbytes, ctypes.byref(opts),
+        _stream(stream)))
+    llmint8_matmul.last_launches = int(opts.launches)
+    return out
+
+
+def llmint8_matmul_host(X_host: torch.Tensor, w: PreparedWeight,
+                        alpha: float, out_host: torch.Tensor,
+                        workspace: Workspace, stream=None) -> torch.Tensor:
+    """End-to-end form: host fp16 X in, host fp16 C out (synchronises)."""
+    if X_host.is_cuda or out_host.is_cuda:
+        raise ValueError("X_host and out_host must be host tensors")
+    s, h = X_host.shape
+    _check("llmint8_matmul_host", load_library().llmint8_matmul_host(
+        _ptr(X_host), s, ctypes.byref(w.c), float(alpha), _ptr(out_host),
+        _ptr(workspace.buf), workspace.nbytes, _stream(stream)))
+    return out_host
+
+
+def llmint8_read_outlier_tiles(workspace: Workspace, stream=None):
+    """(n, XO [s,n] fp16, WO [n,o] fp16) of the last matmul on `workspace`."""
+    s, h, o = workspace.s, workspace.h, workspace.o
+    n = ctypes.c_int32(0)
+    XO = torch.empty((s * h,), dtype=torch.float16)
+    WO = torch.empty((h * o,), dtype=torch.float16)
+    _check("llmint8_read_outlier_tiles", load_library().llmint8_read_outlier_tiles(
+        _ptr(workspace.buf), workspace.nbytes, s, h, o, ctypes.byref(n),
+        _ptr(XO), _ptr(WO), _stream(stream)))
+    k = n.value
+    return k, XO[: s * k].view(s, k), WO[: k * o].view(k, o)
+
+
+def llmint8_read_device_status(workspace: Workspace, stream=None) -> int:
+    bits = ctypes.c_int32(0)
+    rc = load_library().llmint8_read_device_status(
+        _ptr(workspace.buf), workspace.nbytes, ctypes.byref(bits), _stream(stream))
+    if rc not in (OK, -6):
+        _check("llmint8_read_device_status", rc)
+    return bits.value
+
+
+def effective_tops(s: int, h: int, o: int, seconds: float) -> float:
+    return 2.0 * s * h * o / seconds / 1e12 if seconds > 0 else math.nan

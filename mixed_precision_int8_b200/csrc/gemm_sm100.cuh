@@ -1,0 +1,284 @@
+// K3: the int8 GEMM of LLM.int8() on 5th-generation tensor cores, with the
+// dequantisation, the fp16 outlier product and the fp16 store fused into its
+// epilogue.
+//
+// Math ("The Full LLM.int8() Algorithm", Steps 3-5; "Vector-wise
+// Quantization"):
+//   Ci[i][j]  = sum_k Xq[i][k] * Wq[j][k]                    int8 -> int32
+//   out[i][j] = fp16( Ci[i][j] * (ax[i] / 16129) * aw[j]
+//                     + sum_t XO[i][t] * WO[t][j] )          fp32
+//
+// Structure (one persistent CTA per SM, 256 threads):
+//   warp 0      TMA producer: Xq and Wq tiles (128-byte swizzle) into a
+//               4-stage shared-memory ring, completion on mbarriers
+//   warp 1      one thread issues tcgen05.mma.kind::i8 (M=128, N=256, K=32)
+//               into a TMEM accumulator; tcgen05.commit frees ring slots
+//   warp 2      allocates / frees the 512 TMEM columns (2 accumulators)
+//   warps 4-7   epilogue: tcgen05.ld of the int32 accumulator (each warp
+//               owns 32 TMEM lanes = 32 output rows), dequantise, add the
+//               outlier product on CUDA cores, store fp16; the other
+//               accumulator is being filled by the MMA meanwhile.
+// Every wait is bounded by the global timer; on a timeout the CTA records a
+// status bit, drains its in-flight copies and MMAs, frees TMEM and returns.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_fp16.h>
+
+#include "ptx_sm100.cuh"
+
+namespace llmint8 {
+namespace gemm {
+
+constexpr int BM = 128;           // output rows per tile (MMA M)
+constexpr int BN = 256;           // output columns per tile (MMA N)
+constexpr int BK = 128;           // int8 reduction bytes per stage
+constexpr int STAGES = 4;
+constexpr int UMMA_K = 32;        // K of one kind::i8 MMA
+constexpr uint32_t A_STAGE_BYTES = BM * BK;
+constexpr uint32_t B_STAGE_BYTES = BN * BK;
+constexpr int NUM_ACC = 2;
+constexpr uint32_t TMEM_COLS = 512;  // NUM_ACC * BN int32 columns
+constexpr int NUM_THREADS = 256;
+constexpr int EPI_WARP0 = 4;
+constexpr int NUM_EPI_THREADS = 128;
+constexpr size_t SMEM_BYTES =
+    1024 + (size_t)STAGES * (A_STAGE_BYTES + B_STAGE_BYTES) + 256;
+
+static_assert(NUM_ACC * BN <= 512, "TMEM holds 512 columns");
+
+struct Params {
+  int32_t s, h, o;
+  int32_t num_m_blocks, num_n_blocks, num_k_blocks;
+  const float *ax;        // [s]
+  const float *aw;        // [o]
+  const uint16_t *XO;     // [s][n_out] fp16
+  const uint16_t *WO;     // [n_out][o] fp16
+  const int32_t *n_out;   // device scalar |O|
+  uint16_t *out;          // [s][o] fp16
+  int32_t *ci;            // optional [s][o] int32
+  int32_t *status;        // device status word
+  uint64_t timeout_ns;
+};
+
+__device__ __forceinline__ uint32_t f2h2(float a, float b) {
+  const __half2 v = __floats2half2_rn(a, b);
+  return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    k_gemm_i8_fused(const __grid_constant__ CUtensorMap tmA,
+                    const __grid_constant__ CUtensorMap tmB, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (raw_addr & 1023u)) & 1023u;
+  uint8_t *base = smem_raw + pad;
+  const uint32_t sA = smem_u32(base);
+  const uint32_t sB = sA + STAGES * A_STAGE_BYTES;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(base + STAGES * (A_STAGE_BYTES + B_STAGE_BYTES));
+  // barrier indices
+  const uint32_t bar0 = smem_u32(bars);
+  auto full_bar = [&](int st) { return bar0 + 8u * st; };
+  auto empty_bar = [&](int st) { return bar0 + 8u * (STAGES + st); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + NUM_ACC + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 2 * NUM_ACC);
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 2 * NUM_ACC + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(full_bar(i), 1);
+      mbar_init(empty_bar(i), 1);
+    }
+    for (int a = 0; a < NUM_ACC; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), NUM_EPI_THREADS);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  const int32_t num_tiles = p.num_m_blocks * p.num_n_blocks;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------ TMA producer
+    uint32_t stage = 0, phase = 0;
+    uint32_t issued = 0, last_par = 0;  // per-stage bits, for the drain
+    bool ok = true;
+    for (int32_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      const int32_t m_blk = tile % p.num_m_blocks;
+      const int32_t n_blk = tile / p.num_m_blocks;
+      for (int32_t kb = 0; kb < p.num_k_blocks; ++kb) {
+        if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, p.status,
+                               LLMINT8_DEV_TIMEOUT_PRODUCER, p.timeout_ns)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(full_bar(stage), A_STAGE_BYTES + B_STAGE_BYTES);
+        tma_load_2d(sA + stage * A_STAGE_BYTES, &tmA, full_bar(stage), kb * BK, m_blk * BM);
+        tma_load_2d(sB + stage * B_STAGE_BYTES, &tmB, full_bar(stage), kb * BK, n_blk * BN);
+        issued |= 1u << stage;
+        last_par = (last_par & ~(1u << stage)) | (phase << stage);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!ok) {
+      // let every copy this thread started land before shared memory goes
+      volatile int never = 0;
+      for (int st = 0; st < STAGES; ++st)
+        if ((issued >> st) & 1u)
+          mbar_wait_bounded(full_bar(st), (last_par >> st) & 1u, &never, p.status,
+                            LLMINT8_DEV_TIMEOUT_DRAIN, p.timeout_ns);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------- MMA issuer
+    constexpr uint32_t idesc = idesc_i8_s32(BM, BN);
+    uint32_t stage = 0, phase = 0;
+    bool ok = true;
+    bool any = false;
+    int32_t it = 0;
+    for (int32_t tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+      const uint32_t acc = it & 1, acc_par = (it >> 1) & 1;
+      if (!mbar_wait_bounded(tempty_bar(acc), acc_par ^ 1u, abort_flag, p.status,
+                             LLMINT8_DEV_TIMEOUT_MMA, p.timeout_ns)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * BN;
+      for (int32_t kb = 0; kb < p.num_k_blocks; ++kb) {
+        if (!mbar_wait_bounded(full_bar(stage), phase, abort_flag, p.status,
+                               LLMINT8_DEV_TIMEOUT_MMA, p.timeout_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t a_desc = smem_desc_kmajor_sw128(sA + stage * A_STAGE_BYTES);
+        const uint64_t b_desc = smem_desc_kmajor_sw128(sB + stage * B_STAGE_BYTES);
+#pragma unroll
+        for (int k = 0; k < BK / UMMA_K; ++k) {
+          // advance the start address by k*32 bytes inside the swizzle atom
+          mma_i8(d_tmem, a_desc + (uint64_t)((k * UMMA_K) >> 4),
+                 b_desc + (uint64_t)((k * UMMA_K) >> 4), idesc, (kb > 0 || k > 0) ? 1u : 0u);
+        }
+        any = true;
+        mma_commit(empty_bar(stage));
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      mma_commit(tfull_bar(acc));
+    }
+    if (!ok && any) {
+      volatile int never = 0;
+      mma_commit(drain_bar);
+      mbar_wait_bounded(drain_bar, 0, &never, p.status, LLMINT8_DEV_TIMEOUT_DRAIN,
+                        p.timeout_ns);
+    }
+  } else if (warp >= EPI_WARP0) {
+    // --------------------------------------------------------- epilogue
+    const int ew = warp - EPI_WARP0;  // TMEM lane quarter of this warp
+    const int32_t n_out = *p.n_out;
+    int32_t it = 0;
+    for (int32_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+      const uint32_t acc = it & 1, acc_par = (it >> 1) & 1;
+      if (!mbar_wait_bounded(tfull_bar(acc), acc_par, abort_flag, p.status,
+                             LLMINT8_DEV_TIMEOUT_EPILOGUE, p.timeout_ns))
+        break;
+      tc_fence_after();
+      const int32_t m_blk = tile % p.num_m_blocks;
+      const int32_t n_blk = tile / p.num_m_blocks;
+      const int32_t row = m_blk * BM + ew * 32 + lane;
+      const bool row_ok = row < p.s;
+      const float rs = row_ok ? p.ax[row] * (1.0f / 16129.0f) : 0.0f;
+      const uint32_t t_row = tmem_base + ((uint32_t)(ew * 32) << 16) + acc * BN;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        __syncwarp();
+        tmem_ld_32x32b_x32(t_row + c * 32, v);
+        tmem_ld_wait();
+        const int32_t j0 = n_blk * BN + c * 32;
+        if (j0 >= p.o || !row_ok) continue;  // lanes reconverge at __syncwarp
+        const bool full = (j0 + 32 <= p.o);  // else exactly 16 valid (o % 16 == 0)
+        float accf[32];
+        const float4 *awp = reinterpret_cast<const float4 *>(p.aw + j0);
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+          float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (full || q4 < 4) a4 = __ldg(awp + q4);
+          accf[4 * q4 + 0] = (float)(int32_t)v[4 * q4 + 0] * rs * a4.x;
+          accf[4 * q4 + 1] = (float)(int32_t)v[4 * q4 + 1] * rs * a4.y;
+          accf[4 * q4 + 2] = (float)(int32_t)v[4 * q4 + 2] * rs * a4.z;
+          accf[4 * q4 + 3] = (float)(int32_t)v[4 * q4 + 3] * rs * a4.w;
+        }
+        const uint16_t *xo_row = p.XO + (int64_t)row * n_out;
+        for (int32_t t = 0; t < n_out; ++t) {
+          const float xo = __half2float(__ushort_as_half(xo_row[t]));
+          const uint4 *wp = reinterpret_cast<const uint4 *>(p.WO + (int64_t)t * p.o + j0);
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) {
+            if (!full && q8 >= 2) break;
+            const uint4 w8 = __ldg(wp + q8);
+            const uint32_t ww[4] = {w8.x, w8.y, w8.z, w8.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&ww[e]));
+              accf[8 * q8 + 2 * e] = fmaf(xo, f.x, accf[8 * q8 + 2 * e]);
+              accf[8 * q8 + 2 * e + 1] = fmaf(xo, f.y, accf[8 * q8 + 2 * e + 1]);
+            }
+          }
+        }
+        uint4 *op = reinterpret_cast<uint4 *>(p.out + (int64_t)row * p.o + j0);
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8) {
+          if (!full && q8 >= 2) break;
+          op[q8] = make_uint4(f2h2(accf[8 * q8 + 0], accf[8 * q8 + 1]),
+                              f2h2(accf[8 * q8 + 2], accf[8 * q8 + 3]),
+                              f2h2(accf[8 * q8 + 4], accf[8 * q8 + 5]),
+                              f2h2(accf[8 * q8 + 6], accf[8 * q8 + 7]));
+        }
+        if (p.ci != nullptr) {
+          int4 *cp = reinterpret_cast<int4 *>(p.ci + (int64_t)row * p.o + j0);
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            if (!full && q4 >= 4) break;
+            cp[q4] = make_int4((int)v[4 * q4], (int)v[4 * q4 + 1], (int)v[4 * q4 + 2],
+                               (int)v[4 * q4 + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(tempty_bar(acc));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem_base, TMEM_COLS);
+}
+
+}  // namespace gemm
+}  // namespace llmint8

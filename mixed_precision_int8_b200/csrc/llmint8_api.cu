@@ -1,0 +1,499 @@
+// C ABI of the LLM.int8() linear-layer library (declared in include/llmint8.h):
+// argument validation, workspace layout, TMA descriptor creation and the
+// launch sequence of the kernels in quant_kernels.cuh and gemm_sm100.cuh.
+// Host code only enqueues work; it never allocates device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "llmint8.h"
+#include "quant_kernels.cuh"
+#include "gemm_sm100.cuh"
+#include "decode_sm100.cuh"
+
+namespace {
+
+using namespace llmint8;
+
+constexpr int64_t kMaxH = 133144;  // 127*127*h must fit int32
+constexpr int64_t kDecodeMaxRows = decode::MAX_ROWS;
+constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per individual wait
+
+// ----------------------------------------------------------- device info
+struct DeviceInfo {
+  bool init = false;
+  bool supported = false;
+  int sm_count = 0;
+  bool gemm_attr = false;
+  bool decode_attr = false;
+};
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mutex;
+
+llmint8_status device_info(DeviceInfo **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return LLMINT8_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceInfo &d = g_dev[dev];
+  if (!d.init) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return LLMINT8_ERR_CUDA;
+    d.supported = (prop.major == 10 && prop.minor == 0);
+    d.sm_count = prop.multiProcessorCount;
+    if (d.supported) {
+      if (cudaFuncSetAttribute(gemm::k_gemm_i8_fused, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)gemm::SMEM_BYTES) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+      if (cudaFuncSetAttribute(decode::k_decode_i8, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)decode::SMEM_BYTES) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+    }
+    d.init = true;
+  }
+  if (!d.supported) return LLMINT8_ERR_UNSUPPORTED;
+  *out = &d;
+  return LLMINT8_OK;
+}
+
+// ----------------------------------------------------- TMA descriptors
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D int8 tensor [rows][inner] with row stride `inner` bytes, box
+// [box_rows][box_inner] landing in shared memory with the 128-byte swizzle.
+bool make_tmap_i8(CUtensorMap *map, const void *ptr, uint64_t inner, uint64_t rows,
+                  uint32_t box_inner, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------ workspace layout
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Layout {
+  size_t status, mask, wprefix, idx, ax, xq, xo, wo, cacc, end;
+  size_t xstage, ostage, end_host;
+};
+
+int32_t mask_words(int64_t h) { return (int32_t)((h + 31) / 32); }
+
+Layout layout_for(int64_t s, int64_t h, int64_t o) {
+  Layout L;
+  size_t off = 0;
+  L.status = off;  off = align256(off + 256);
+  L.mask = off;    off = align256(off + 4 * (size_t)mask_words(h));
+  L.wprefix = off; off = align256(off + 4 * ((size_t)mask_words(h) + 1));
+  L.idx = off;     off = align256(off + 4 * (size_t)h);
+  L.ax = off;      off = align256(off + 4 * (size_t)s);
+  L.xq = off;      off = align256(off + (size_t)s * h);
+  L.xo = off;      off = align256(off + 2 * (size_t)s * h);
+  L.wo = off;      off = align256(off + 2 * (size_t)h * o);
+  L.cacc = off;    off = align256(off + 4 * (size_t)kDecodeMaxRows * o);
+  L.end = off;
+  L.xstage = off;  off = align256(off + 2 * (size_t)s * h);
+  L.ostage = off;  off = align256(off + 2 * (size_t)s * o);
+  L.end_host = off;
+  return L;
+}
+
+// status block: [0] device status bits, [1] |O|
+int32_t *status_word(void *ws) { return reinterpret_cast<int32_t *>(ws); }
+int32_t *count_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 1; }
+
+// --------------------------------------------------------- validation
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+llmint8_status check_hw(int64_t h, int64_t o) {
+  if (h < 16 || h > kMaxH || (h % 16) != 0) return LLMINT8_ERR_SHAPE;
+  if (o < 16 || (o % 16) != 0 || o > (int64_t)INT32_MAX / 2) return LLMINT8_ERR_SHAPE;
+  return LLMINT8_OK;
+}
+
+llmint8_status check_alpha(float alpha) {
+  if (std::isnan(alpha) || alpha < 0.0f) return LLMINT8_ERR_ARG;
+  return LLMINT8_OK;
+}
+
+float half_bits_value(uint32_t b) {
+  const int e = (b >> 10) & 0x1f, m = b & 0x3ff;
+  if (e == 0) return std::ldexp((float)m, -24);
+  if (e == 31) return m ? NAN : INFINITY;
+  return std::ldexp((float)(1024 + m), e - 25);
+}
+
+// Smallest non-negative binary16 magnitude bit pattern whose value is >=
+// alpha (0x7C00 = +inf when none is finite), so that for a non-NaN x,
+// |x| >= alpha  <=>  (bits(x) & 0x7FFF) >= threshold.
+uint32_t threshold_bits(float alpha) {
+  uint32_t lo = 0, hi = 0x7C00;
+  while (lo < hi) {
+    const uint32_t mid = (lo + hi) / 2;
+    if (half_bits_value(mid) >= alpha) hi = mid;
+    else lo = mid + 1;
+  }
+  return lo;
+}
+
+cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+
+llmint8_status last_launch() {
+  return cudaGetLastError() == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA;
+}
+
+// Steps 1 and 4 (activation side): bitmask, compaction, row scales and codes.
+// Returns the number of kernels enqueued through *launches.
+llmint8_status enqueue_activation_pass(const DeviceInfo &dev, const uint16_t *X, int64_t s,
+                                       int64_t h, float alpha, uint32_t *mask,
+                                       int32_t *wprefix, int32_t *idx, int32_t *count,
+                                       uint8_t *flags, int8_t *Xq, float *ax, uint16_t *XO,
+                                       cudaStream_t st, int32_t *launches) {
+  const int32_t nwords = mask_words(h);
+  const int32_t hh = (int32_t)h;
+  k_reset_mask<<<(nwords + 255) / 256, 256, 0, st>>>(mask, nwords, count);
+  const int gx = (int)((h + kColsPerBlock - 1) / kColsPerBlock);
+  const int64_t want_blocks = 4 * (int64_t)dev.sm_count;
+  int64_t gy_target = (want_blocks + gx - 1) / gx;
+  int64_t rpb = (s + gy_target - 1) / gy_target;
+  if (rpb < 4) rpb = 4;
+  if ((s + rpb - 1) / rpb > 65535) rpb = (s + 65534) / 65535;
+  const int gy = (int)((s + rpb - 1) / rpb);
+  k_outlier_columns<<<dim3(gx, gy), kColThreads, 0, st>>>(X, s, hh, threshold_bits(alpha),
+                                                         (int32_t)rpb, mask);
+  k_compact_outliers<<<1, kCompactThreads, 0, st>>>(mask, nwords, hh, wprefix, idx, count, flags);
+  const int64_t rb = (s + kRowsPerBlock - 1) / kRowsPerBlock;
+  k_quantize_rows<<<(unsigned)rb, kRowThreads, 0, st>>>(X, s, hh, mask, wprefix, count, Xq, ax,
+                                                       XO);
+  *launches += 4;
+  return last_launch();
+}
+
+llmint8_status validate_weight(const llmint8_weight *w) {
+  if (!w || !w->wq_dev || !w->aw_dev) return LLMINT8_ERR_NULL;
+  llmint8_status st = check_hw(w->h, w->o);
+  if (st) return st;
+  if (!aligned(w->wq_dev, 16) || !aligned(w->aw_dev, 16)) return LLMINT8_ERR_ALIGN;
+  return LLMINT8_OK;
+}
+
+llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w, float alpha,
+                           uint16_t *out, void *ws, size_t ws_bytes, llmint8_matmul_opts *opts,
+                           cudaStream_t st, bool host_layout) {
+  if (opts) opts->launches = 0;
+  llmint8_status rc = validate_weight(w);
+  if (rc) return rc;
+  if (s < 0 || s > (int64_t)INT32_MAX) return LLMINT8_ERR_SHAPE;
+  if ((rc = check_alpha(alpha))) return rc;
+  const int path = opts ? opts->path : 0;
+  if (path < 0 || path > 2 || (path == 2 && s > kDecodeMaxRows)) return LLMINT8_ERR_ARG;
+  if (s == 0) return LLMINT8_OK;
+  if (!X || !out || !ws) return LLMINT8_ERR_NULL;
+  if (!aligned(X, 16) || !aligned(out, 16) || !aligned(ws, 256)) return LLMINT8_ERR_ALIGN;
+  if (opts && opts->ci_dev && !aligned(opts->ci_dev, 16)) return LLMINT8_ERR_ALIGN;
+  const int64_t h = w->h, o = w->o;
+  const Layout L = layout_for(s, h, o);
+  if (ws_bytes < (host_layout ? L.end_host : L.end)) return LLMINT8_ERR_WORKSPACE;
+  DeviceInfo *dev = nullptr;
+  if ((rc = device_info(&dev))) return rc;
+
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  uint32_t *mask = reinterpret_cast<uint32_t *>(wsb + L.mask);
+  int32_t *wprefix = reinterpret_cast<int32_t *>(wsb + L.wprefix);
+  int32_t *idx = reinterpret_cast<int32_t *>(wsb + L.idx);
+  float *ax = reinterpret_cast<float *>(wsb + L.ax);
+  int8_t *xq = reinterpret_cast<int8_t *>(wsb + L.xq);
+  uint16_t *xo = reinterpret_cast<uint16_t *>(wsb + L.xo);
+  uint16_t *wo = reinterpret_cast<uint16_t *>(wsb + L.wo);
+  int32_t *cacc = reinterpret_cast<int32_t *>(wsb + L.cacc);
+  int32_t *count = count_word(ws);
+  int32_t *status = status_word(ws);
+
+  const bool use_decode = (path == 2) || (path == 0 && s <= kDecodeMaxRows);
+
+  // Tensor maps first: a failure here must leave nothing enqueued.
+  CUtensorMap tmA, tmB;
+  if (use_decode) {
+    // A = Wq tiles (rows of o), B = Xq rows (s <= 16, zero-filled to 16)
+    if (!make_tmap_i8(&tmA, w->wq_dev, (uint64_t)h, (uint64_t)o, decode::BK, decode::BM) ||
+        !make_tmap_i8(&tmB, xq, (uint64_t)h, (uint64_t)s, decode::BK, decode::BN))
+      return LLMINT8_ERR_CUDA;
+  } else {
+    if (!make_tmap_i8(&tmA, xq, (uint64_t)h, (uint64_t)s, gemm::BK, gemm::BM) ||
+        !make_tmap_i8(&tmB, w->wq_dev, (uint64_t)h, (uint64_t)o, gemm::BK, gemm::BN))
+      return LLMINT8_ERR_CUDA;
+  }
+
+  int32_t launches = 0;
+  if ((rc = enqueue_activation_pass(*dev, X, s, h, alpha, mask, wprefix, idx, count, nullptr, xq,
+                                    ax, xo, st, &launches)))
+    return rc;
+  {
+    dim3 grid((unsigned)((o + 255) / 256), 8);
+    k_outlier_weights<<<grid, 256, 0, st>>>(w->wq_dev, w->aw_dev, (int32_t)h, (int32_t)o, idx,
+                                           count, wo);
+    ++launches;
+  }
+  if (use_decode) {
+    decode::Params p;
+    p.s = (int32_t)s;
+    p.h = (int32_t)h;
+    p.o = (int32_t)o;
+    p.num_m_blocks = (int32_t)((o + decode::BM - 1) / decode::BM);
+    p.num_k_blocks = (int32_t)((h + decode::BK - 1) / decode::BK);
+    p.ax = ax;
+    p.aw = w->aw_dev;
+    p.XO = xo;
+    p.WO = wo;
+    p.n_out = count;
+    p.out = out;
+    p.ci = opts ? opts->ci_dev : nullptr;
+    p.cacc = cacc;
+    p.status = status;
+    p.timeout_ns = kTimeoutNs;
+    const int64_t total_units = (int64_t)p.num_m_blocks * p.num_k_blocks;
+    int grid = dev->sm_count;
+    if (total_units < grid) grid = (int)total_units;
+    p.units_total = total_units;
+    decode::k_decode_zero<<<(unsigned)((kDecodeMaxRows * o + 1023) / 1024), 256, 0, st>>>(
+        cacc, (int64_t)kDecodeMaxRows * o);
+    ++launches;
+    if (opts && opts->gemm_event_start)
+      cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->gemm_event_start), st);
+    decode::k_decode_i8<<<grid, decode::NUM_THREADS, decode::SMEM_BYTES, st>>>(tmA, tmB, p);
+    if (opts && opts->gemm_event_stop)
+      cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->gemm_event_stop), st);
+    ++launches;
+    decode::k_decode_finish<<<(unsigned)((s * o + 255) / 256), 256, 0, st>>>(p);
+    ++launches;
+  } else {
+    gemm::Params p;
+    p.s = (int32_t)s;
+    p.h = (int32_t)h;
+    p.o = (int32_t)o;
+    p.num_m_blocks = (int32_t)((s + gemm::BM - 1) / gemm::BM);
+    p.num_n_blocks = (int32_t)((o + gemm::BN - 1) / gemm::BN);
+    p.num_k_blocks = (int32_t)((h + gemm::BK - 1) / gemm::BK);
+    p.ax = ax;
+    p.aw = w->aw_dev;
+    p.XO = xo;
+    p.WO = wo;
+    p.n_out = count;
+    p.out = out;
+    p.ci = opts ? opts->ci_dev : nullptr;
+    p.status = status;
+    p.timeout_ns = kTimeoutNs;
+    const int64_t tiles = (int64_t)p.num_m_blocks * p.num_n_blocks;
+    const int grid = (int)(tiles < dev->sm_count ? tiles : dev->sm_count);
+    if (opts && opts->gemm_event_start)
+      cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->gemm_event_start), st);
+    gemm::k_gemm_i8_fused<<<grid, gemm::NUM_THREADS, gemm::SMEM_BYTES, st>>>(tmA, tmB, p);
+    if (opts && opts->gemm_event_stop)
+      cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->gemm_event_stop), st);
+    ++launches;
+  }
+  if (opts) opts->launches = launches;
+  return last_launch();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *llmint8_status_string(llmint8_status st) {
+  switch (st) {
+    case LLMINT8_OK: return "ok";
+    case LLMINT8_ERR_NULL: return "required pointer is NULL";
+    case LLMINT8_ERR_SHAPE: return "size breaks the shape rules";
+    case LLMINT8_ERR_ALIGN: return "pointer breaks the alignment rules";
+    case LLMINT8_ERR_WORKSPACE: return "workspace too small";
+    case LLMINT8_ERR_CUDA: return "CUDA call failed";
+    case LLMINT8_ERR_DEVICE_STATUS: return "a kernel flagged an anomaly";
+    case LLMINT8_ERR_ARG: return "invalid scalar argument";
+    case LLMINT8_ERR_UNSUPPORTED: return "current device is not sm_100";
+  }
+  return "unknown status";
+}
+
+size_t llmint8_workspace_size(int64_t s, int64_t h, int64_t o) {
+  if (s < 0 || h < 0 || o < 0) return 0;
+  return layout_for(s, h, o).end;
+}
+
+llmint8_status llmint8_workspace_init(void *ws_dev, size_t ws_bytes, void *stream) {
+  if (!ws_dev) return LLMINT8_ERR_NULL;
+  if (!aligned(ws_dev, 256)) return LLMINT8_ERR_ALIGN;
+  if (ws_bytes < 256) return LLMINT8_ERR_WORKSPACE;
+  return cudaMemsetAsync(ws_dev, 0, 256, as_stream(stream)) == cudaSuccess ? LLMINT8_OK
+                                                                           : LLMINT8_ERR_CUDA;
+}
+
+size_t llmint8_workspace_size_host(int64_t s, int64_t h, int64_t o) {
+  if (s < 0 || h < 0 || o < 0) return 0;
+  return layout_for(s, h, o).end_host;
+}
+
+int64_t llmint8_decode_max_rows(void) { return kDecodeMaxRows; }
+
+llmint8_status llmint8_prepare_weight(const uint16_t *W_dev, int64_t h, int64_t o,
+                                      llmint8_weight *out, void *stream) {
+  if (!W_dev || !out || !out->wq_dev || !out->aw_dev) return LLMINT8_ERR_NULL;
+  llmint8_status rc = check_hw(h, o);
+  if (rc) return rc;
+  if (out->h != h || out->o != o) return LLMINT8_ERR_SHAPE;
+  if (!aligned(W_dev, 16) || !aligned(out->wq_dev, 16) || !aligned(out->aw_dev, 16))
+    return LLMINT8_ERR_ALIGN;
+  DeviceInfo *dev = nullptr;
+  if ((rc = device_info(&dev))) return rc;
+  cudaStream_t st = as_stream(stream);
+  uint32_t *awb = reinterpret_cast<uint32_t *>(out->aw_dev);
+  const int32_t hh = (int32_t)h, oo = (int32_t)o;
+  k_zero_u32<<<(unsigned)((o + 255) / 256), 256, 0, st>>>(awb, o);
+  const int gx = (int)((o / 8 + 255) / 256);
+  int64_t gy_target = (8 * (int64_t)dev->sm_count + gx - 1) / gx;
+  int64_t rpb = (h + gy_target - 1) / gy_target;
+  if (rpb < 8) rpb = 8;
+  const int gy = (int)((h + rpb - 1) / rpb);
+  k_weight_colmax<<<dim3(gx, gy), 256, 0, st>>>(W_dev, hh, oo, (int32_t)rpb, awb);
+  k_weight_codes<<<dim3((unsigned)((o + kWqTile - 1) / kWqTile),
+                        (unsigned)((h + kWqTile - 1) / kWqTile)),
+                   256, 0, st>>>(W_dev, hh, oo, awb, out->wq_dev);
+  k_widen_scales<<<(unsigned)((o + 255) / 256), 256, 0, st>>>(awb, oo);
+  return last_launch();
+}
+
+size_t llmint8_quantize_rows_scratch_size(int64_t h) {
+  if (h < 0) return 0;
+  return align256(4 * (size_t)mask_words(h)) + align256(4 * ((size_t)mask_words(h) + 1));
+}
+
+llmint8_status llmint8_quantize_rows(const uint16_t *X_dev, int64_t s, int64_t h, float alpha,
+                                     int8_t *Xq_dev, float *ax_dev, uint8_t *flags_dev,
+                                     int32_t *idx_dev, int32_t *n_outliers_dev,
+                                     void *scratch_dev, size_t scratch_bytes, void *stream) {
+  if (h < 16 || h > kMaxH || (h % 16) != 0) return LLMINT8_ERR_SHAPE;
+  if (s < 0 || s > (int64_t)INT32_MAX) return LLMINT8_ERR_SHAPE;
+  llmint8_status rc = check_alpha(alpha);
+  if (rc) return rc;
+  if (!flags_dev || !idx_dev || !n_outliers_dev || !scratch_dev) return LLMINT8_ERR_NULL;
+  if (s > 0 && (!X_dev || !Xq_dev || !ax_dev)) return LLMINT8_ERR_NULL;
+  if ((s > 0 && (!aligned(X_dev, 16) || !aligned(Xq_dev, 16))) || !aligned(scratch_dev, 256) ||
+      !aligned(idx_dev, 4) || !aligned(n_outliers_dev, 4) || (s > 0 && !aligned(ax_dev, 4)))
+    return LLMINT8_ERR_ALIGN;
+  if (scratch_bytes < llmint8_quantize_rows_scratch_size(h)) return LLMINT8_ERR_WORKSPACE;
+  DeviceInfo *dev = nullptr;
+  if ((rc = device_info(&dev))) return rc;
+  uint8_t *sb = static_cast<uint8_t *>(scratch_dev);
+  uint32_t *mask = reinterpret_cast<uint32_t *>(sb);
+  int32_t *wprefix = reinterpret_cast<int32_t *>(sb + align256(4 * (size_t)mask_words(h)));
+  int32_t launches = 0;
+  return enqueue_activation_pass(*dev, X_dev, s, h, alpha, mask, wprefix, idx_dev, n_outliers_dev,
+                                 flags_dev, Xq_dev, ax_dev, nullptr, as_stream(stream), &launches);
+}
+
+llmint8_status llmint8_matmul(const uint16_t *X_dev, int64_t s, const llmint8_weight *w,
+                              float alpha, uint16_t *out_dev, void *ws_dev, size_t ws_bytes,
+                              void *stream) {
+  return matmul_impl(X_dev, s, w, alpha, out_dev, ws_dev, ws_bytes, nullptr, as_stream(stream),
+                     false);
+}
+
+llmint8_status llmint8_matmul_ex(const uint16_t *X_dev, int64_t s, const llmint8_weight *w,
+                                 float alpha, uint16_t *out_dev, void *ws_dev, size_t ws_bytes,
+                                 llmint8_matmul_opts *opts, void *stream) {
+  return matmul_impl(X_dev, s, w, alpha, out_dev, ws_dev, ws_bytes, opts, as_stream(stream),
+                     false);
+}
+
+llmint8_status llmint8_matmul_host(const uint16_t *X_host, int64_t s, const llmint8_weight *w,
+                                   float alpha, uint16_t *out_host, void *ws_dev, size_t ws_bytes,
+                                   void *stream) {
+  llmint8_status rc = validate_weight(w);
+  if (rc) return rc;
+  if (s < 0 || s > (int64_t)INT32_MAX) return LLMINT8_ERR_SHAPE;
+  if ((rc = check_alpha(alpha))) return rc;
+  if (s == 0) return LLMINT8_OK;
+  if (!X_host || !out_host || !ws_dev) return LLMINT8_ERR_NULL;
+  if (!aligned(ws_dev, 256)) return LLMINT8_ERR_ALIGN;
+  const Layout L = layout_for(s, w->h, w->o);
+  if (ws_bytes < L.end_host) return LLMINT8_ERR_WORKSPACE;
+  cudaStream_t st = as_stream(stream);
+  uint8_t *wsb = static_cast<uint8_t *>(ws_dev);
+  uint16_t *xd = reinterpret_cast<uint16_t *>(wsb + L.xstage);
+  uint16_t *od = reinterpret_cast<uint16_t *>(wsb + L.ostage);
+  if (cudaMemcpyAsync(xd, X_host, 2 * (size_t)s * w->h, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return LLMINT8_ERR_CUDA;
+  if ((rc = matmul_impl(xd, s, w, alpha, od, ws_dev, ws_bytes, nullptr, st, true))) return rc;
+  if (cudaMemcpyAsync(out_host, od, 2 * (size_t)s * w->o, cudaMemcpyDeviceToHost, st) !=
+      cudaSuccess)
+    return LLMINT8_ERR_CUDA;
+  return cudaStreamSynchronize(st) == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA;
+}
+
+llmint8_status llmint8_read_outlier_tiles(const void *ws_dev, size_t ws_bytes, int64_t s,
+                                          int64_t h, int64_t o, int32_t *n_out_host,
+                                          uint16_t *XO_host, uint16_t *WO_host, void *stream) {
+  if (!ws_dev || !n_out_host) return LLMINT8_ERR_NULL;
+  if (s < 0 || h < 0 || o < 0) return LLMINT8_ERR_SHAPE;
+  const Layout L = layout_for(s, h, o);
+  if (ws_bytes < L.end) return LLMINT8_ERR_WORKSPACE;
+  cudaStream_t st = as_stream(stream);
+  const uint8_t *wsb = static_cast<const uint8_t *>(ws_dev);
+  int32_t n = 0;
+  if (cudaMemcpyAsync(&n, wsb + 4, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return LLMINT8_ERR_CUDA;
+  if (n < 0 || n > h) return LLMINT8_ERR_DEVICE_STATUS;
+  *n_out_host = n;
+  if (XO_host && n > 0 &&
+      cudaMemcpyAsync(XO_host, wsb + L.xo, 2 * (size_t)s * n, cudaMemcpyDeviceToHost, st) !=
+          cudaSuccess)
+    return LLMINT8_ERR_CUDA;
+  if (WO_host && n > 0 &&
+      cudaMemcpyAsync(WO_host, wsb + L.wo, 2 * (size_t)n * o, cudaMemcpyDeviceToHost, st) !=
+          cudaSuccess)
+    return LLMINT8_ERR_CUDA;
+  return cudaStreamSynchronize(st) == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA;
+}
+
+llmint8_status llmint8_read_device_status(void *ws_dev, size_t ws_bytes, int32_t *bits_out,
+                                          void *stream) {
+  if (!ws_dev) return LLMINT8_ERR_NULL;
+  if (ws_bytes < 256) return LLMINT8_ERR_WORKSPACE;
+  cudaStream_t st = as_stream(stream);
+  int32_t bits = 0;
+  if (cudaMemcpyAsync(&bits, ws_dev, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemsetAsync(ws_dev, 0, 4, st) != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess)
+    return LLMINT8_ERR_CUDA;
+  if (bits_out) *bits_out = bits;
+  return bits ? LLMINT8_ERR_DEVICE_STATUS : LLMINT8_OK;
+}
+
+}  // extern "C"

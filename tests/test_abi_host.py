@@ -1,0 +1,168 @@
+"""Host-side checks of the C ABI that need no GPU: the library builds and
+loads, exports every entry point the header declares, sizes workspaces as
+documented and rejects invalid arguments before touching the device.
+
+Invalid-argument calls here use placeholder pointers that must never be
+dereferenced: every call is chosen so that host validation rejects it first.
+They are skipped when a GPU is visible (the GPU suite covers validation with
+real device buffers).
+"""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+import torch
+
+from mixed_precision_int8_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "llmint8.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.load_library()
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"LLMINT8_API\s+[\w\s\*]*?\b(llmint8_\w+)\s*\(",
+                                 text)))
+
+
+def test_header_declares_the_entry_points_of_the_boundary():
+    names = _declared_functions()
+    for required in ("llmint8_prepare_weight", "llmint8_matmul",
+                     "llmint8_quantize_rows", "llmint8_workspace_size",
+                     "llmint8_status_string"):
+        assert required in names
+    assert set(names) == set(binding.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_library_has_no_torch_or_oracle_dependency():
+    import subprocess
+    out = subprocess.run(["ldd", binding.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    assert "torch" not in out and "oracle" not in out
+
+
+def test_status_strings(lib):
+    for code in range(-8, 1):
+        assert binding.status_string(code)
+    assert binding.status_string(-3) == "pointer breaks the alignment rules"
+
+
+def test_workspace_size_formula(lib):
+    def a256(x):
+        return (x + 255) // 256 * 256
+
+    for s, h, o in [(16, 256, 256), (2048, 4096, 4096), (8, 12288, 49152),
+                    (3, 272, 784)]:
+        nw = (h + 31) // 32
+        exp = (256 + a256(4 * nw) + a256(4 * (nw + 1)) + a256(4 * h)
+               + a256(4 * s) + a256(s * h) + a256(2 * s * h) + a256(2 * h * o)
+               + a256(4 * 16 * o))
+        assert lib.llmint8_workspace_size(s, h, o) == exp
+        assert (lib.llmint8_workspace_size_host(s, h, o)
+                == exp + a256(2 * s * h) + a256(2 * s * o))
+    assert lib.llmint8_workspace_size(-1, 16, 16) == 0
+    assert lib.llmint8_decode_max_rows() == 16
+
+
+needs_no_gpu = pytest.mark.skipif(torch.cuda.is_available(),
+                                  reason="placeholder pointers: CPU box only")
+
+FAKE = ctypes.c_void_p(1 << 20)  # 16/256-aligned, never dereferenced
+
+
+def _weight(h, o, wq=FAKE, aw=FAKE):
+    return binding.llmint8_weight(h, o, wq, aw)
+
+
+@needs_no_gpu
+@pytest.mark.parametrize("h,o", [(8, 256), (100, 256), (133160, 256),
+                                 (256, 8), (256, 100)])
+def test_matmul_rejects_bad_shapes(lib, h, o):
+    w = _weight(h, o)
+    rc = lib.llmint8_matmul(FAKE, 4, ctypes.byref(w), 6.0, FAKE, FAKE,
+                            1 << 40, None)
+    assert rc == -2
+
+
+@needs_no_gpu
+def test_matmul_rejects_nulls_alignment_alpha_and_small_workspace(lib):
+    w = _weight(256, 256)
+    big = 1 << 40
+    null_w = _weight(256, 256, wq=None)
+    assert lib.llmint8_matmul(FAKE, 4, ctypes.byref(null_w), 6.0, FAKE, FAKE,
+                              big, None) == -1
+    assert lib.llmint8_matmul(None, 4, ctypes.byref(w), 6.0, FAKE, FAKE,
+                              big, None) == -1
+    assert lib.llmint8_matmul(ctypes.c_void_p((1 << 20) + 2), 4,
+                              ctypes.byref(w), 6.0, FAKE, FAKE, big, None) == -3
+    assert lib.llmint8_matmul(FAKE, 4, ctypes.byref(w), 6.0, FAKE,
+                              ctypes.c_void_p((1 << 20) + 16), big, None) == -3
+    for bad_alpha in (-1.0, math.nan):
+        assert lib.llmint8_matmul(FAKE, 4, ctypes.byref(w), bad_alpha, FAKE,
+                                  FAKE, big, None) == -7
+    need = lib.llmint8_workspace_size(4, 256, 256)
+    assert lib.llmint8_matmul(FAKE, 4, ctypes.byref(w), 6.0, FAKE, FAKE,
+                              need - 1, None) == -4
+    assert lib.llmint8_matmul(FAKE, -1, ctypes.byref(w), 6.0, FAKE, FAKE,
+                              big, None) == -2
+    # s == 0 is a validated no-op
+    assert lib.llmint8_matmul(None, 0, ctypes.byref(w), 6.0, None, None, 0,
+                              None) == 0
+    # forcing the decode kernel beyond its row limit
+    opts = binding.llmint8_matmul_opts()
+    opts.path = 2
+    assert lib.llmint8_matmul_ex(FAKE, 17, ctypes.byref(w), 6.0, FAKE, FAKE,
+                                 big, ctypes.byref(opts), None) == -7
+    opts.path = 3
+    assert lib.llmint8_matmul_ex(FAKE, 4, ctypes.byref(w), 6.0, FAKE, FAKE,
+                                 big, ctypes.byref(opts), None) == -7
+
+
+@needs_no_gpu
+def test_prepare_and_quantize_rows_validation(lib):
+    w = _weight(256, 256)
+    assert lib.llmint8_prepare_weight(None, 256, 256, ctypes.byref(w),
+                                      None) == -1
+    assert lib.llmint8_prepare_weight(FAKE, 256, 512, ctypes.byref(w),
+                                      None) == -2
+    assert lib.llmint8_prepare_weight(FAKE, 24, 256, ctypes.byref(w),
+                                      None) == -2
+    nb = lib.llmint8_quantize_rows_scratch_size(256)
+    assert nb > 0
+    args = [FAKE, 4, 256, 6.0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, nb, None]
+    bad = list(args)
+    bad[2] = 250
+    assert lib.llmint8_quantize_rows(*bad) == -2
+    bad = list(args)
+    bad[10] = nb - 1
+    assert lib.llmint8_quantize_rows(*bad) == -4
+    bad = list(args)
+    bad[3] = -0.5
+    assert lib.llmint8_quantize_rows(*bad) == -7
+    bad = list(args)
+    bad[6] = None
+    assert lib.llmint8_quantize_rows(*bad) == -1
+
+
+@needs_no_gpu
+def test_valid_call_without_a_gpu_reports_cuda_error_not_a_fallback(lib):
+    # Arguments pass validation; with no device the library must fail, never
+    # compute on the host.
+    w = _weight(256, 256)
+    need = lib.llmint8_workspace_size(4, 256, 256)
+    rc = lib.llmint8_matmul(FAKE, 4, ctypes.byref(w), 6.0, FAKE, FAKE, need,
+                            None)
+    assert rc in (-5, -8)

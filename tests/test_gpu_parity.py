@@ -1,0 +1,236 @@
+"""GPU parity of the CUDA path (through the C ABI) against the CPU oracle.
+
+Bit-exact: outlier flags / list / count, row scales, int8 row codes, weight
+scales and codes, the fp16 outlier tiles and the int32 accumulators.
+Within |gpu - oracle| <= 2e-3 (1 + |oracle|): the fp16 output.
+
+Small cases run the oracle on every output; the five OPT-shaped workloads
+run it on seeded row x column samples (each output element of the method
+depends only on its row of X, the global outlier set and its weight column).
+"""
+import functools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mixed_precision_int8_b200 import binding, build, workloads
+from tests.parity_utils import (assert_close_fp16, gpu_matmul, gpu_prepare,
+                                oracle_prepared, sample_cols, sample_rows,
+                                to_dev)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    build.build()
+    binding.load_library()
+    yield
+
+
+# (s, h, o, outlier columns, alpha) — ragged tails in every dimension
+SMALL = [
+    (16, 256, 256, (7, 200), 6.0),
+    (1, 128, 256, (3,), 6.0),
+    (3, 144, 48, (0, 143), 6.0),
+    (8, 512, 784, (5, 6, 7), 6.0),
+    (17, 256, 272, (100,), 6.0),
+    (129, 272, 784, (1, 2, 270), 6.0),
+    (300, 1024, 528, tuple(range(0, 1024, 64)), 6.0),      # |O| = 16
+    (200, 1040, 256, tuple(range(3, 1040, 61)), 6.0),      # |O| = 17
+    (64, 256, 512, (9, 99), math.inf),                    # decomposition off
+    (40, 128, 256, (), 0.0),                               # every column out
+    (256, 4096, 256, (11, 4000), 6.0),
+]
+
+
+def _small_inputs(case, seed=0):
+    s, h, o, cols, alpha = case
+    rng = np.random.default_rng(1000 + seed + s + h + o)
+    X = workloads.random_x(rng, s, h, outlier_cols=cols, lo=6.0, hi=60.0)
+    W = workloads.random_w(rng, h, o, sigma=0.02)
+    return X, W, alpha
+
+
+def _check_quantize_rows(X, alpha):
+    Xq, ax, flags, idx, n = binding.llmint8_quantize_rows(to_dev(X), alpha)
+    torch.cuda.synchronize()
+    f_ref, idx_ref, n_ref = oracle.detect_outliers(X, alpha)
+    assert int(n.item()) == n_ref
+    assert np.array_equal(flags.cpu().numpy(), f_ref)
+    assert np.array_equal(idx.cpu().numpy()[:n_ref], idx_ref)
+    Xq_ref, ax_ref = oracle.quantize_rows(X, f_ref)
+    assert np.array_equal(ax.cpu().numpy(), ax_ref)
+    assert np.array_equal(Xq.cpu().numpy(), Xq_ref)
+    return f_ref, idx_ref
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: f"{c[0]}x{c[1]}x{c[2]}a{c[4]}")
+def test_quantize_rows_bit_exact_small(case):
+    X, _, alpha = _small_inputs(case)
+    _check_quantize_rows(X, alpha)
+
+
+def test_quantize_rows_special_rows():
+    rng = np.random.default_rng(5)
+    X = workloads.random_x(rng, 12, 256, outlier_cols=(4,), row_frac=1.0)
+    X[3] = 0                      # all-zero row: ax = 0, codes 0
+    X[5] = 0
+    X[5, 4] = 20.0                # only the outlier entry nonzero
+    X[7, 9] = np.float16(6.0)     # exactly alpha: column 9 becomes outlier
+    X[8, 10] = np.float16(5.9960938)
+    X[9, :] = np.float16(-3.0)    # constant row: all codes -127
+    X[9, 4] = 8.0
+    X[10, 11] = np.float16(127.0 / 16.0)   # tie cases of the rounding rule
+    X[10, 12:20] = (np.arange(8) * 2 + 1).astype(np.float16) / np.float16(32)
+    f, idx = _check_quantize_rows(X, 6.0)
+    assert 9 in idx.tolist() and 10 not in idx.tolist()
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: f"{c[0]}x{c[1]}x{c[2]}")
+def test_prepare_weight_bit_exact_small(case):
+    _, W, _ = _small_inputs(case)
+    W[:, 1] = 0  # a zero column
+    pw, _ = gpu_prepare(W)
+    torch.cuda.synchronize()
+    Wq_ref, aw_ref = oracle.prepare_weight(W)
+    assert np.array_equal(pw.aw.cpu().numpy(), aw_ref)
+    assert np.array_equal(pw.wq.cpu().numpy(), Wq_ref)
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: f"{c[0]}x{c[1]}x{c[2]}a{c[4]}")
+def test_matmul_small_cases(case):
+    X, W, alpha = _small_inputs(case)
+    s = X.shape[0]
+    pw, _ = gpu_prepare(W)
+    Wq_ref, aw_ref = oracle.prepare_weight(W)
+    ref, ci_ref = oracle.matmul(X, Wq_ref, aw_ref, alpha, want_ci=True)
+    paths = [1, 2] if s <= 16 else [1]
+    for path in paths:
+        out, ci, ws = gpu_matmul(X, pw, alpha, path=path, want_ci=True)
+        assert np.array_equal(ci, ci_ref), f"int32 accumulators, path {path}"
+        assert_close_fp16(out, ref, f"out path {path}")
+    # fp16 outlier tiles of the last call, bit-exact
+    f_ref, idx_ref, n_ref = oracle.detect_outliers(X, alpha)
+    n, XO, WO = binding.llmint8_read_outlier_tiles(ws)
+    assert n == n_ref
+    assert np.array_equal(XO.numpy().view(np.uint16),
+                          np.ascontiguousarray(X[:, idx_ref]).view(np.uint16))
+    WO_ref = oracle.outlier_weights(Wq_ref, aw_ref, idx_ref)
+    assert np.array_equal(WO.numpy().view(np.uint16), WO_ref.view(np.uint16))
+
+
+def test_matmul_zero_rows_and_zero_weight_columns():
+    rng = np.random.default_rng(9)
+    X = workloads.random_x(rng, 20, 256, outlier_cols=(4, 77), row_frac=1.0)
+    X[2] = 0
+    X[6] = 0
+    X[6, 4] = -9.5
+    W = workloads.random_w(rng, 256, 256)
+    W[:, 3] = 0
+    W[:, 200] = 0
+    pw, _ = gpu_prepare(W)
+    Wq_ref, aw_ref = oracle.prepare_weight(W)
+    ref, ci_ref = oracle.matmul(X, Wq_ref, aw_ref, 6.0, want_ci=True)
+    out, ci, _ = gpu_matmul(X, pw, 6.0, want_ci=True)
+    assert np.array_equal(ci, ci_ref)
+    assert_close_fp16(out, ref)
+    assert np.all(out[2] == 0) and np.all(out[:, 3] == 0)
+
+
+def test_repeated_calls_are_deterministic_and_status_stays_clear():
+    X, W, alpha = _small_inputs(SMALL[5])
+    pw, _ = gpu_prepare(W)
+    Xd = to_dev(X)
+    ws = binding.Workspace(X.shape[0], pw.h, pw.o)
+    outs = [binding.llmint8_matmul(Xd, pw, alpha, workspace=ws).cpu().numpy()
+            for _ in range(3)]
+    assert all(np.array_equal(outs[0].view(np.uint16), o.view(np.uint16))
+               for o in outs[1:])
+    assert binding.llmint8_read_device_status(ws) == 0
+
+
+def test_host_buffer_entry_point_matches_device_path():
+    X, W, alpha = _small_inputs(SMALL[4])
+    s, h = X.shape
+    pw, _ = gpu_prepare(W)
+    dev_out, _, _ = gpu_matmul(X, pw, alpha)
+    Xh = torch.from_numpy(X).pin_memory()
+    outh = torch.empty((s, pw.o), dtype=torch.float16).pin_memory()
+    ws = binding.Workspace(s, h, pw.o, host=True)
+    binding.llmint8_matmul_host(Xh, pw, alpha, outh, ws)
+    assert np.array_equal(outh.numpy().view(np.uint16), dev_out.view(np.uint16))
+
+
+def test_invalid_arguments_with_real_buffers_enqueue_nothing():
+    X, W, alpha = _small_inputs(SMALL[0])
+    pw, _ = gpu_prepare(W)
+    Xd = to_dev(X)
+    ws = binding.Workspace(16, 256, 256)
+    out = torch.zeros((16, 256), dtype=torch.float16, device="cuda")
+    with pytest.raises(binding.Llmint8Error) as e:
+        binding.llmint8_matmul(Xd, pw, -1.0, out=out, workspace=ws)
+    assert e.value.code == -7
+    small = binding.Workspace(16, 256, 256)
+    small.nbytes -= 1
+    with pytest.raises(binding.Llmint8Error) as e:
+        binding.llmint8_matmul(Xd, pw, 6.0, out=out, workspace=small)
+    assert e.value.code == -4
+    with pytest.raises(ValueError):
+        binding.llmint8_matmul(Xd[:, :240].contiguous(), pw, 6.0,
+                               out=out, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(out).item() == 0
+
+
+# ------------------------------------------------ the five OPT-shaped loads
+
+@functools.lru_cache(maxsize=1)
+def _workload(name):
+    wl, X, cols, W = workloads.make_inputs(name)
+    pw, Wd = gpu_prepare(W)
+    del Wd
+    torch.cuda.synchronize()
+    return wl, X, cols, W, pw
+
+
+@pytest.mark.parametrize("name", workloads.WORKLOAD_ORDER)
+def test_workload_quantize_rows_bit_exact(name):
+    wl, X, cols, W, pw = _workload(name)
+    f_ref, idx_ref = _check_quantize_rows(X, wl.alpha)
+    assert set(cols.tolist()) <= set(idx_ref.tolist())
+
+
+@pytest.mark.parametrize("name", workloads.WORKLOAD_ORDER)
+def test_workload_prepare_weight_bit_exact(name):
+    wl, X, cols, W, pw = _workload(name)
+    c = sample_cols(wl.o, 512) if wl.o > 4096 else None
+    Wq_ref, aw_ref = oracle_prepared(W, c)
+    wq = pw.wq.cpu().numpy()
+    aw = pw.aw.cpu().numpy()
+    if c is not None:
+        wq, aw = wq[c], aw[c]
+    assert np.array_equal(aw, aw_ref)
+    assert np.array_equal(wq, Wq_ref)
+
+
+@pytest.mark.parametrize("name", workloads.WORKLOAD_ORDER)
+def test_workload_matmul(name):
+    wl, X, cols, W, pw = _workload(name)
+    rows = sample_rows(wl.s, 48)
+    c = sample_cols(wl.o, 512)
+    Wq_ref, aw_ref = oracle_prepared(W, c)
+    ref, ci_ref = oracle.matmul(X, Wq_ref, aw_ref, wl.alpha, rows=rows,
+                                want_ci=True)
+    paths = [0, 1] if wl.s <= 16 else [0]
+    for path in paths:
+        out, ci, ws = gpu_matmul(X, pw, wl.alpha, path=path, want_ci=True)
+        assert np.array_equal(ci[np.ix_(rows, c)], ci_ref), f"Ci path {path}"
+        assert_close_fp16(out[np.ix_(rows, c)], ref, f"out path {path}")
+        # properties that hold for every output: finite, and rows with no
+        # outlier entry and zero codes are exactly zero
+        assert np.isfinite(out.astype(np.float32)).all()
