@@ -270,7 +270,7 @@ def run_ours(args, world, rank, local):
     if clocks:
         clocks.stop()
     step_ms = [a.elapsed_time(b) for a, b in zip(starts, stops)]
-    gemm_ms = [a.elapsed_time(b) for a, b in zip(g0, g1)]
+    gemm_ms = [binding.event_elapsed_ms(a, b) for a, b in zip(g0, g1)]
     ms_per_step = max_over_ranks(sum(step_ms) / K, world, dev)
     gemm_ms_avg = sum(gemm_ms) / K
     status_bits = binding.llmint8_read_device_status(ws)

@@ -213,6 +213,10 @@ def llmint8_matmul(X: torch.Tensor, w: PreparedWeight, alpha: float = 6.0,
             raise ValueError("ci must be int32 [s,o]")
         opts.ci_dev = ci.data_ptr()
     if events is not None:
+        for e in events:  # torch creates its events lazily, on first record
+            if not e.cuda_event:
+                e.record(stream if stream is not None
+                         else torch.cuda.current_stream())
         opts.gemm_event_start = events[0].cuda_event
         opts.gemm_event_stop = events[1].cuda_event
     _check("llmint8_matmul_ex", load_library().llmint8_matmul_ex(
@@ -256,6 +260,28 @@ def llmint8_read_device_status(workspace: Workspace, stream=None) -> int:
     if rc not in (OK, -6):
         _check("llmint8_read_device_status", rc)
     return bits.value
+
+
+_cudart = None
+
+
+def event_elapsed_ms(start, stop) -> float:
+    """Milliseconds between two torch.cuda.Event objects recorded by the
+    library (torch's own elapsed_time only accepts events torch recorded)."""
+    global _cudart
+    if _cudart is None:
+        cand = os.path.join(os.path.dirname(torch.__file__), "..", "nvidia",
+                            "cuda_runtime", "lib", "libcudart.so.12")
+        _cudart = ctypes.CDLL(cand if os.path.exists(cand) else "libcudart.so.12")
+        _cudart.cudaEventElapsedTime.argtypes = [ctypes.POINTER(ctypes.c_float),
+                                                 _vp, _vp]
+        _cudart.cudaEventElapsedTime.restype = ctypes.c_int
+    ms = ctypes.c_float(0.0)
+    rc = _cudart.cudaEventElapsedTime(ctypes.byref(ms), _vp(start.cuda_event),
+                                      _vp(stop.cuda_event))
+    if rc != 0:
+        raise RuntimeError(f"cudaEventElapsedTime failed ({rc})")
+    return float(ms.value)
 
 
 def effective_tops(s: int, h: int, o: int, seconds: float) -> float:
