@@ -8,7 +8,8 @@
 // evenly over one persistent CTA per SM, so every SM streams the same share
 // of the weight whatever the wave count. Each CTA adds its partial int32
 // accumulators into a [16][o] int32 buffer with integer atomics (exact and
-// order-independent), and a small finishing kernel applies the
+// order-independent; the buffer is zeroed by the call's first kernel), and a
+// small finishing kernel applies the
 // dequantisation, the fp16 outlier product and the fp16 store:
 //   out[i][j] = fp16( Ci[i][j] * (ax[i] / 16129) * aw[j] + sum_t XO[i][t] WO[t][j] )
 // ("The Full LLM.int8() Algorithm", Steps 3-5).
@@ -65,12 +66,6 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&v)
       : "memory");
 }
 
-__global__ void k_decode_zero(int32_t *__restrict__ cacc, int64_t n) {
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x)
-    cacc[i] = 0;
-}
-
 // Units [u0, u1) of this CTA: unit u is k-block (u % nk) of weight tile
 // (u / nk). Consecutive units of one tile form a segment, accumulated in one
 // TMEM buffer and then flushed by the epilogue.
@@ -124,6 +119,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  grid_dependency_wait();
 
   int64_t u0, u1;
   cta_units(p, u0, u1);
@@ -242,6 +238,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 // Dequantisation, outlier product and fp16 store for the s <= 16 rows.
 __global__ void __launch_bounds__(256) k_decode_finish(const Params p) {
+  grid_dependency_wait();
   const int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   if (g >= (int64_t)p.s * p.o) return;
   const int32_t i = (int32_t)(g / p.o);

@@ -14,10 +14,13 @@
 //   warp 1      one thread issues tcgen05.mma.kind::i8 (M=128, N=256, K=32)
 //               into a TMEM accumulator; tcgen05.commit frees ring slots
 //   warp 2      allocates / frees the 512 TMEM columns (2 accumulators)
-//   warps 4-7   epilogue: tcgen05.ld of the int32 accumulator (each warp
-//               owns 32 TMEM lanes = 32 output rows), dequantise, add the
-//               outlier product on CUDA cores, store fp16; the other
-//               accumulator is being filled by the MMA meanwhile.
+//   warps 4-7   epilogue: stage the tile's column scales and fp16 outlier
+//               rows in shared memory while the MMA runs, then tcgen05.ld
+//               the int32 accumulator (each warp owns 32 TMEM lanes = 32
+//               output rows), dequantise, add the outlier product on CUDA
+//               cores, and write fp16 through a 128B-swizzled staging block
+//               with TMA stores; the other accumulator is being filled by
+//               the MMA meanwhile.
 // Every wait is bounded by the global timer; on a timeout the CTA records a
 // status bit, drains its in-flight copies and MMAs, frees TMEM and returns.
 #pragma once
@@ -43,10 +46,20 @@ constexpr uint32_t TMEM_COLS = 512;  // NUM_ACC * BN int32 columns
 constexpr int NUM_THREADS = 256;
 constexpr int EPI_WARP0 = 4;
 constexpr int NUM_EPI_THREADS = 128;
-constexpr size_t SMEM_BYTES =
-    1024 + (size_t)STAGES * (A_STAGE_BYTES + B_STAGE_BYTES) + 256;
+constexpr int EPI_BARRIER = 1;       // named barrier of the 4 epilogue warps
+constexpr int OUT_BOX_COLS = 64;     // fp16 columns per TMA store (128 bytes)
+constexpr uint32_t OUT_STAGE_BYTES = 32 * OUT_BOX_COLS * 2;  // per epilogue warp
+constexpr int FAST_OUTLIERS = 16;    // outlier rows kept in shared memory
+constexpr uint32_t RING_BYTES = STAGES * (A_STAGE_BYTES + B_STAGE_BYTES);
+constexpr uint32_t OUT_OFF = RING_BYTES;
+constexpr uint32_t WO_OFF = OUT_OFF + 4 * OUT_STAGE_BYTES;
+constexpr uint32_t AW_OFF = WO_OFF + FAST_OUTLIERS * BN * 2;
+constexpr uint32_t BAR_OFF = AW_OFF + BN * 4;
+constexpr size_t SMEM_BYTES = 1024 + BAR_OFF + 256;
 
 static_assert(NUM_ACC * BN <= 512, "TMEM holds 512 columns");
+static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+static_assert(OUT_OFF % 1024 == 0, "swizzled staging must be 1024-byte aligned");
 
 struct Params {
   int32_t s, h, o;
@@ -56,7 +69,6 @@ struct Params {
   const uint16_t *XO;     // [s][n_out] fp16
   const uint16_t *WO;     // [n_out][o] fp16
   const int32_t *n_out;   // device scalar |O|
-  uint16_t *out;          // [s][o] fp16
   int32_t *ci;            // optional [s][o] int32
   int32_t *status;        // device status word
   uint64_t timeout_ns;
@@ -69,15 +81,15 @@ __device__ __forceinline__ uint32_t f2h2(float a, float b) {
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_gemm_i8_fused(const __grid_constant__ CUtensorMap tmA,
-                    const __grid_constant__ CUtensorMap tmB, const Params p) {
+                    const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmOut, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (raw_addr & 1023u)) & 1023u;
   uint8_t *base = smem_raw + pad;
   const uint32_t sA = smem_u32(base);
   const uint32_t sB = sA + STAGES * A_STAGE_BYTES;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(base + STAGES * (A_STAGE_BYTES + B_STAGE_BYTES));
-  // barrier indices
+  uint64_t *bars = reinterpret_cast<uint64_t *>(base + BAR_OFF);
   const uint32_t bar0 = smem_u32(bars);
   auto full_bar = [&](int st) { return bar0 + 8u * st; };
   auto empty_bar = [&](int st) { return bar0 + 8u * (STAGES + st); };
@@ -104,6 +116,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmOut);
   }
   if (warp == 2) {
     tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
@@ -113,6 +126,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // Everything above overlaps the tail of the preceding kernel when launched
+  // as a programmatic dependent; from here on its outputs are read.
+  grid_dependency_wait();
 
   const int32_t num_tiles = p.num_m_blocks * p.num_n_blocks;
 
@@ -199,19 +215,50 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp >= EPI_WARP0) {
     // --------------------------------------------------------- epilogue
     const int ew = warp - EPI_WARP0;  // TMEM lane quarter of this warp
+    const int et = threadIdx.x - EPI_WARP0 * 32;  // 0..127
     const int32_t n_out = *p.n_out;
+    const int32_t n_fast = n_out < FAST_OUTLIERS ? n_out : FAST_OUTLIERS;
+    uint16_t *sWO = reinterpret_cast<uint16_t *>(base + WO_OFF);  // [16][BN]
+    float *sAW = reinterpret_cast<float *>(base + AW_OFF);         // [BN]
+    uint8_t *sOut = base + OUT_OFF + ew * OUT_STAGE_BYTES;         // [32][128 B]
+    const uint32_t sOut_addr = smem_u32(sOut);
     int32_t it = 0;
     for (int32_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const uint32_t acc = it & 1, acc_par = (it >> 1) & 1;
-      if (!mbar_wait_bounded(tfull_bar(acc), acc_par, abort_flag, p.status,
-                             LLMINT8_DEV_TIMEOUT_EPILOGUE, p.timeout_ns))
-        break;
-      tc_fence_after();
       const int32_t m_blk = tile % p.num_m_blocks;
       const int32_t n_blk = tile / p.num_m_blocks;
+      const int32_t n0 = n_blk * BN;
+      // (1) column scales and fp16 outlier rows of this tile into shared
+      //     memory, while the MMA still works on the accumulator
+      named_barrier(EPI_BARRIER, NUM_EPI_THREADS);  // previous tile done reading
+      for (int i = et; i < BN; i += NUM_EPI_THREADS) {
+        const int32_t j = n0 + i;
+        sAW[i] = j < p.o ? __ldg(p.aw + j) : 0.0f;
+      }
+      for (int i = et; i < n_fast * (BN / 8); i += NUM_EPI_THREADS) {
+        const int t = i / (BN / 8);
+        const int c8 = (i % (BN / 8)) * 8;
+        const int32_t j = n0 + c8;
+        uint4 w8 = make_uint4(0u, 0u, 0u, 0u);
+        if (j < p.o) w8 = __ldg(reinterpret_cast<const uint4 *>(p.WO + (int64_t)t * p.o + j));
+        *reinterpret_cast<uint4 *>(sWO + t * BN + c8) = w8;
+      }
+      named_barrier(EPI_BARRIER, NUM_EPI_THREADS);
+      // (2) this thread's row: scale and outlier activations
       const int32_t row = m_blk * BM + ew * 32 + lane;
       const bool row_ok = row < p.s;
-      const float rs = row_ok ? p.ax[row] * (1.0f / 16129.0f) : 0.0f;
+      const float rs = row_ok ? __ldg(p.ax + row) * (1.0f / 16129.0f) : 0.0f;
+      float xo[FAST_OUTLIERS];
+#pragma unroll
+      for (int t = 0; t < FAST_OUTLIERS; ++t)
+        xo[t] = (t < n_fast && row_ok)
+                    ? __half2float(__ushort_as_half(p.XO[(int64_t)row * n_out + t]))
+                    : 0.0f;
+      // (3) accumulator; a timeout in any epilogue thread stops all of them
+      const bool ready = mbar_wait_bounded(tfull_bar(acc), acc_par, abort_flag, p.status,
+                                           LLMINT8_DEV_TIMEOUT_EPILOGUE, p.timeout_ns);
+      if (named_barrier_or(EPI_BARRIER, NUM_EPI_THREADS, !ready)) break;
+      tc_fence_after();
       const uint32_t t_row = tmem_base + ((uint32_t)(ew * 32) << 16) + acc * BN;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
@@ -219,47 +266,75 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         __syncwarp();
         tmem_ld_32x32b_x32(t_row + c * 32, v);
         tmem_ld_wait();
-        const int32_t j0 = n_blk * BN + c * 32;
-        if (j0 >= p.o || !row_ok) continue;  // lanes reconverge at __syncwarp
-        const bool full = (j0 + 32 <= p.o);  // else exactly 16 valid (o % 16 == 0)
+        if (c == BN / 32 - 1) {
+          // the accumulator is fully read: hand it back to the MMA warp
+          tc_fence_before();
+          mbar_arrive(tempty_bar(acc));
+        }
         float accf[32];
-        const float4 *awp = reinterpret_cast<const float4 *>(p.aw + j0);
 #pragma unroll
         for (int q4 = 0; q4 < 8; ++q4) {
-          float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (full || q4 < 4) a4 = __ldg(awp + q4);
+          const float4 a4 = *reinterpret_cast<const float4 *>(sAW + c * 32 + 4 * q4);
           accf[4 * q4 + 0] = (float)(int32_t)v[4 * q4 + 0] * rs * a4.x;
           accf[4 * q4 + 1] = (float)(int32_t)v[4 * q4 + 1] * rs * a4.y;
           accf[4 * q4 + 2] = (float)(int32_t)v[4 * q4 + 2] * rs * a4.z;
           accf[4 * q4 + 3] = (float)(int32_t)v[4 * q4 + 3] * rs * a4.w;
         }
-        const uint16_t *xo_row = p.XO + (int64_t)row * n_out;
-        for (int32_t t = 0; t < n_out; ++t) {
-          const float xo = __half2float(__ushort_as_half(xo_row[t]));
-          const uint4 *wp = reinterpret_cast<const uint4 *>(p.WO + (int64_t)t * p.o + j0);
 #pragma unroll
-          for (int q8 = 0; q8 < 4; ++q8) {
-            if (!full && q8 >= 2) break;
-            const uint4 w8 = __ldg(wp + q8);
-            const uint32_t ww[4] = {w8.x, w8.y, w8.z, w8.w};
+        for (int t = 0; t < FAST_OUTLIERS; ++t) {
+          if (t < n_fast) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&ww[e]));
-              accf[8 * q8 + 2 * e] = fmaf(xo, f.x, accf[8 * q8 + 2 * e]);
-              accf[8 * q8 + 2 * e + 1] = fmaf(xo, f.y, accf[8 * q8 + 2 * e + 1]);
+            for (int q8 = 0; q8 < 4; ++q8) {
+              const uint4 w8 = *reinterpret_cast<const uint4 *>(sWO + t * BN + c * 32 + 8 * q8);
+              const uint32_t ww[4] = {w8.x, w8.y, w8.z, w8.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&ww[e]));
+                accf[8 * q8 + 2 * e] = fmaf(xo[t], f.x, accf[8 * q8 + 2 * e]);
+                accf[8 * q8 + 2 * e + 1] = fmaf(xo[t], f.y, accf[8 * q8 + 2 * e + 1]);
+              }
             }
           }
         }
-        uint4 *op = reinterpret_cast<uint4 *>(p.out + (int64_t)row * p.o + j0);
+        // outlier columns beyond the shared-memory fast path (|O| > 16)
+        const int32_t j0 = n0 + c * 32;
+        for (int32_t t = FAST_OUTLIERS; t < n_out; ++t) {
+          const float x = row_ok ? __half2float(__ushort_as_half(p.XO[(int64_t)row * n_out + t]))
+                                 : 0.0f;
+          const uint16_t *wr = p.WO + (int64_t)t * p.o;
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            const float w = (j0 + q < p.o) ? __half2float(__ushort_as_half(wr[j0 + q])) : 0.0f;
+            accf[q] = fmaf(x, w, accf[q]);
+          }
+        }
+        // stage 32 fp16 (64 bytes) of this row into the 128B-swizzled block
+        // of 64 columns; chunk k of row r lives at 16-byte slot k ^ (r & 7)
+        const int half = c & 1;
+        if (half == 0) {
+          if (lane == 0) bulk_wait_group_read0();  // previous store has read it
+          __syncwarp();
+        }
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8) {
-          if (!full && q8 >= 2) break;
-          op[q8] = make_uint4(f2h2(accf[8 * q8 + 0], accf[8 * q8 + 1]),
-                              f2h2(accf[8 * q8 + 2], accf[8 * q8 + 3]),
-                              f2h2(accf[8 * q8 + 4], accf[8 * q8 + 5]),
-                              f2h2(accf[8 * q8 + 6], accf[8 * q8 + 7]));
+          const int chunk = half * 4 + q8;
+          const uint4 h8 = make_uint4(f2h2(accf[8 * q8 + 0], accf[8 * q8 + 1]),
+                                      f2h2(accf[8 * q8 + 2], accf[8 * q8 + 3]),
+                                      f2h2(accf[8 * q8 + 4], accf[8 * q8 + 5]),
+                                      f2h2(accf[8 * q8 + 6], accf[8 * q8 + 7]));
+          *reinterpret_cast<uint4 *>(sOut + lane * 128 + ((chunk ^ (lane & 7)) * 16)) = h8;
         }
-        if (p.ci != nullptr) {
+        if (half == 1) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          const int32_t bx = n0 + (c - 1) * 32, by = m_blk * BM + ew * 32;
+          if (lane == 0 && bx < p.o && by < p.s) {  // partial boxes are clipped by TMA
+            tma_store_2d(&tmOut, sOut_addr, bx, by);
+            bulk_commit_group();
+          }
+        }
+        if (p.ci != nullptr && row_ok && j0 < p.o) {
+          const bool full = (j0 + 32 <= p.o);
           int4 *cp = reinterpret_cast<int4 *>(p.ci + (int64_t)row * p.o + j0);
 #pragma unroll
           for (int q4 = 0; q4 < 8; ++q4) {
@@ -269,9 +344,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
-      tc_fence_before();
-      mbar_arrive(tempty_bar(acc));
     }
+    if (lane == 0) bulk_wait_group0();
   }
 
   tc_fence_before();

@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "llmint8.h"
 #include "quant_kernels.cuh"
@@ -96,6 +97,21 @@ bool make_tmap_i8(CUtensorMap *map, const void *ptr, uint64_t inner, uint64_t ro
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D fp16 tensor [rows][inner] (row stride 2*inner bytes) for TMA stores of
+// [box_rows][box_inner] blocks staged with the 128-byte swizzle.
+bool make_tmap_f16(CUtensorMap *map, void *ptr, uint64_t inner, uint64_t rows,
+                   uint32_t box_inner, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {2 * inner};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, ptr, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------ workspace layout
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -125,9 +141,10 @@ Layout layout_for(int64_t s, int64_t h, int64_t o) {
   return L;
 }
 
-// status block: [0] device status bits, [1] |O|
+// status block: [0] device status bits, [1] |O|, [2] column-pass block counter
 int32_t *status_word(void *ws) { return reinterpret_cast<int32_t *>(ws); }
 int32_t *count_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 1; }
+int32_t *block_counter_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 2; }
 
 // --------------------------------------------------------- validation
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -169,30 +186,96 @@ llmint8_status last_launch() {
   return cudaGetLastError() == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA;
 }
 
-// Steps 1 and 4 (activation side): bitmask, compaction, row scales and codes.
-// Returns the number of kernels enqueued through *launches.
-llmint8_status enqueue_activation_pass(const DeviceInfo &dev, const uint16_t *X, int64_t s,
-                                       int64_t h, float alpha, uint32_t *mask,
-                                       int32_t *wprefix, int32_t *idx, int32_t *count,
-                                       uint8_t *flags, int8_t *Xq, float *ax, uint16_t *XO,
+// Launch with programmatic stream serialization when `pdl`: the kernel may
+// be scheduled while its predecessor drains; it orders itself after the
+// predecessor with griddepcontrol.wait before touching memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                   cudaStream_t st, bool pdl, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// Steps 1, 2 and 4 (activation side, plus the fp16 outlier rows of W when
+// WO != nullptr): bitmask + compaction, then row scales, codes and outlier
+// tiles. Adds the number of kernels enqueued to *launches.
+struct ActivationArgs {
+  const uint16_t *X;
+  int64_t s, h;
+  float alpha;
+  uint32_t *mask;
+  int32_t *wprefix, *idx, *count, *block_counter;
+  uint8_t *flags;
+  int8_t *Xq;
+  float *ax;
+  uint16_t *XO;
+  const int8_t *wq;
+  const float *aw;
+  int64_t o;
+  uint16_t *WO;
+  int32_t *zero_buf;
+  int64_t zero_n;
+};
+
+template <int NV>
+cudaError_t launch_rows(const ActivationArgs &a, int64_t wo_blocks, cudaStream_t st) {
+  return launch(k_rows_and_outlier_w<NV>, dim3((unsigned)(a.s + wo_blocks)),
+                dim3(kRowRegThreads), 0, st, true, a.X, a.s, (int32_t)a.h,
+                (const uint32_t *)a.mask, (const int32_t *)a.wprefix, (const int32_t *)a.count,
+                a.Xq, a.ax, a.XO, a.wq, a.aw, (int32_t)a.o, (const int32_t *)a.idx, a.WO,
+                (int32_t)wo_blocks);
+}
+
+llmint8_status enqueue_activation_pass(const DeviceInfo &dev, const ActivationArgs &a,
                                        cudaStream_t st, int32_t *launches) {
-  const int32_t nwords = mask_words(h);
-  const int32_t hh = (int32_t)h;
-  k_reset_mask<<<(nwords + 255) / 256, 256, 0, st>>>(mask, nwords, count);
-  const int gx = (int)((h + kColsPerBlock - 1) / kColsPerBlock);
+  const int32_t nwords = mask_words(a.h);
+  const int32_t hh = (int32_t)a.h;
+  int64_t reset_threads = nwords > a.zero_n ? nwords : a.zero_n;
+  int64_t reset_blocks = (reset_threads + 255) / 256;
+  if (reset_blocks < 1) reset_blocks = 1;
+  if (reset_blocks > 4 * (int64_t)dev.sm_count) reset_blocks = 4 * (int64_t)dev.sm_count;
+  cudaError_t e = launch(k_reset_mask, dim3((unsigned)reset_blocks), dim3(256), 0, st, false,
+                         a.mask, nwords, a.count, a.block_counter, a.zero_buf, a.zero_n);
+  if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+  const int gx = (int)((a.h + kColsPerBlock - 1) / kColsPerBlock);
   const int64_t want_blocks = 4 * (int64_t)dev.sm_count;
   int64_t gy_target = (want_blocks + gx - 1) / gx;
-  int64_t rpb = (s + gy_target - 1) / gy_target;
-  if (rpb < 4) rpb = 4;
-  if ((s + rpb - 1) / rpb > 65535) rpb = (s + 65534) / 65535;
-  const int gy = (int)((s + rpb - 1) / rpb);
-  k_outlier_columns<<<dim3(gx, gy), kColThreads, 0, st>>>(X, s, hh, threshold_bits(alpha),
-                                                         (int32_t)rpb, mask);
-  k_compact_outliers<<<1, kCompactThreads, 0, st>>>(mask, nwords, hh, wprefix, idx, count, flags);
-  const int64_t rb = (s + kRowsPerBlock - 1) / kRowsPerBlock;
-  k_quantize_rows<<<(unsigned)rb, kRowThreads, 0, st>>>(X, s, hh, mask, wprefix, count, Xq, ax,
-                                                       XO);
-  *launches += 4;
+  int64_t rpb = (a.s + gy_target - 1) / gy_target;
+  if (rpb < 8) rpb = 8;
+  if ((a.s + rpb - 1) / rpb > 65535) rpb = (a.s + 65534) / 65535;
+  const int gy = (int)((a.s + rpb - 1) / rpb);
+  e = launch(k_outlier_columns, dim3(gx, gy), dim3(kColThreads), 0, st, true, a.X, a.s, hh,
+             threshold_bits(a.alpha), (int32_t)rpb, a.mask, a.count, a.block_counter, a.wprefix,
+             a.idx, a.flags);
+  if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+  const int64_t nv = (a.h + 1023) / 1024;
+  const int64_t wo_blocks_reg = a.WO ? (a.o + kRowRegThreads - 1) / kRowRegThreads : 0;
+  if (nv <= 16 && a.s + wo_blocks_reg <= (int64_t)INT32_MAX) {
+    if (nv <= 1) e = launch_rows<1>(a, wo_blocks_reg, st);
+    else if (nv <= 2) e = launch_rows<2>(a, wo_blocks_reg, st);
+    else if (nv <= 4) e = launch_rows<4>(a, wo_blocks_reg, st);
+    else if (nv <= 8) e = launch_rows<8>(a, wo_blocks_reg, st);
+    else if (nv <= 12) e = launch_rows<12>(a, wo_blocks_reg, st);
+    else e = launch_rows<16>(a, wo_blocks_reg, st);
+  } else {
+    const int64_t rb = (a.s + kRowsPerBlock - 1) / kRowsPerBlock;
+    const int64_t wob = a.WO ? (a.o + kRowThreads - 1) / kRowThreads : 0;
+    e = launch(k_rows_and_outlier_w_any, dim3((unsigned)(rb + wob)), dim3(kRowThreads), 0, st,
+               true, a.X, a.s, hh, (const uint32_t *)a.mask, (const int32_t *)a.wprefix,
+               (const int32_t *)a.count, a.Xq, a.ax, a.XO, a.wq, a.aw, (int32_t)a.o,
+               (const int32_t *)a.idx, a.WO, (int32_t)wob);
+  }
+  if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+  *launches += 3;
   return last_launch();
 }
 
@@ -239,7 +322,7 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
   const bool use_decode = (path == 2) || (path == 0 && s <= kDecodeMaxRows);
 
   // Tensor maps first: a failure here must leave nothing enqueued.
-  CUtensorMap tmA, tmB;
+  CUtensorMap tmA, tmB, tmOut;
   if (use_decode) {
     // A = Wq tiles (rows of o), B = Xq rows (s <= 16, zero-filled to 16)
     if (!make_tmap_i8(&tmA, w->wq_dev, (uint64_t)h, (uint64_t)o, decode::BK, decode::BM) ||
@@ -247,20 +330,37 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
       return LLMINT8_ERR_CUDA;
   } else {
     if (!make_tmap_i8(&tmA, xq, (uint64_t)h, (uint64_t)s, gemm::BK, gemm::BM) ||
-        !make_tmap_i8(&tmB, w->wq_dev, (uint64_t)h, (uint64_t)o, gemm::BK, gemm::BN))
+        !make_tmap_i8(&tmB, w->wq_dev, (uint64_t)h, (uint64_t)o, gemm::BK, gemm::BN) ||
+        !make_tmap_f16(&tmOut, out, (uint64_t)o, (uint64_t)s, gemm::OUT_BOX_COLS, 32))
       return LLMINT8_ERR_CUDA;
   }
 
   int32_t launches = 0;
-  if ((rc = enqueue_activation_pass(*dev, X, s, h, alpha, mask, wprefix, idx, count, nullptr, xq,
-                                    ax, xo, st, &launches)))
-    return rc;
-  {
-    dim3 grid((unsigned)((o + 255) / 256), 8);
-    k_outlier_weights<<<grid, 256, 0, st>>>(w->wq_dev, w->aw_dev, (int32_t)h, (int32_t)o, idx,
-                                           count, wo);
-    ++launches;
-  }
+  ActivationArgs act;
+  act.X = X;
+  act.s = s;
+  act.h = h;
+  act.alpha = alpha;
+  act.mask = mask;
+  act.wprefix = wprefix;
+  act.idx = idx;
+  act.count = count;
+  act.block_counter = block_counter_word(ws);
+  act.flags = nullptr;
+  act.Xq = xq;
+  act.ax = ax;
+  act.XO = xo;
+  act.wq = w->wq_dev;
+  act.aw = w->aw_dev;
+  act.o = o;
+  act.WO = wo;
+  act.zero_buf = use_decode ? cacc : nullptr;
+  act.zero_n = use_decode ? (int64_t)kDecodeMaxRows * o : 0;
+  if ((rc = enqueue_activation_pass(*dev, act, st, &launches))) return rc;
+  const bool timed = opts && (opts->gemm_event_start || opts->gemm_event_stop);
+  if (opts && opts->gemm_event_start)
+    cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->gemm_event_start), st);
+  cudaError_t e;
   if (use_decode) {
     decode::Params p;
     p.s = (int32_t)s;
@@ -282,17 +382,15 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
     int grid = dev->sm_count;
     if (total_units < grid) grid = (int)total_units;
     p.units_total = total_units;
-    decode::k_decode_zero<<<(unsigned)((kDecodeMaxRows * o + 1023) / 1024), 256, 0, st>>>(
-        cacc, (int64_t)kDecodeMaxRows * o);
-    ++launches;
-    if (opts && opts->gemm_event_start)
-      cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->gemm_event_start), st);
-    decode::k_decode_i8<<<grid, decode::NUM_THREADS, decode::SMEM_BYTES, st>>>(tmA, tmB, p);
+    e = launch(decode::k_decode_i8, dim3(grid), dim3(decode::NUM_THREADS), decode::SMEM_BYTES, st,
+               !timed, tmA, tmB, p);
+    if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
     if (opts && opts->gemm_event_stop)
       cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->gemm_event_stop), st);
-    ++launches;
-    decode::k_decode_finish<<<(unsigned)((s * o + 255) / 256), 256, 0, st>>>(p);
-    ++launches;
+    e = launch(decode::k_decode_finish, dim3((unsigned)((s * o + 255) / 256)), dim3(256), 0, st,
+               !timed, p);
+    if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+    launches += 2;
   } else {
     gemm::Params p;
     p.s = (int32_t)s;
@@ -306,15 +404,14 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
     p.XO = xo;
     p.WO = wo;
     p.n_out = count;
-    p.out = out;
     p.ci = opts ? opts->ci_dev : nullptr;
     p.status = status;
     p.timeout_ns = kTimeoutNs;
     const int64_t tiles = (int64_t)p.num_m_blocks * p.num_n_blocks;
     const int grid = (int)(tiles < dev->sm_count ? tiles : dev->sm_count);
-    if (opts && opts->gemm_event_start)
-      cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->gemm_event_start), st);
-    gemm::k_gemm_i8_fused<<<grid, gemm::NUM_THREADS, gemm::SMEM_BYTES, st>>>(tmA, tmB, p);
+    e = launch(gemm::k_gemm_i8_fused, dim3(grid), dim3(gemm::NUM_THREADS), gemm::SMEM_BYTES, st,
+               !timed, tmA, tmB, tmOut, p);
+    if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
     if (opts && opts->gemm_event_stop)
       cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->gemm_event_stop), st);
     ++launches;
@@ -391,7 +488,7 @@ llmint8_status llmint8_prepare_weight(const uint16_t *W_dev, int64_t h, int64_t 
 
 size_t llmint8_quantize_rows_scratch_size(int64_t h) {
   if (h < 0) return 0;
-  return align256(4 * (size_t)mask_words(h)) + align256(4 * ((size_t)mask_words(h) + 1));
+  return 256 + align256(4 * (size_t)mask_words(h)) + align256(4 * ((size_t)mask_words(h) + 1));
 }
 
 llmint8_status llmint8_quantize_rows(const uint16_t *X_dev, int64_t s, int64_t h, float alpha,
@@ -411,11 +508,21 @@ llmint8_status llmint8_quantize_rows(const uint16_t *X_dev, int64_t s, int64_t h
   DeviceInfo *dev = nullptr;
   if ((rc = device_info(&dev))) return rc;
   uint8_t *sb = static_cast<uint8_t *>(scratch_dev);
-  uint32_t *mask = reinterpret_cast<uint32_t *>(sb);
-  int32_t *wprefix = reinterpret_cast<int32_t *>(sb + align256(4 * (size_t)mask_words(h)));
+  ActivationArgs act = {};
+  act.X = X_dev;
+  act.s = s;
+  act.h = h;
+  act.alpha = alpha;
+  act.block_counter = reinterpret_cast<int32_t *>(sb);
+  act.mask = reinterpret_cast<uint32_t *>(sb + 256);
+  act.wprefix = reinterpret_cast<int32_t *>(sb + 256 + align256(4 * (size_t)mask_words(h)));
+  act.idx = idx_dev;
+  act.count = n_outliers_dev;
+  act.flags = flags_dev;
+  act.Xq = Xq_dev;
+  act.ax = ax_dev;
   int32_t launches = 0;
-  return enqueue_activation_pass(*dev, X_dev, s, h, alpha, mask, wprefix, idx_dev, n_outliers_dev,
-                                 flags_dev, Xq_dev, ax_dev, nullptr, as_stream(stream), &launches);
+  return enqueue_activation_pass(*dev, act, as_stream(stream), &launches);
 }
 
 llmint8_status llmint8_matmul(const uint16_t *X_dev, int64_t s, const llmint8_weight *w,
