@@ -151,21 +151,30 @@ class ClockSampler:
 
 # ------------------------------------------------------------ CPU oracle
 
-def cpu_oracle_run(wl, X, Wq, aw, budget_s: float, max_rows: int = None):
-    """Time the oracle on a row sample sized to ~budget_s seconds."""
+def cpu_oracle_run(wl, X, Wq, aw, budget_s: float):
+    """Time the oracle on a row sample sized to about budget_s seconds.
+
+    The sample is grown by 4x until a run takes a quarter of the budget (the
+    outlier set is always computed over all rows, a fixed cost), then scaled
+    to the budget and timed once more."""
     import oracle
     rng = np.random.default_rng(123)
-    probe_rows = np.sort(rng.choice(wl.s, size=min(wl.s, 2), replace=False))
-    t = time.perf_counter()
-    oracle.matmul(X, Wq, aw, wl.alpha, rows=probe_rows)
-    dt = max(time.perf_counter() - t, 1e-4) / len(probe_rows)
-    n = int(max(1, min(wl.s, budget_s / dt)))
-    if max_rows:
-        n = min(n, max_rows)
-    rows = np.sort(rng.choice(wl.s, size=n, replace=False))
-    t = time.perf_counter()
-    oracle.matmul(X, Wq, aw, wl.alpha, rows=rows)
-    el = time.perf_counter() - t
+    order = rng.permutation(wl.s)
+
+    def timed(n):
+        rows = np.sort(order[:n])
+        t = time.perf_counter()
+        oracle.matmul(X, Wq, aw, wl.alpha, rows=rows)
+        return time.perf_counter() - t
+
+    n = min(wl.s, 4)
+    el = timed(n)
+    while el < budget_s / 4 and n < wl.s:
+        n = min(wl.s, n * 4)
+        el = timed(n)
+    n_final = int(max(1, min(wl.s, n * budget_s / max(el, 1e-6))))
+    if n_final != n:
+        n, el = n_final, timed(n_final)
     tops = 2.0 * n * wl.h * wl.o / el / 1e12
     return {"value": tops, "unit": UNIT, "cores": oracle.num_threads(),
             "kind": "oracle",
