@@ -72,7 +72,8 @@ typedef enum {
     LLMINT8_ERR_CUDA = -5,          /* a CUDA runtime/driver call failed */
     LLMINT8_ERR_DEVICE_STATUS = -6, /* a kernel flagged an anomaly */
     LLMINT8_ERR_ARG = -7,           /* a scalar argument is invalid */
-    LLMINT8_ERR_UNSUPPORTED = -8    /* current device is not sm_100 */
+    LLMINT8_ERR_UNSUPPORTED = -8,   /* current device is not sm_100 */
+    LLMINT8_ERR_TOO_LARGE = -9      /* problem exceeds the no-alloc scratch */
 } llmint8_status;
 
 /* Bits of the device status word (llmint8_read_device_status). */
@@ -199,6 +200,34 @@ LLMINT8_API llmint8_status llmint8_read_outlier_tiles(const void *ws_dev, size_t
  * set (bits also stored in *bits_out when non-NULL), else LLMINT8_OK. */
 LLMINT8_API llmint8_status llmint8_read_device_status(void *ws_dev, size_t ws_bytes,
                                           int32_t *bits_out, void *stream);
+
+/* Allocation-free form of llmint8_matmul (the pages have no counterpart: it
+ * is a deployment convenience, not part of the method).
+ *
+ * Some callers cannot give the library a device workspace: they run where
+ * device allocation is not allowed or not possible at call time, e.g. an
+ * operator invoked from inside another runtime's execution callback whose
+ * memory plan is fixed, or a host program with no allocator of its own for
+ * scratch buffers. For them this entry point takes only the inputs and the
+ * output and uses instead a scratch buffer that lives inside the library: a
+ * static device array of LLMINT8_NOALLOC_MAX_SCRATCH_BYTES bytes, which every
+ * GPU that loads the library keeps reserved until the process exits.
+ *
+ * - It accepts the problems whose workspace, llmint8_workspace_size(s, h, o),
+ *   fits that maximum and returns LLMINT8_ERR_TOO_LARGE for the others.
+ * - It never calls cudaMalloc/cudaFree or any allocating routine.
+ * - The first call on a device looks up the array's device address with that
+ *   device current and clears the array's status block; make that first call
+ *   before any stream capture on that device.
+ * - Every call on a device shares the one array and leaves its contents
+ *   behind for the next call (each call resets what it needs). Calls whose
+ *   execution can overlap on the GPU (other streams, other host threads)
+ *   race on it and must be serialised by the caller.
+ * Results equal llmint8_matmul's for the same inputs. */
+#define LLMINT8_NOALLOC_MAX_SCRATCH_BYTES (64ull << 20)
+LLMINT8_API llmint8_status llmint8_matmul_noalloc(const uint16_t *X_dev, int64_t s,
+                                                  const llmint8_weight *w, float alpha,
+                                                  uint16_t *out_dev, void *stream);
 
 /* Largest s the decode kernel accepts. */
 LLMINT8_API int64_t llmint8_decode_max_rows(void);

@@ -21,7 +21,8 @@ LIB_PATH = os.path.join(_HERE, "libllmint8.so")
 OK = 0
 STATUS_NAMES = {0: "OK", -1: "ERR_NULL", -2: "ERR_SHAPE", -3: "ERR_ALIGN",
                 -4: "ERR_WORKSPACE", -5: "ERR_CUDA", -6: "ERR_DEVICE_STATUS",
-                -7: "ERR_ARG", -8: "ERR_UNSUPPORTED"}
+                -7: "ERR_ARG", -8: "ERR_UNSUPPORTED", -9: "ERR_TOO_LARGE"}
+NOALLOC_MAX_SCRATCH_BYTES = 64 << 20  # LLMINT8_NOALLOC_MAX_SCRATCH_BYTES
 
 _c_i64, _c_i32, _c_f32 = ctypes.c_int64, ctypes.c_int32, ctypes.c_float
 _vp, _sz = ctypes.c_void_p, ctypes.c_size_t
@@ -77,6 +78,8 @@ def load_library():
                                         _vp, _vp, _vp], _c_i32),
         "llmint8_read_device_status": ([_vp, _sz, _vp, _vp], _c_i32),
         "llmint8_decode_max_rows": ([], _c_i64),
+        "llmint8_matmul_noalloc": ([_vp, _c_i64, ctypes.POINTER(llmint8_weight),
+                                    _c_f32, _vp, _vp], _c_i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -91,7 +94,8 @@ EXPORTED = ("llmint8_status_string", "llmint8_workspace_size",
             "llmint8_prepare_weight", "llmint8_quantize_rows_scratch_size",
             "llmint8_quantize_rows", "llmint8_matmul", "llmint8_matmul_ex",
             "llmint8_matmul_host", "llmint8_read_outlier_tiles",
-            "llmint8_read_device_status", "llmint8_decode_max_rows")
+            "llmint8_read_device_status", "llmint8_decode_max_rows",
+            "llmint8_matmul_noalloc")
 
 
 def status_string(code: int) -> str:
@@ -224,6 +228,25 @@ def llmint8_matmul(X: torch.Tensor, w: PreparedWeight, alpha: float = 6.0,
         _ptr(workspace.buf), workspace.nbytes, ctypes.byref(opts),
         _stream(stream)))
     llmint8_matmul.last_launches = int(opts.launches)
+    return out
+
+
+def llmint8_matmul_noalloc(X: torch.Tensor, w: PreparedWeight,
+                           alpha: float = 6.0,
+                           out: Optional[torch.Tensor] = None,
+                           stream=None) -> torch.Tensor:
+    """llmint8_matmul without a caller workspace: the library's own static
+    device scratch is used instead (see include/llmint8.h for who needs this
+    and its limits). Only `out` may be allocated here, by torch, when it is
+    not given."""
+    _f16_dev(X, "X")
+    s, h = X.shape
+    if h != w.h:
+        raise ValueError(f"X has h={h}, weight has h={w.h}")
+    if out is None:
+        out = torch.empty((s, w.o), dtype=torch.float16, device=X.device)
+    _check("llmint8_matmul_noalloc", load_library().llmint8_matmul_noalloc(
+        _ptr(X), s, ctypes.byref(w.c), float(alpha), _ptr(out), _stream(stream)))
     return out
 
 

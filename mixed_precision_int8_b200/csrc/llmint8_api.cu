@@ -435,6 +435,8 @@ const char *llmint8_status_string(llmint8_status st) {
     case LLMINT8_ERR_DEVICE_STATUS: return "a kernel flagged an anomaly";
     case LLMINT8_ERR_ARG: return "invalid scalar argument";
     case LLMINT8_ERR_UNSUPPORTED: return "current device is not sm_100";
+    case LLMINT8_ERR_TOO_LARGE:
+      return "problem needs more scratch than the no-alloc entry point holds";
   }
   return "unknown status";
 }
@@ -604,3 +606,61 @@ llmint8_status llmint8_read_device_status(void *ws_dev, size_t ws_bytes, int32_t
 }
 
 }  // extern "C"
+
+// ----------------------------------------------------------------------------
+// Allocation-free entry point: llmint8_matmul on a scratch buffer that is a
+// static device array of this library, for callers that cannot allocate
+// device memory or hand over a workspace at call time.
+// ----------------------------------------------------------------------------
+static __device__ __align__(256) uint8_t g_noalloc_scratch[LLMINT8_NOALLOC_MAX_SCRATCH_BYTES];
+
+namespace {
+
+struct NoAllocSlot {
+  bool ready = false;
+  void *ptr = nullptr;  // device address of g_noalloc_scratch on that device
+};
+NoAllocSlot g_noalloc[kMaxDevices];
+std::mutex g_noalloc_mutex;
+
+// Device address of the scratch array on the current device. In host code
+// the array's name is only a host-side stand-in, so the address is asked of
+// the runtime once per device (with that device current) and cached. The
+// first lookup also clears the status block, asynchronously on `st`.
+llmint8_status noalloc_scratch(cudaStream_t st, void **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return LLMINT8_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  NoAllocSlot &slot = g_noalloc[dev];
+  if (!slot.ready) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return LLMINT8_ERR_CUDA;
+    if (cudaMemsetAsync(p, 0, 256, st) != cudaSuccess) return LLMINT8_ERR_CUDA;
+    slot.ptr = p;
+    slot.ready = true;
+  }
+  *out = slot.ptr;
+  return LLMINT8_OK;
+}
+
+}  // namespace
+
+extern "C" llmint8_status llmint8_matmul_noalloc(const uint16_t *X_dev, int64_t s,
+                                                 const llmint8_weight *w, float alpha,
+                                                 uint16_t *out_dev, void *stream) {
+  llmint8_status rc = validate_weight(w);
+  if (rc) return rc;
+  if (s < 0 || s > (int64_t)INT32_MAX) return LLMINT8_ERR_SHAPE;
+  if (layout_for(s, w->h, w->o).end > (size_t)LLMINT8_NOALLOC_MAX_SCRATCH_BYTES)
+    return LLMINT8_ERR_TOO_LARGE;
+  if (s == 0) return llmint8_matmul(X_dev, s, w, alpha, out_dev, nullptr, 0, stream);
+  DeviceInfo *dev = nullptr;
+  if ((rc = device_info(&dev))) return rc;
+  cudaStream_t st = as_stream(stream);
+  void *ws = nullptr;
+  if ((rc = noalloc_scratch(st, &ws))) return rc;
+  return matmul_impl(X_dev, s, w, alpha, out_dev, ws, (size_t)LLMINT8_NOALLOC_MAX_SCRATCH_BYTES,
+                     nullptr, st, false);
+}

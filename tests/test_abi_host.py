@@ -158,6 +158,17 @@ def test_prepare_and_quantize_rows_validation(lib):
 
 
 @needs_no_gpu
+def test_noalloc_size_limit_is_checked_on_the_host(lib):
+    s, h, o = 16, 4096, 8192
+    assert lib.llmint8_workspace_size(s, h, o) > binding.NOALLOC_MAX_SCRATCH_BYTES
+    w = _weight(h, o)
+    assert lib.llmint8_matmul_noalloc(FAKE, s, ctypes.byref(w), 6.0, FAKE,
+                                      None) == -9
+    assert lib.llmint8_matmul_noalloc(FAKE, s, ctypes.byref(_weight(h, 24)),
+                                      6.0, FAKE, None) == -2
+
+
+@needs_no_gpu
 def test_valid_call_without_a_gpu_reports_cuda_error_not_a_fallback(lib):
     # Arguments pass validation; with no device the library must fail, never
     # compute on the host.
