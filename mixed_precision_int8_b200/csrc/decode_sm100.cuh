@@ -7,12 +7,19 @@
 // zero-filled by TMA beyond s). The (weight tile, k-block) units are split
 // evenly over one persistent CTA per SM, so every SM streams the same share
 // of the weight whatever the wave count. Each CTA adds its partial int32
-// accumulators into a [16][o] int32 buffer with integer atomics (exact and
-// order-independent; the buffer is zeroed by the call's first kernel), and a
-// small finishing kernel applies the
-// dequantisation, the fp16 outlier product and the fp16 store:
-//   out[i][j] = fp16( Ci[i][j] * (ax[i] / 16129) * aw[j] + sum_t XO[i][t] WO[t][j] )
-// ("The Full LLM.int8() Algorithm", Steps 3-5).
+// accumulators into a [s][o] int32 buffer with integer atomics (exact and
+// order-independent; the buffer is zeroed by the call's first kernel).
+//
+// The rest of the layer is folded into the same kernel:
+//  - the fp16 outlier weight rows WO[t][j] = fp16(fp32(fp32(wq[j][O_t]) *
+//    aw[j]) / 127) are read out of the weight tiles already streaming through
+//    shared memory (the MMA warp reads a stage whose k-block holds an
+//    outlier column before its commit releases the stage), so the column
+//    gather costs no HBM traffic;
+//  - the last CTA to finish a tile (an atomic arrival count; nobody waits)
+//    applies the dequantisation, the fp16 outlier product and the store:
+//      out[i][j] = fp16( Ci[i][j] * (ax[i] / 16129) * aw[j] + sum_t XO[i][t] WO[t][j] )
+// ("The Full LLM.int8() Algorithm", Steps 2-5).
 #pragma once
 
 #include <cstdint>
@@ -25,19 +32,38 @@ namespace llmint8 {
 namespace decode {
 
 constexpr int MAX_ROWS = 16;
-constexpr int BM = 128;  // weight rows (output columns) per tile: MMA M
-constexpr int BN = 16;   // X rows, zero-padded: MMA N
-constexpr int BK = 128;  // reduction bytes per stage
-constexpr int STAGES = 10;
+constexpr int BM = 128;   // weight rows (output columns) per tile: MMA M
+constexpr int BN = 16;    // X rows, zero-padded: MMA N
+constexpr int BOX_K = 128;  // reduction bytes of one TMA box (one 128B swizzle row)
+constexpr int SUB = 2;      // boxes per stage
+constexpr int BK = BOX_K * SUB;  // reduction bytes per stage
+constexpr int STAGES = 5;
 constexpr int UMMA_K = 32;
-constexpr uint32_t A_STAGE_BYTES = BM * BK;  // 16 KB
-constexpr uint32_t B_STAGE_BYTES = BN * BK;  // 2 KB
+constexpr uint32_t A_BOX_BYTES = BM * BOX_K;   // 16 KB
+constexpr uint32_t B_BOX_BYTES = BN * BOX_K;   // 2 KB
+constexpr uint32_t A_STAGE_BYTES = A_BOX_BYTES * SUB;
+constexpr uint32_t B_STAGE_BYTES = B_BOX_BYTES * SUB;
 constexpr int NUM_ACC = 2;
 constexpr uint32_t TMEM_COLS = 32;
 constexpr int NUM_THREADS = 256;
 constexpr int EPI_WARP0 = 4;
 constexpr int NUM_EPI_THREADS = 128;
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * (A_STAGE_BYTES + B_STAGE_BYTES) + 256;
+constexpr int MAX_MASK_WORDS = (133144 + 31) / 32;  // h <= 133144
+constexpr uint32_t RING_BYTES = STAGES * (A_STAGE_BYTES + B_STAGE_BYTES);
+constexpr int MAX_KB_WORDS = (MAX_MASK_WORDS * 32 / BK + 31) / 32 + 1;
+static_assert(BK % 32 == 0 && (BK / 32) <= 32, "mask words per k-block");
+// outlier bitmask words, their prefix counts, then one bit per k-block that
+// holds an outlier column
+constexpr uint32_t MASK_OFF = RING_BYTES;
+constexpr uint32_t KB_OFF = MASK_OFF + 4 * (2 * MAX_MASK_WORDS + 1);
+// mbarriers need 8-byte alignment; start them on a 128-byte boundary
+constexpr uint32_t BAR_OFF = (KB_OFF + 4 * MAX_KB_WORDS + 127) & ~127u;
+constexpr size_t SMEM_BYTES = 1024 + BAR_OFF + 256;
+static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+static_assert(BAR_OFF % 8 == 0, "mbarrier alignment");
+static_assert((2 * STAGES + 2 * NUM_ACC + 1) * 8 + 12 <= 256, "barrier block size");
+
+constexpr int EPI_BARRIER = 1;
 
 struct Params {
   int32_t s, h, o;
@@ -45,15 +71,30 @@ struct Params {
   int64_t units_total;
   const float *ax;
   const float *aw;
-  const uint16_t *XO;
-  const uint16_t *WO;
+  const uint32_t *mask;   // outlier-column bitmask [ceil(h/32)]
+  const int32_t *word_prefix;  // outlier columns before each mask word
+  const uint16_t *XO;     // [s][n_out] fp16
+  uint16_t *WO;           // [n_out][o] fp16, written here
   const int32_t *n_out;
   uint16_t *out;
-  int32_t *ci;    // optional exact accumulators [s][o]
-  int32_t *cacc;  // [MAX_ROWS][o] int32 partial-sum buffer
+  int32_t *ci;            // optional exact accumulators [s][o]
+  int32_t *cacc;          // [s][o] int32 partial sums (zeroed before the launch)
+  int32_t *tile_count;    // [num_m_blocks] arrivals (zeroed before the launch)
   int32_t *status;
   uint64_t timeout_ns;
 };
+
+// Generic pointer to shared-memory address `saddr` + stage offset.
+__device__ __forceinline__ const void *base_ptr_of(uint32_t sA, uint32_t stage) {
+  extern __shared__ uint8_t smem_raw[];
+  return smem_raw + (sA - smem_u32(smem_raw)) + stage * A_STAGE_BYTES;
+}
+
+// Index of the CTA whose unit range contains unit u (inverse of cta_units).
+__device__ __forceinline__ int64_t cta_of_unit(const Params &p, int64_t u) {
+  const int64_t G = gridDim.x;
+  return (G * (u + 1) + p.units_total - 1) / p.units_total - 1;
+}
 
 __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&v)[16]) {
   asm volatile(
@@ -83,7 +124,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t *base = smem_raw + pad;
   const uint32_t sA = smem_u32(base);
   const uint32_t sB = sA + STAGES * A_STAGE_BYTES;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(base + STAGES * (A_STAGE_BYTES + B_STAGE_BYTES));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(base + BAR_OFF);
+  uint32_t *s_mask = reinterpret_cast<uint32_t *>(base + MASK_OFF);
+  int32_t *s_prefix = reinterpret_cast<int32_t *>(s_mask + MAX_MASK_WORDS);
+  uint32_t *s_kb = reinterpret_cast<uint32_t *>(base + KB_OFF);
   const uint32_t bar0 = smem_u32(bars);
   auto full_bar = [&](int st) { return bar0 + 8u * st; };
   auto empty_bar = [&](int st) { return bar0 + 8u * (STAGES + st); };
@@ -92,6 +136,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 2 * NUM_ACC);
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 2 * NUM_ACC + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+  // segments whose outlier weight rows the MMA warp has published (monotonic)
+  volatile int *wo_segments = reinterpret_cast<volatile int *>(tmem_holder + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -101,6 +147,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(full_bar(i), 1);
       mbar_init(empty_bar(i), 1);
     }
+    *wo_segments = 0;
     for (int a = 0; a < NUM_ACC; ++a) {
       mbar_init(tfull_bar(a), 1);
       mbar_init(tempty_bar(a), NUM_EPI_THREADS);
@@ -139,9 +186,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         break;
       }
       mbar_arrive_expect_tx(full_bar(stage), A_STAGE_BYTES + B_STAGE_BYTES);
-      tma_load_2d_hint(sA + stage * A_STAGE_BYTES, &tmA, full_bar(stage), kb * BK, m_blk * BM,
-                       pol_w);
-      tma_load_2d(sB + stage * B_STAGE_BYTES, &tmB, full_bar(stage), kb * BK, 0);
+#pragma unroll
+      for (int b = 0; b < SUB; ++b) {
+        tma_load_2d_hint(sA + stage * A_STAGE_BYTES + b * A_BOX_BYTES, &tmA, full_bar(stage),
+                         kb * BK + b * BOX_K, m_blk * BM, pol_w);
+        tma_load_2d(sB + stage * B_STAGE_BYTES + b * B_BOX_BYTES, &tmB, full_bar(stage),
+                    kb * BK + b * BOX_K, 0);
+      }
       issued |= 1u << stage;
       last_par = (last_par & ~(1u << stage)) | (phase << stage);
       if (++stage == STAGES) {
@@ -156,48 +207,140 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           mbar_wait_bounded(full_bar(st), (last_par >> st) & 1u, &never, p.status,
                             LLMINT8_DEV_TIMEOUT_DRAIN, p.timeout_ns);
     }
-  } else if (warp == 1 && lane == 0) {
-    // ------------------------------------------------------- MMA issuer
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer (lane 0)
+    // The whole warp also reads the fp16 outlier weight rows out of stages
+    // whose k-block holds an outlier column: for column c of the k-block,
+    // row r of the 128B-swizzled box holds wq[j][c] in 16-byte chunk
+    // ((c - k0) / 16) ^ (r % 8). The reads finish before lane 0's commit
+    // releases the stage (a stage holds SUB boxes of BOX_K columns; column c
+    // of the stage lives in box c / BOX_K). Which k-blocks hold outlier columns is the same
+    // for every tile, so a per-k-block bitmap is built once and the next
+    // such k-block is kept in a register: an ordinary stage costs one
+    // compare. After each segment the rows are published (fence) by bumping
+    // wo_segments.
     constexpr uint32_t idesc = idesc_i8_s32(BM, BN);
+    const int32_t n_out = *p.n_out;
+    const int32_t nwords = (p.h + 31) >> 5;
+    const int32_t kb_words = (int32_t)((nk + 31) >> 5);
+    for (int32_t w = lane; w < nwords; w += 32) {
+      s_mask[w] = __ldg(p.mask + w);
+      s_prefix[w] = __ldg(p.word_prefix + w);
+    }
+    __syncwarp();
+    for (int32_t kw = 0; kw < kb_words; ++kw) {
+      const int32_t kb = kw * 32 + lane;
+      bool has = false;
+      if (kb < nk)
+        for (int32_t w = kb * (BK / 32); w < min(nwords, (kb + 1) * (BK / 32)); ++w)
+          has |= s_mask[w] != 0u;
+      const uint32_t word = __ballot_sync(0xFFFFFFFFu, has);
+      if (lane == 0) s_kb[kw] = word;
+    }
+    __syncwarp();
+    // first k-block >= kb holding an outlier column (nk if none)
+    auto next_outlier_kb = [&](int32_t kb) -> int32_t {
+      if (n_out == 0) return (int32_t)nk;
+      for (int32_t kw = kb >> 5; kw < kb_words; ++kw) {
+        uint32_t m = s_kb[kw];
+        if (kw == (kb >> 5)) m &= ~0u << (kb & 31);
+        if (m) return kw * 32 + __ffs(m) - 1;
+      }
+      return (int32_t)nk;
+    };
     uint32_t stage = 0, phase = 0;
     bool ok = true, any = false;
     int32_t it = 0;
+    float aw_rows[BM / 32];  // column scales of this lane's 4 tile rows
     for (int64_t u = u0; u < u1 && ok; ++it) {
       const int64_t m_blk = u / nk;
       const int64_t seg_end = min(u1, (m_blk + 1) * nk);
       const uint32_t acc = it & 1, acc_par = (it >> 1) & 1;
-      if (!mbar_wait_bounded(tempty_bar(acc), acc_par ^ 1u, abort_flag, p.status,
-                             LLMINT8_DEV_TIMEOUT_MMA, p.timeout_ns)) {
+      int32_t next_kb = next_outlier_kb((int32_t)(u - m_blk * nk));
+#pragma unroll
+      for (int q = 0; q < BM / 32; ++q) {
+        const int64_t j = m_blk * BM + lane + 32 * q;
+        aw_rows[q] = (n_out > 0 && j < p.o) ? __ldg(p.aw + j) : 0.0f;
+      }
+      // every lane waits; a vote keeps the warp's decision uniform
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(tempty_bar(acc), acc_par ^ 1u, abort_flag,
+                                                     p.status, LLMINT8_DEV_TIMEOUT_MMA,
+                                                     p.timeout_ns))) {
         ok = false;
         break;
       }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + acc * BN;
       for (int64_t v = u; v < seg_end; ++v) {
-        if (!mbar_wait_bounded(full_bar(stage), phase, abort_flag, p.status,
-                               LLMINT8_DEV_TIMEOUT_MMA, p.timeout_ns)) {
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait_bounded(full_bar(stage), phase, abort_flag,
+                                                       p.status, LLMINT8_DEV_TIMEOUT_MMA,
+                                                       p.timeout_ns))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint64_t a_desc = smem_desc_kmajor_sw128(sA + stage * A_STAGE_BYTES);
-        const uint64_t b_desc = smem_desc_kmajor_sw128(sB + stage * B_STAGE_BYTES);
+        if (lane == 0) {
 #pragma unroll
-        for (int k = 0; k < BK / UMMA_K; ++k)
-          mma_i8(d_tmem, a_desc + (uint64_t)((k * UMMA_K) >> 4),
-                 b_desc + (uint64_t)((k * UMMA_K) >> 4), idesc, (v > u || k > 0) ? 1u : 0u);
+          for (int b = 0; b < SUB; ++b) {
+            const uint64_t a_desc =
+                smem_desc_kmajor_sw128(sA + stage * A_STAGE_BYTES + b * A_BOX_BYTES);
+            const uint64_t b_desc =
+                smem_desc_kmajor_sw128(sB + stage * B_STAGE_BYTES + b * B_BOX_BYTES);
+#pragma unroll
+            for (int k = 0; k < BOX_K / UMMA_K; ++k)
+              mma_i8(d_tmem, a_desc + (uint64_t)((k * UMMA_K) >> 4),
+                     b_desc + (uint64_t)((k * UMMA_K) >> 4), idesc,
+                     (v > u || b > 0 || k > 0) ? 1u : 0u);
+          }
+        }
         any = true;
-        mma_commit(empty_bar(stage));
+        const int32_t kb = (int32_t)(v - m_blk * nk);
+        if (kb == next_kb) {
+          const int32_t k0 = kb * BK;
+          const int32_t w0 = k0 >> 5;
+          const int32_t nw = (p.h - k0) < BK ? (p.h - k0 + 31) >> 5 : BK / 32;
+          const uint8_t *stage_a = reinterpret_cast<const uint8_t *>(base_ptr_of(sA, stage));
+          for (int32_t w = 0; w < nw; ++w) {
+            uint32_t bits = s_mask[w0 + w];
+            int32_t rank = s_prefix[w0 + w];
+            while (bits) {
+              const int b = __ffs(bits) - 1;
+              bits &= bits - 1;
+              const int32_t cc = w * 32 + b;  // column inside the k-block
+              const uint8_t *box = stage_a + (cc / BOX_K) * A_BOX_BYTES;
+              const int32_t cb = cc % BOX_K;  // column inside that box
+#pragma unroll
+              for (int q = 0; q < BM / 32; ++q) {
+                const int r = lane + 32 * q;
+                const int64_t j = m_blk * BM + r;
+                if (j < p.o) {
+                  const int8_t code = static_cast<int8_t>(
+                      box[r * BOX_K + ((((cb >> 4) ^ (r & 7)) << 4) | (cb & 15))]);
+                  const float prod = static_cast<float>(code) * aw_rows[q];
+                  p.WO[(int64_t)rank * p.o + j] =
+                      __half_as_ushort(__float2half_rn(__fdiv_rn(prod, 127.0f)));
+                }
+              }
+              ++rank;
+            }
+          }
+          next_kb = next_outlier_kb(kb + 1);
+          __syncwarp();  // every lane has read the stage before it is released
+        }
+        if (lane == 0) mma_commit(empty_bar(stage));
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1u;
         }
       }
       if (!ok) break;
-      mma_commit(tfull_bar(acc));
+      if (lane == 0) mma_commit(tfull_bar(acc));
+      __threadfence();  // publish this segment's outlier weight rows
+      __syncwarp();
+      if (lane == 0) *wo_segments = it + 1;
       u = seg_end;
     }
-    if (!ok && any) {
+    if (!ok && any && lane == 0) {
       volatile int never = 0;
       mma_commit(drain_bar);
       mbar_wait_bounded(drain_bar, 0, &never, p.status, LLMINT8_DEV_TIMEOUT_DRAIN, p.timeout_ns);
@@ -205,14 +348,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp >= EPI_WARP0) {
     // ---------------------------------------------------------- epilogue
     const int ew = warp - EPI_WARP0;
+    const int et = threadIdx.x - EPI_WARP0 * 32;  // 0..127: one tile column
+    const int32_t n_out = *p.n_out;
+    __shared__ int last_arrival;
     int32_t it = 0;
     for (int64_t u = u0; u < u1; ++it) {
       const int64_t m_blk = u / nk;
       const int64_t seg_end = min(u1, (m_blk + 1) * nk);
       const uint32_t acc = it & 1, acc_par = (it >> 1) & 1;
-      if (!mbar_wait_bounded(tfull_bar(acc), acc_par, abort_flag, p.status,
-                             LLMINT8_DEV_TIMEOUT_EPILOGUE, p.timeout_ns))
-        break;
+      const int64_t j = m_blk * BM + et;  // this thread's output column
+      const bool ready = mbar_wait_bounded(tfull_bar(acc), acc_par, abort_flag, p.status,
+                                           LLMINT8_DEV_TIMEOUT_EPILOGUE, p.timeout_ns);
+      if (named_barrier_or(EPI_BARRIER, NUM_EPI_THREADS, !ready)) break;
       tc_fence_after();
       uint32_t v[16];
       __syncwarp();
@@ -220,11 +367,58 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(tempty_bar(acc));
-      const int64_t j = m_blk * BM + ew * 32 + lane;
       if (j < p.o) {
 #pragma unroll
         for (int i = 0; i < BN; ++i)
           if (i < p.s && v[i] != 0u) atomicAdd(p.cacc + (int64_t)i * p.o + j, (int32_t)v[i]);
+      }
+      // count this CTA's arrival on the tile once its accumulators and its
+      // outlier weight rows (warp 3) are visible; the last contributor
+      // finishes the tile
+      bool rows_ok = true;
+      if (*wo_segments <= it) {  // bounded wait for the MMA warp's publication
+        const uint64_t t0 = global_timer_ns();
+        while (*wo_segments <= it) {
+          if (*abort_flag || global_timer_ns() - t0 > p.timeout_ns) {
+            if (!*abort_flag) {
+              *abort_flag = 1;
+              atomicOr(p.status, LLMINT8_DEV_TIMEOUT_EPILOGUE);
+            }
+            rows_ok = false;
+            break;
+          }
+        }
+      }
+      __threadfence();
+      if (named_barrier_or(EPI_BARRIER, NUM_EPI_THREADS, !rows_ok)) break;
+      if (et == 0) {
+        const int64_t contrib = cta_of_unit(p, (m_blk + 1) * nk - 1) - cta_of_unit(p, m_blk * nk) + 1;
+        last_arrival = (atomicAdd(p.tile_count + m_blk, 1) == (int32_t)(contrib - 1));
+      }
+      named_barrier(EPI_BARRIER, NUM_EPI_THREADS);
+      if (last_arrival && j < p.o) {
+        __threadfence();
+        const float awj = __ldcg(p.aw + j);
+        float wo[16];
+        const int32_t nf = n_out < 16 ? n_out : 16;
+#pragma unroll
+        for (int t = 0; t < 16; ++t)
+          wo[t] = (t < nf) ? __half2float(__ushort_as_half(__ldcg(p.WO + (int64_t)t * p.o + j)))
+                           : 0.0f;
+        for (int32_t i = 0; i < p.s; ++i) {
+          const int32_t c = __ldcg(p.cacc + (int64_t)i * p.o + j);
+          float acc_f = (float)c * (__ldg(p.ax + i) * (1.0f / 16129.0f)) * awj;
+          const uint16_t *xo = p.XO + (int64_t)i * n_out;
+#pragma unroll
+          for (int t = 0; t < 16; ++t)
+            if (t < nf) acc_f = fmaf(__half2float(__ushort_as_half(__ldcg(xo + t))), wo[t], acc_f);
+          for (int32_t t = 16; t < n_out; ++t)
+            acc_f = fmaf(__half2float(__ushort_as_half(__ldcg(xo + t))),
+                         __half2float(__ushort_as_half(__ldcg(p.WO + (int64_t)t * p.o + j))),
+                         acc_f);
+          p.out[(int64_t)i * p.o + j] = __half_as_ushort(__float2half_rn(acc_f));
+          if (p.ci) p.ci[(int64_t)i * p.o + j] = c;
+        }
       }
       u = seg_end;
     }
@@ -234,24 +428,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 2) tmem_dealloc(tmem_base, TMEM_COLS);
-}
-
-// Dequantisation, outlier product and fp16 store for the s <= 16 rows.
-__global__ void __launch_bounds__(256) k_decode_finish(const Params p) {
-  grid_dependency_wait();
-  const int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-  if (g >= (int64_t)p.s * p.o) return;
-  const int32_t i = (int32_t)(g / p.o);
-  const int32_t j = (int32_t)(g - (int64_t)i * p.o);
-  const int32_t n_out = *p.n_out;
-  const int32_t c = p.cacc[(int64_t)i * p.o + j];
-  float acc = (float)c * (p.ax[i] * (1.0f / 16129.0f)) * p.aw[j];
-  const uint16_t *xo = p.XO + (int64_t)i * n_out;
-  for (int32_t t = 0; t < n_out; ++t)
-    acc = fmaf(__half2float(__ushort_as_half(xo[t])),
-               __half2float(__ushort_as_half(p.WO[(int64_t)t * p.o + j])), acc);
-  p.out[g] = __half_as_ushort(__float2half_rn(acc));
-  if (p.ci) p.ci[g] = c;
 }
 
 }  // namespace decode

@@ -60,6 +60,8 @@ constexpr size_t SMEM_BYTES = 1024 + BAR_OFF + 256;
 static_assert(NUM_ACC * BN <= 512, "TMEM holds 512 columns");
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 static_assert(OUT_OFF % 1024 == 0, "swizzled staging must be 1024-byte aligned");
+static_assert(BAR_OFF % 8 == 0, "mbarrier alignment");
+static_assert((2 * STAGES + 2 * NUM_ACC + 1) * 8 + 8 <= 256, "barrier block size");
 
 struct Params {
   int32_t s, h, o;

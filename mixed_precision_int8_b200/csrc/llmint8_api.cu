@@ -116,7 +116,7 @@ bool make_tmap_f16(CUtensorMap *map, void *ptr, uint64_t inner, uint64_t rows,
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct Layout {
-  size_t status, mask, wprefix, idx, ax, xq, xo, wo, cacc, end;
+  size_t status, mask, wprefix, idx, ax, xq, xo, wo, tiles, cacc, end;
   size_t xstage, ostage, end_host;
 };
 
@@ -133,6 +133,7 @@ Layout layout_for(int64_t s, int64_t h, int64_t o) {
   L.xq = off;      off = align256(off + (size_t)s * h);
   L.xo = off;      off = align256(off + 2 * (size_t)s * h);
   L.wo = off;      off = align256(off + 2 * (size_t)h * o);
+  L.tiles = off;   off = align256(off + 4 * (size_t)((o + decode::BM - 1) / decode::BM));
   L.cacc = off;    off = align256(off + 4 * (size_t)kDecodeMaxRows * o);
   L.end = off;
   L.xstage = off;  off = align256(off + 2 * (size_t)s * h);
@@ -325,8 +326,8 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
   CUtensorMap tmA, tmB, tmOut;
   if (use_decode) {
     // A = Wq tiles (rows of o), B = Xq rows (s <= 16, zero-filled to 16)
-    if (!make_tmap_i8(&tmA, w->wq_dev, (uint64_t)h, (uint64_t)o, decode::BK, decode::BM) ||
-        !make_tmap_i8(&tmB, xq, (uint64_t)h, (uint64_t)s, decode::BK, decode::BN))
+    if (!make_tmap_i8(&tmA, w->wq_dev, (uint64_t)h, (uint64_t)o, decode::BOX_K, decode::BM) ||
+        !make_tmap_i8(&tmB, xq, (uint64_t)h, (uint64_t)s, decode::BOX_K, decode::BN))
       return LLMINT8_ERR_CUDA;
   } else {
     if (!make_tmap_i8(&tmA, xq, (uint64_t)h, (uint64_t)s, gemm::BK, gemm::BM) ||
@@ -353,10 +354,37 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
   act.wq = w->wq_dev;
   act.aw = w->aw_dev;
   act.o = o;
-  act.WO = wo;
-  act.zero_buf = use_decode ? cacc : nullptr;
-  act.zero_n = use_decode ? (int64_t)kDecodeMaxRows * o : 0;
-  if ((rc = enqueue_activation_pass(*dev, act, st, &launches))) return rc;
+  // decode: the W^O gather and the finishing step run inside the decode
+  // kernel; its tile counters and the s rows of int32 partial sums (one
+  // contiguous region) start from zero
+  act.WO = use_decode ? nullptr : wo;
+  int32_t *tiles = reinterpret_cast<int32_t *>(wsb + L.tiles);
+  act.zero_buf = use_decode ? tiles : nullptr;
+  act.zero_n = use_decode ? (int64_t)((L.cacc - L.tiles) / 4) + s * o : 0;
+  if (use_decode) {
+    // two launches of 1024-column blocks; the first also zeroes the tile
+    // counters and the s rows of int32 partial sums (extra blocks). This
+    // path needs no outlier list (the decode kernel reads outlier rows of W
+    // with the bitmask and prefix counts), so the list's region holds the
+    // per-block row maxima ([col_blocks][16] words <= h words)
+    const int32_t col_blocks = (int32_t)((h + kDecodeColsPerBlock - 1) / kDecodeColsPerBlock);
+    int64_t zb = (act.zero_n + kDecodeThreads * 8 - 1) / (kDecodeThreads * 8);
+    if (zb > 2 * (int64_t)dev->sm_count) zb = 2 * (int64_t)dev->sm_count;
+    if (zb < 1) zb = 1;
+    uint32_t *partial = reinterpret_cast<uint32_t *>(idx);  // idx unused on this path
+    cudaError_t e0 = launch(k_decode_colpass, dim3((unsigned)(col_blocks + zb)),
+                            dim3(kDecodeThreads), 0, st, false, X, (int32_t)s, (int32_t)h,
+                            threshold_bits(alpha), mask, partial, col_blocks, act.zero_buf,
+                            act.zero_n);
+    if (e0 != cudaSuccess) return LLMINT8_ERR_CUDA;
+    e0 = launch(k_decode_rowpass, dim3((unsigned)col_blocks), dim3(kDecodeThreads), 0, st, true,
+                X, (int32_t)s, (int32_t)h, (const uint32_t *)mask, (const uint32_t *)partial,
+                col_blocks, wprefix, count, ax, xq, xo);
+    if (e0 != cudaSuccess) return LLMINT8_ERR_CUDA;
+    launches += 2;
+  } else if ((rc = enqueue_activation_pass(*dev, act, st, &launches))) {
+    return rc;
+  }
   const bool timed = opts && (opts->gemm_event_start || opts->gemm_event_stop);
   if (opts && opts->gemm_event_start)
     cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->gemm_event_start), st);
@@ -370,12 +398,15 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
     p.num_k_blocks = (int32_t)((h + decode::BK - 1) / decode::BK);
     p.ax = ax;
     p.aw = w->aw_dev;
+    p.mask = mask;
+    p.word_prefix = wprefix;
     p.XO = xo;
     p.WO = wo;
     p.n_out = count;
     p.out = out;
     p.ci = opts ? opts->ci_dev : nullptr;
     p.cacc = cacc;
+    p.tile_count = tiles;
     p.status = status;
     p.timeout_ns = kTimeoutNs;
     const int64_t total_units = (int64_t)p.num_m_blocks * p.num_k_blocks;
@@ -387,10 +418,7 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
     if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
     if (opts && opts->gemm_event_stop)
       cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->gemm_event_stop), st);
-    e = launch(decode::k_decode_finish, dim3((unsigned)((s * o + 255) / 256)), dim3(256), 0, st,
-               !timed, p);
-    if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
-    launches += 2;
+    launches += 1;
   } else {
     gemm::Params p;
     p.s = (int32_t)s;

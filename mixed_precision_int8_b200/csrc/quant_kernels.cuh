@@ -43,11 +43,10 @@ __device__ __forceinline__ int32_t absmax_code(float x, float a) {
 __device__ __forceinline__ int32_t absmax_code_recip(float x, float a, float r) {
   const float t = 127.0f * fabsf(x);
   float n = floorf(fmaf(t, r, 0.5f));
-  if (fmaf(-(n - 0.5f), a, t) < 0.0f)
-    n -= 1.0f;
-  else if (fmaf(-(n + 0.5f), a, t) >= 0.0f)
-    n += 1.0f;
-  n = fminf(n, 127.0f);
+  // (n + 1/2) a > (n - 1/2) a, so at most one of the two corrections applies
+  const float below = fmaf(-(n - 0.5f), a, t) < 0.0f ? 1.0f : 0.0f;
+  const float above = fmaf(-(n + 0.5f), a, t) >= 0.0f ? 1.0f : 0.0f;
+  n = fminf(n + above - below, 127.0f);
   return static_cast<int32_t>(copysignf(n, x));
 }
 
@@ -220,10 +219,10 @@ __global__ void __launch_bounds__(kColThreads)
 // and, in the same launch, the W half of Step 2 (k_rows_and_outlier_w).
 
 // Outlier position of column c + e (its rank among the outlier columns).
-__device__ __forceinline__ int32_t outlier_rank(const int32_t *__restrict__ word_prefix,
-                                                uint32_t mask_word, int32_t c, int e) {
+__device__ __forceinline__ int32_t outlier_rank(const int32_t *word_prefix, uint32_t mask_word,
+                                                int32_t c, int e) {
   const int bit = (c & 31) + e;
-  return __ldg(word_prefix + (c >> 5)) + __popc(mask_word & ((1u << bit) - 1u));
+  return word_prefix[c >> 5] + __popc(mask_word & ((1u << bit) - 1u));
 }
 
 // Four codes (low bytes of a..d) packed into one word, byte 0 = a.
@@ -237,7 +236,7 @@ __device__ __forceinline__ uint32_t pack4_bytes(int32_t a, int32_t b, int32_t c,
 // scale is a (r ~ 1/a; a == 0 gives zero codes).
 __device__ __forceinline__ void quantize_chunk(const uint4 v, uint32_t mw, int32_t c, float a,
                                                float r, int64_t row, int32_t n_out,
-                                               const int32_t *__restrict__ word_prefix,
+                                               const int32_t *word_prefix,
                                                int8_t *__restrict__ qr,
                                                uint16_t *__restrict__ XO) {
   const uint32_t mk = (mw >> (c & 31)) & 0xFFu;
@@ -425,6 +424,162 @@ __global__ void __launch_bounds__(kRowThreads)
     const uint4 v = __ldg(reinterpret_cast<const uint4 *>(xr + c));
     quantize_chunk(v, __ldg(mask + (c >> 5)), c, a, r, row, n_out, word_prefix, qr, XO);
   }
+}
+
+// ----------------------------------------------------- K1 for s <= 16
+// Decode-sized calls (s <= 16): every thread loads all s rows of its 8
+// columns, so it knows those columns' outlier status by itself. Two launches
+// of kDecodeColsPerBlock-column blocks then cover the activation side with
+// no atomics and nothing to zero beforehand:
+//   k_decode_colpass: bitmask words (plain stores) and, per block, the
+//                     maximum over its regular columns of every row;
+//                     extra blocks zero `zero_buf`.
+//   k_decode_rowpass: row scales (max over the blocks' partial maxima),
+//                     outlier prefix counts, |O|, codes and the fp16 outlier
+//                     columns of X.
+constexpr int kDecodeThreads = 128;
+constexpr int kDecodeColsPerBlock = kDecodeThreads * 8;
+constexpr int kSmallMaxRows = 16;
+
+__global__ void __launch_bounds__(kDecodeThreads)
+    k_decode_colpass(const uint16_t *__restrict__ X, int32_t s, int32_t h, uint32_t thresh_bits,
+                     uint32_t *__restrict__ mask, uint32_t *__restrict__ partial_max,
+                     int32_t col_blocks, int32_t *__restrict__ zero_buf, int64_t zero_n) {
+  __shared__ uint32_t red[kDecodeThreads / 32][kSmallMaxRows];
+  grid_dependency_wait();
+  grid_dependency_trigger();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if ((int32_t)blockIdx.x >= col_blocks) {
+    const int64_t stride = (int64_t)(gridDim.x - col_blocks) * blockDim.x;
+    for (int64_t i = (int64_t)(blockIdx.x - col_blocks) * blockDim.x + tid; i < zero_n;
+         i += stride)
+      zero_buf[i] = 0;
+    return;
+  }
+  const int32_t c = blockIdx.x * kDecodeColsPerBlock + tid * 8;
+  uint4 v[kSmallMaxRows];
+  uint32_t m2[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+  for (int i = 0; i < kSmallMaxRows; ++i)
+    if (i < s && c < h) v[i] = __ldg(reinterpret_cast<const uint4 *>(X + (int64_t)i * h + c));
+#pragma unroll
+  for (int i = 0; i < kSmallMaxRows; ++i) {
+    if (i < s && c < h) {
+      m2[0] = __vmaxu2(m2[0], v[i].x & 0x7FFF7FFFu);
+      m2[1] = __vmaxu2(m2[1], v[i].y & 0x7FFF7FFFu);
+      m2[2] = __vmaxu2(m2[2], v[i].z & 0x7FFF7FFFu);
+      m2[3] = __vmaxu2(m2[3], v[i].w & 0x7FFF7FFFu);
+    }
+  }
+  uint32_t m8 = 0;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    m8 |= ((m2[e] & 0xFFFFu) >= thresh_bits ? 1u : 0u) << (2 * e);
+    m8 |= ((m2[e] >> 16) >= thresh_bits ? 1u : 0u) << (2 * e + 1);
+  }
+  if (c >= h) m8 = 0;
+  uint32_t word = m8 << (8 * (lane & 3));
+  word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
+  word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
+  if ((lane & 3) == 0 && c < h) mask[c >> 5] = word;
+  // per-row maxima over this thread's regular columns, reduced over the block
+#pragma unroll
+  for (int i = 0; i < kSmallMaxRows; ++i) {
+    if (i < s) {
+      uint32_t m = (c < h) ? max_halves(regular_absmax2(0u, v[i], m8)) : 0u;
+#pragma unroll
+      for (int d = 16; d > 0; d >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, d));
+      if (lane == 0) red[warp][i] = m;
+    }
+  }
+  __syncthreads();
+  if (tid < s) {
+    uint32_t m = 0;
+#pragma unroll
+    for (int w = 0; w < kDecodeThreads / 32; ++w) m = max(m, red[w][tid]);
+    partial_max[(int64_t)blockIdx.x * kSmallMaxRows + tid] = m;
+  }
+}
+
+__global__ void __launch_bounds__(kDecodeThreads)
+    k_decode_rowpass(const uint16_t *__restrict__ X, int32_t s, int32_t h,
+                     const uint32_t *__restrict__ mask, const uint32_t *__restrict__ partial_max,
+                     int32_t col_blocks, int32_t *__restrict__ word_prefix,
+                     int32_t *__restrict__ count, float *__restrict__ ax,
+                     int8_t *__restrict__ Xq, uint16_t *__restrict__ XO) {
+  __shared__ float row_a[kSmallMaxRows], row_r[kSmallMaxRows];
+  __shared__ int32_t s_prefix[kDecodeColsPerBlock / 32];
+  __shared__ int32_t red_before[kDecodeThreads / 32], red_total[kDecodeThreads / 32];
+  grid_dependency_wait();
+  grid_dependency_trigger();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int32_t nwords = (h + 31) >> 5;
+  const int32_t w_begin = blockIdx.x * (kDecodeColsPerBlock / 32);
+  // row scales: maximum over every column block's partial maximum
+  if (tid < s) {
+    uint32_t m = 0;
+    for (int32_t b = 0; b < col_blocks; ++b)
+      m = max(m, __ldg(partial_max + (int64_t)b * kSmallMaxRows + tid));
+    const float a = half_bits_to_float(m);
+    row_a[tid] = a;
+    row_r[tid] = a > 0.0f ? __frcp_rn(a) : 0.0f;
+    if (blockIdx.x == 0) ax[tid] = a;
+  }
+  // outlier columns before this block, and in total
+  int32_t before = 0, total = 0;
+  for (int32_t w = tid; w < nwords; w += kDecodeThreads) {
+    const int32_t pc = __popc(__ldg(mask + w));
+    total += pc;
+    if (w < w_begin) before += pc;
+  }
+#pragma unroll
+  for (int d = 16; d > 0; d >>= 1) {
+    before += __shfl_xor_sync(0xFFFFFFFFu, before, d);
+    total += __shfl_xor_sync(0xFFFFFFFFu, total, d);
+  }
+  if (lane == 0) {
+    red_before[warp] = before;
+    red_total[warp] = total;
+  }
+  __syncthreads();
+  before = 0;
+  total = 0;
+#pragma unroll
+  for (int w = 0; w < kDecodeThreads / 32; ++w) {
+    before += red_before[w];
+    total += red_total[w];
+  }
+  // prefix counts of this block's 32 mask words (one warp)
+  if (warp == 0) {
+    const int32_t w = w_begin + lane;
+    const int32_t pc = (w < nwords) ? __popc(__ldg(mask + w)) : 0;
+    int32_t incl = pc;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+      if (lane >= d) incl += y;
+    }
+    const int32_t pre = before + incl - pc;
+    s_prefix[lane] = pre;
+    if (w < nwords) word_prefix[w] = pre;
+    if (w == nwords - 1) word_prefix[nwords] = pre + pc;
+  }
+  if (blockIdx.x == 0 && tid == 0) *count = total;
+  __syncthreads();
+  // codes and the fp16 outlier columns of this block's columns, all rows
+  const int32_t c = blockIdx.x * kDecodeColsPerBlock + tid * 8;
+  if (c >= h) return;
+  const uint32_t mw = __ldg(mask + (c >> 5));
+  uint4 v[kSmallMaxRows];
+#pragma unroll
+  for (int i = 0; i < kSmallMaxRows; ++i)
+    if (i < s) v[i] = __ldg(reinterpret_cast<const uint4 *>(X + (int64_t)i * h + c));
+  const int32_t *pre_local = s_prefix - w_begin;  // indexed by global word
+#pragma unroll
+  for (int i = 0; i < kSmallMaxRows; ++i)
+    if (i < s)
+      quantize_chunk(v[i], mw, c, row_a[i], row_r[i], i, total, pre_local, Xq + (int64_t)i * h,
+                     XO);
 }
 
 // ------------------------------------------------------------------- K0

@@ -45,6 +45,8 @@ SMALL = [
     (64, 256, 512, (9, 99), math.inf),                    # decomposition off
     (40, 128, 256, (), 0.0),                               # every column out
     (256, 4096, 256, (11, 4000), 6.0),
+    (9, 1040, 256, tuple(range(3, 1040, 61)), 6.0),        # decode, |O| = 17
+    (12, 256, 272, (), 0.0),                               # decode, |O| = h
 ]
 
 
