@@ -15,12 +15,12 @@
 //               into a TMEM accumulator; tcgen05.commit frees ring slots
 //   warp 2      allocates / frees the 512 TMEM columns (2 accumulators)
 //   warps 4-7   epilogue: stage the tile's column scales and fp16 outlier
-//               rows in shared memory while the MMA runs, then tcgen05.ld
-//               the int32 accumulator (each warp owns 32 TMEM lanes = 32
-//               output rows), dequantise, add the outlier product on CUDA
-//               cores, and write fp16 through a 128B-swizzled staging block
-//               with TMA stores; the other accumulator is being filled by
-//               the MMA meanwhile.
+//               rows (as fp32) in shared memory while the MMA runs, then
+//               tcgen05.ld the int32 accumulator (each warp owns 32 TMEM
+//               lanes = 32 output rows), dequantise and add the outlier
+//               product with packed f32x2 FMAs on CUDA cores, and write fp16
+//               through a 128B-swizzled staging block with TMA stores; the
+//               other accumulator is being filled by the MMA meanwhile.
 // Every wait is bounded by the global timer; on a timeout the CTA records a
 // status bit, drains its in-flight copies and MMAs, frees TMEM and returns.
 #pragma once
@@ -52,8 +52,8 @@ constexpr uint32_t OUT_STAGE_BYTES = 32 * OUT_BOX_COLS * 2;  // per epilogue war
 constexpr int FAST_OUTLIERS = 16;    // outlier rows kept in shared memory
 constexpr uint32_t RING_BYTES = STAGES * (A_STAGE_BYTES + B_STAGE_BYTES);
 constexpr uint32_t OUT_OFF = RING_BYTES;
-constexpr uint32_t WO_OFF = OUT_OFF + 4 * OUT_STAGE_BYTES;
-constexpr uint32_t AW_OFF = WO_OFF + FAST_OUTLIERS * BN * 2;
+constexpr uint32_t WO_OFF = OUT_OFF + 4 * OUT_STAGE_BYTES;  // fp32 [FAST_OUTLIERS][BN]
+constexpr uint32_t AW_OFF = WO_OFF + FAST_OUTLIERS * BN * 4;
 constexpr uint32_t BAR_OFF = AW_OFF + BN * 4;
 constexpr size_t SMEM_BYTES = 1024 + BAR_OFF + 256;
 
@@ -220,7 +220,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int et = threadIdx.x - EPI_WARP0 * 32;  // 0..127
     const int32_t n_out = *p.n_out;
     const int32_t n_fast = n_out < FAST_OUTLIERS ? n_out : FAST_OUTLIERS;
-    uint16_t *sWO = reinterpret_cast<uint16_t *>(base + WO_OFF);  // [16][BN]
+    float *sWO = reinterpret_cast<float *>(base + WO_OFF);         // [16][BN] fp32
     float *sAW = reinterpret_cast<float *>(base + AW_OFF);         // [BN]
     uint8_t *sOut = base + OUT_OFF + ew * OUT_STAGE_BYTES;         // [32][128 B]
     const uint32_t sOut_addr = smem_u32(sOut);
@@ -243,7 +243,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int32_t j = n0 + c8;
         uint4 w8 = make_uint4(0u, 0u, 0u, 0u);
         if (j < p.o) w8 = __ldg(reinterpret_cast<const uint4 *>(p.WO + (int64_t)t * p.o + j));
-        *reinterpret_cast<uint4 *>(sWO + t * BN + c8) = w8;
+        const uint32_t ww[4] = {w8.x, w8.y, w8.z, w8.w};
+        float4 *dst = reinterpret_cast<float4 *>(sWO + t * BN + c8);
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float2 f0 = __half22float2(*reinterpret_cast<const __half2 *>(&ww[2 * e]));
+          const float2 f1 = __half22float2(*reinterpret_cast<const __half2 *>(&ww[2 * e + 1]));
+          dst[e] = make_float4(f0.x, f0.y, f1.x, f1.y);
+        }
       }
       named_barrier(EPI_BARRIER, NUM_EPI_THREADS);
       // (2) this thread's row: scale and outlier activations
@@ -273,42 +280,60 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tc_fence_before();
           mbar_arrive(tempty_bar(acc));
         }
-        float accf[32];
+        // outlier product e = sum_t xo[t] * WO[t][j], then
+        // out = fp16(ci * (rs * aw[j]) + e), two columns per packed op
+        uint64_t e2[16];
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          const float4 a4 = *reinterpret_cast<const float4 *>(sAW + c * 32 + 4 * q4);
-          accf[4 * q4 + 0] = (float)(int32_t)v[4 * q4 + 0] * rs * a4.x;
-          accf[4 * q4 + 1] = (float)(int32_t)v[4 * q4 + 1] * rs * a4.y;
-          accf[4 * q4 + 2] = (float)(int32_t)v[4 * q4 + 2] * rs * a4.z;
-          accf[4 * q4 + 3] = (float)(int32_t)v[4 * q4 + 3] * rs * a4.w;
-        }
+        for (int q = 0; q < 16; ++q) e2[q] = 0ull;
 #pragma unroll
         for (int t = 0; t < FAST_OUTLIERS; ++t) {
           if (t < n_fast) {
+            const uint64_t x2 = f32x2_pack(xo[t], xo[t]);
+            const float4 *wrow = reinterpret_cast<const float4 *>(sWO + t * BN + c * 32);
 #pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8) {
-              const uint4 w8 = *reinterpret_cast<const uint4 *>(sWO + t * BN + c * 32 + 8 * q8);
-              const uint32_t ww[4] = {w8.x, w8.y, w8.z, w8.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&ww[e]));
-                accf[8 * q8 + 2 * e] = fmaf(xo[t], f.x, accf[8 * q8 + 2 * e]);
-                accf[8 * q8 + 2 * e + 1] = fmaf(xo[t], f.y, accf[8 * q8 + 2 * e + 1]);
-              }
+            for (int q4 = 0; q4 < 8; ++q4) {
+              const float4 w = wrow[q4];
+              e2[2 * q4] = f32x2_fma(x2, f32x2_pack(w.x, w.y), e2[2 * q4]);
+              e2[2 * q4 + 1] = f32x2_fma(x2, f32x2_pack(w.z, w.w), e2[2 * q4 + 1]);
             }
           }
         }
-        // outlier columns beyond the shared-memory fast path (|O| > 16)
         const int32_t j0 = n0 + c * 32;
-        for (int32_t t = FAST_OUTLIERS; t < n_out; ++t) {
-          const float x = row_ok ? __half2float(__ushort_as_half(p.XO[(int64_t)row * n_out + t]))
-                                 : 0.0f;
-          const uint16_t *wr = p.WO + (int64_t)t * p.o;
+        if (n_out > FAST_OUTLIERS) {
+          // outlier columns beyond the shared-memory fast path (|O| > 16)
+          float ef[32];
 #pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            const float w = (j0 + q < p.o) ? __half2float(__ushort_as_half(wr[j0 + q])) : 0.0f;
-            accf[q] = fmaf(x, w, accf[q]);
+          for (int q = 0; q < 16; ++q) {
+            ef[2 * q] = f32x2_lo(e2[q]);
+            ef[2 * q + 1] = f32x2_hi(e2[q]);
           }
+          for (int32_t t = FAST_OUTLIERS; t < n_out; ++t) {
+            const float x =
+                row_ok ? __half2float(__ushort_as_half(p.XO[(int64_t)row * n_out + t])) : 0.0f;
+            const uint16_t *wr = p.WO + (int64_t)t * p.o;
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+              const float w = (j0 + q < p.o) ? __half2float(__ushort_as_half(wr[j0 + q])) : 0.0f;
+              ef[q] = fmaf(x, w, ef[q]);
+            }
+          }
+#pragma unroll
+          for (int q = 0; q < 16; ++q) e2[q] = f32x2_pack(ef[2 * q], ef[2 * q + 1]);
+        }
+        const uint64_t rs2 = f32x2_pack(rs, rs);
+        uint32_t h2[16];  // fp16 pairs of the 32 outputs
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const float4 a4 = *reinterpret_cast<const float4 *>(sAW + c * 32 + 4 * q4);
+          const uint64_t sv0 = f32x2_mul(rs2, f32x2_pack(a4.x, a4.y));
+          const uint64_t sv1 = f32x2_mul(rs2, f32x2_pack(a4.z, a4.w));
+          const uint64_t c0 = f32x2_pack((float)(int32_t)v[4 * q4], (float)(int32_t)v[4 * q4 + 1]);
+          const uint64_t c1 =
+              f32x2_pack((float)(int32_t)v[4 * q4 + 2], (float)(int32_t)v[4 * q4 + 3]);
+          const uint64_t r0 = f32x2_fma(c0, sv0, e2[2 * q4]);
+          const uint64_t r1 = f32x2_fma(c1, sv1, e2[2 * q4 + 1]);
+          h2[2 * q4] = f2h2(f32x2_lo(r0), f32x2_hi(r0));
+          h2[2 * q4 + 1] = f2h2(f32x2_lo(r1), f32x2_hi(r1));
         }
         // stage 32 fp16 (64 bytes) of this row into the 128B-swizzled block
         // of 64 columns; chunk k of row r lives at 16-byte slot k ^ (r & 7)
@@ -320,10 +345,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8) {
           const int chunk = half * 4 + q8;
-          const uint4 h8 = make_uint4(f2h2(accf[8 * q8 + 0], accf[8 * q8 + 1]),
-                                      f2h2(accf[8 * q8 + 2], accf[8 * q8 + 3]),
-                                      f2h2(accf[8 * q8 + 4], accf[8 * q8 + 5]),
-                                      f2h2(accf[8 * q8 + 6], accf[8 * q8 + 7]));
+          const uint4 h8 = make_uint4(h2[4 * q8], h2[4 * q8 + 1], h2[4 * q8 + 2], h2[4 * q8 + 3]);
           *reinterpret_cast<uint4 *>(sOut + lane * 128 + ((chunk ^ (lane & 7)) * 16)) = h8;
         }
         if (half == 1) {
