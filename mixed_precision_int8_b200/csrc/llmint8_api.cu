@@ -251,7 +251,7 @@ llmint8_status enqueue_activation_pass(const DeviceInfo &dev, const ActivationAr
   const int64_t want_blocks = 4 * (int64_t)dev.sm_count;
   int64_t gy_target = (want_blocks + gx - 1) / gx;
   int64_t rpb = (a.s + gy_target - 1) / gy_target;
-  if (rpb < 8) rpb = 8;
+  rpb = (rpb + 7) / 8 * 8;  // whole batches of eight rows in flight per thread
   if ((a.s + rpb - 1) / rpb > 65535) rpb = (a.s + 65534) / 65535;
   const int gy = (int)((a.s + rpb - 1) / rpb);
   e = launch(k_outlier_columns, dim3(gx, gy), dim3(kColThreads), 0, st, true, a.X, a.s, hh,

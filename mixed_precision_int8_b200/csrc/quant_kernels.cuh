@@ -50,6 +50,25 @@ __device__ __forceinline__ int32_t absmax_code_recip(float x, float a, float r) 
   return static_cast<int32_t>(copysignf(n, x));
 }
 
+// Fast form of absmax_code_recip. With r = 1/a correctly rounded, y =
+// fma(t, r, 1/2) is within 2^-16 of t/a + 1/2 (t/a <= 127: the reciprocal
+// contributes < 2^-17 and the fma rounding <= 2^-18), so when the fractional
+// part of y is at least 2^-15 away from an integer, floor(y) is already
+// floor(t/a + 1/2), the exactly rounded code. Only values that close to a
+// rounding boundary (about 6 in 10^5) take the exact two-residual correction.
+__device__ __forceinline__ int32_t absmax_code_fast(float x, float a, float r) {
+  const float t = 127.0f * fabsf(x);
+  const float y = fmaf(t, r, 0.5f);
+  const float n0 = floorf(y);
+  float n = n0;
+  if (fabsf((y - n0) - 0.5f) > 0.5f - 3.0517578125e-05f) {  // within 2^-15 of an integer
+    const float below = fmaf(-(n0 - 0.5f), a, t) < 0.0f ? 1.0f : 0.0f;
+    const float above = fmaf(-(n0 + 0.5f), a, t) >= 0.0f ? 1.0f : 0.0f;
+    n = fminf(n0 + above - below, 127.0f);
+  }
+  return static_cast<int32_t>(copysignf(n, x));
+}
+
 __device__ __forceinline__ float half_bits_to_float(uint32_t b) {
   return __half2float(__ushort_as_half(static_cast<unsigned short>(b)));
 }
@@ -249,8 +268,8 @@ __device__ __forceinline__ void quantize_chunk(const uint4 v, uint32_t mw, int32
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[e]));
-      q[2 * e] = absmax_code_recip(f.x, a, r);
-      q[2 * e + 1] = absmax_code_recip(f.y, a, r);
+      q[2 * e] = absmax_code_fast(f.x, a, r);
+      q[2 * e + 1] = absmax_code_fast(f.y, a, r);
     }
     if (mk != 0u) {
 #pragma unroll
