@@ -81,6 +81,7 @@ typedef enum {
 #define LLMINT8_DEV_TIMEOUT_MMA 0x2       /* MMA issuer gave up waiting */
 #define LLMINT8_DEV_TIMEOUT_EPILOGUE 0x4  /* epilogue gave up waiting */
 #define LLMINT8_DEV_TIMEOUT_DRAIN 0x8     /* drain after an abort timed out */
+#define LLMINT8_DEV_TIMEOUT_ROWS 0x10     /* activation row stream gave up waiting */
 
 /* A prepared (offline-quantised) weight. Buffers are caller-owned device
  * memory: wq_dev is int8 [o][h] (the reduction index k contiguous, i.e. the
@@ -119,8 +120,16 @@ LLMINT8_API const char *llmint8_status_string(llmint8_status st);
  * outlier rows of W) + 4*16*o (decode accumulators) + O(h + s). */
 LLMINT8_API size_t llmint8_workspace_size(int64_t s, int64_t h, int64_t o);
 
-/* Clears the workspace's status block (its first 256 bytes). Call once on a
- * new workspace before its first llmint8_matmul; asynchronous on `stream`. */
+/* Bytes at the front of a workspace that hold state kept between calls: the
+ * status words (first 256 bytes), then the outlier bitmask that the one-read
+ * activation pass accumulates into and leaves zero when it finishes. */
+#define LLMINT8_WORKSPACE_STATE_BYTES 17152
+
+/* Clears the workspace's state block (its first LLMINT8_WORKSPACE_STATE_BYTES
+ * bytes; ws_bytes must cover them). Call once on a new workspace before its
+ * first llmint8_matmul, and again before reusing a workspace after a call
+ * returned LLMINT8_ERR_DEVICE_STATUS (an aborted kernel may leave the state
+ * dirty). Asynchronous on `stream`. */
 LLMINT8_API llmint8_status llmint8_workspace_init(void *ws_dev, size_t ws_bytes, void *stream);
 
 /* Workspace for llmint8_matmul_host: llmint8_workspace_size plus staging
@@ -145,7 +154,8 @@ LLMINT8_API llmint8_status llmint8_prepare_weight(const uint16_t *W_dev, int64_t
  *   ax_dev[i]     = max over non-outlier j of |X[i][j]| (0 if none) (f32 [s])
  *   Xq_dev[i][j]  = q(X[i][j], ax[i]) for non-outlier j, else 0  (i8 [s][h])
  * X_dev is fp16 [s][h]. scratch_dev must hold
- * llmint8_quantize_rows_scratch_size(h) bytes (256-byte aligned). */
+ * llmint8_quantize_rows_scratch_size(h) bytes (256-byte aligned); its
+ * contents need no initialisation (word 1 receives device status bits). */
 LLMINT8_API size_t llmint8_quantize_rows_scratch_size(int64_t h);
 LLMINT8_API llmint8_status llmint8_quantize_rows(const uint16_t *X_dev, int64_t s,
                                      int64_t h, float alpha, int8_t *Xq_dev,

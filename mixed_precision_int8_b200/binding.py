@@ -263,9 +263,13 @@ def llmint8_matmul_host(X_host: torch.Tensor, w: PreparedWeight,
     return out_host
 
 
-def llmint8_read_outlier_tiles(workspace: Workspace, stream=None):
-    """(n, XO [s,n] fp16, WO [n,o] fp16) of the last matmul on `workspace`."""
-    s, h, o = workspace.s, workspace.h, workspace.o
+def llmint8_read_outlier_tiles(workspace: Workspace, s: Optional[int] = None,
+                               stream=None):
+    """(n, XO [s,n] fp16, WO [n,o] fp16) of the last matmul on `workspace`,
+    which had `s` rows (default: the row count the workspace was sized for;
+    the workspace layout depends on it)."""
+    h, o = workspace.h, workspace.o
+    s = workspace.s if s is None else int(s)
     n = ctypes.c_int32(0)
     XO = torch.empty((s * h,), dtype=torch.float16)
     WO = torch.empty((h * o,), dtype=torch.float16)

@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -23,6 +24,8 @@ using namespace llmint8;
 constexpr int64_t kMaxH = 133144;  // 127*127*h must fit int32
 constexpr int64_t kDecodeMaxRows = decode::MAX_ROWS;
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per individual wait
+// dynamic shared memory of k_act_rows (one CTA per SM)
+constexpr uint32_t kActSmemOnePerSm = 220 * 1024;
 
 // ----------------------------------------------------------- device info
 struct DeviceInfo {
@@ -53,6 +56,9 @@ llmint8_status device_info(DeviceInfo **out) {
         return LLMINT8_ERR_CUDA;
       if (cudaFuncSetAttribute(decode::k_decode_i8, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)decode::SMEM_BYTES) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+      if (cudaFuncSetAttribute(k_act_rows, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kActSmemOnePerSm) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
     }
     d.init = true;
@@ -116,16 +122,24 @@ bool make_tmap_f16(CUtensorMap *map, void *ptr, uint64_t inner, uint64_t rows,
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct Layout {
-  size_t status, mask, wprefix, idx, ax, xq, xo, wo, tiles, cacc, end;
+  size_t status, acc, mask, wprefix, idx, ax, xq, xo, wo, tiles, cacc, end;
   size_t xstage, ostage, end_host;
 };
 
 int32_t mask_words(int64_t h) { return (int32_t)((h + 31) / 32); }
 
+// The state block at the front of a workspace, cleared by
+// llmint8_workspace_init and kept by the kernels between calls: the status
+// words, then the accumulation bitmask of the one-read activation pass
+// (sized for the largest h), which that pass leaves zero on exit.
+constexpr size_t kStateBytes = 256 + ((4 * (size_t)((kMaxH + 31) / 32) + 255) & ~size_t(255));
+static_assert(kStateBytes == LLMINT8_WORKSPACE_STATE_BYTES, "state block size");
+
 Layout layout_for(int64_t s, int64_t h, int64_t o) {
   Layout L;
   size_t off = 0;
   L.status = off;  off = align256(off + 256);
+  L.acc = off;     off = kStateBytes;
   L.mask = off;    off = align256(off + 4 * (size_t)mask_words(h));
   L.wprefix = off; off = align256(off + 4 * ((size_t)mask_words(h) + 1));
   L.idx = off;     off = align256(off + 4 * (size_t)h);
@@ -142,10 +156,13 @@ Layout layout_for(int64_t s, int64_t h, int64_t o) {
   return L;
 }
 
-// status block: [0] device status bits, [1] |O|, [2] column-pass block counter
+// status block: [0] device status bits, [1] |O|, [2] column-pass block
+// counter, [3] block counter of the one-read activation pass (zero between
+// calls)
 int32_t *status_word(void *ws) { return reinterpret_cast<int32_t *>(ws); }
 int32_t *count_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 1; }
 int32_t *block_counter_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 2; }
+int32_t *act_counter_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 3; }
 
 // --------------------------------------------------------- validation
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -215,6 +232,9 @@ struct ActivationArgs {
   float alpha;
   uint32_t *mask;
   int32_t *wprefix, *idx, *count, *block_counter;
+  uint32_t *acc_mask;     // one-read pass: accumulation bitmask (zero on entry
+  int32_t *act_counter;   // and exit, with its block counter)
+  bool act_reset;         // zero them first (their state is not known)
   uint8_t *flags;
   int8_t *Xq;
   float *ax;
@@ -225,7 +245,109 @@ struct ActivationArgs {
   uint16_t *WO;
   int32_t *zero_buf;
   int64_t zero_n;
+  int *status;  // device status bits
 };
+
+// Launch plan of k_act_rows (one CTA per SM): `groups` row groups of `wpr`
+// warps, each group with `stages` row buffers of `stage_bytes`. Calls with
+// at least 16 rows per SM run one warp per row, as many as shared memory
+// holds (up to 32); shorter calls spread their rows over every SM in one
+// wave with up to four warps per row (named barriers cap the groups at
+// 15). Two buffers per group when they fit. False when one row does not
+// fit, in which case the two-pass kernels run.
+struct ActPlan {
+  int32_t groups;
+  int32_t wpr;
+  int32_t stages;
+  uint32_t stage_bytes;
+  uint32_t smem;
+  int64_t grid;
+};
+
+bool act_plan(int64_t s, int64_t h, int sm_count, ActPlan *plan) {
+  const uint32_t sb = (uint32_t)((2 * h + 127) / 128 * 128);
+  const uint32_t fixed = act_smem_bytes(0, sb, (int32_t)h);
+  if (fixed + sb + 8 > kActSmemOnePerSm) return false;
+  const int64_t fit = (kActSmemOnePerSm - fixed) / (sb + 8);  // buffers that fit
+  int64_t per_sm = (s + sm_count - 1) / sm_count;
+  if (per_sm < 1) per_sm = 1;
+  int64_t groups, wpr;
+  if (per_sm >= 16 && fit >= 16) {
+    wpr = 1;
+    groups = std::min<int64_t>(std::min<int64_t>(fit, per_sm), kActMaxWarps);
+  } else {
+    groups = std::min<int64_t>(std::min<int64_t>(fit, per_sm), kActMaxGroups);
+    wpr = std::max<int64_t>(1, std::min<int64_t>(kActMaxWpr, kActMaxWarps / groups));
+  }
+  const int64_t stages = fit / groups >= 2 ? 2 : 1;
+  plan->groups = (int32_t)groups;
+  plan->wpr = (int32_t)wpr;
+  plan->stages = (int32_t)stages;
+  plan->stage_bytes = sb;
+  plan->smem = act_smem_bytes((int32_t)(groups * stages), sb, (int32_t)h);
+  int64_t grid = (s + groups - 1) / groups;
+  if (grid > sm_count) grid = sm_count;
+  if (grid < 1) grid = 1;
+  plan->grid = grid;
+  return true;
+}
+
+// Steps 1 and 4 with one read of X (k_act_rows), then the completion of the
+// outlier columns and the fp16 outlier rows of W (k_act_fixup).
+llmint8_status enqueue_activation_fused(const DeviceInfo &dev, const ActivationArgs &a,
+                                        const ActPlan &plan, cudaStream_t st,
+                                        int32_t *launches) {
+  cudaError_t e;
+  if (a.act_reset) {
+    int64_t reset_blocks = (mask_words(a.h) + 255) / 256;
+    if (reset_blocks > 4 * (int64_t)dev.sm_count) reset_blocks = 4 * (int64_t)dev.sm_count;
+    e = launch(k_reset_mask, dim3((unsigned)reset_blocks), dim3(256), 0, st, false, a.acc_mask,
+               mask_words(a.h), a.count, a.act_counter, (int32_t *)nullptr, (int64_t)0);
+    if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+    *launches += 1;
+  }
+  ActRowsParams p;
+  p.X = a.X;
+  p.s = a.s;
+  p.h = (int32_t)a.h;
+  p.thresh_bits = threshold_bits(a.alpha);
+  p.groups = plan.groups;
+  p.wpr = plan.wpr;
+  p.stages = plan.stages;
+  p.stage_bytes = plan.stage_bytes;
+  p.timeout_ns = kTimeoutNs;
+  p.acc_mask = a.acc_mask;
+  p.mask = a.mask;
+  p.count = a.count;
+  p.block_counter = a.act_counter;
+  p.word_prefix = a.wprefix;
+  p.idx = a.idx;
+  p.flags = a.flags;
+  p.Xq = a.Xq;
+  p.ax = a.ax;
+  p.status = a.status;
+  e = launch(k_act_rows, dim3((unsigned)plan.grid), dim3(32 * plan.groups * plan.wpr), plan.smem,
+             st, true, p);
+  if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+  *launches += 1;
+  // WO blocks: enough for 16 outlier columns at four pairs per thread, at
+  // most eight per SM (larger |O| loops)
+  int64_t wo_blocks = 0;
+  if (a.WO) {
+    wo_blocks = (16 * a.o + 4 * kFixThreads - 1) / (4 * kFixThreads);
+    wo_blocks = std::min<int64_t>(std::max<int64_t>(wo_blocks, 1), 8 * (int64_t)dev.sm_count);
+  }
+  const int64_t fix_blocks = wo_blocks + (a.s + kFixRowsPerBlock - 1) / kFixRowsPerBlock;
+  if (fix_blocks > 0) {
+    e = launch(k_act_fixup, dim3((unsigned)fix_blocks), dim3(kFixThreads), 0, st, true, a.X,
+               a.s, (int32_t)a.h, p.thresh_bits, (const uint32_t *)a.mask,
+               (const int32_t *)a.wprefix, (const int32_t *)a.idx, (const int32_t *)a.count,
+               a.Xq, a.ax, a.XO, a.wq, a.aw, (int32_t)a.o, a.WO, (int32_t)wo_blocks);
+    if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+    *launches += 1;
+  }
+  return last_launch();
+}
 
 template <int NV>
 cudaError_t launch_rows(const ActivationArgs &a, int64_t wo_blocks, cudaStream_t st) {
@@ -238,6 +360,9 @@ cudaError_t launch_rows(const ActivationArgs &a, int64_t wo_blocks, cudaStream_t
 
 llmint8_status enqueue_activation_pass(const DeviceInfo &dev, const ActivationArgs &a,
                                        cudaStream_t st, int32_t *launches) {
+  ActPlan plan;
+  if (a.zero_n == 0 && act_plan(a.s, a.h, dev.sm_count, &plan))
+    return enqueue_activation_fused(dev, a, plan, st, launches);
   const int32_t nwords = mask_words(a.h);
   const int32_t hh = (int32_t)a.h;
   int64_t reset_threads = nwords > a.zero_n ? nwords : a.zero_n;
@@ -347,7 +472,11 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
   act.idx = idx;
   act.count = count;
   act.block_counter = block_counter_word(ws);
+  act.acc_mask = reinterpret_cast<uint32_t *>(wsb + L.acc);
+  act.act_counter = act_counter_word(ws);
+  act.act_reset = false;  // the workspace keeps them zero between calls
   act.flags = nullptr;
+  act.status = status;
   act.Xq = xq;
   act.ax = ax;
   act.XO = xo;
@@ -477,9 +606,10 @@ size_t llmint8_workspace_size(int64_t s, int64_t h, int64_t o) {
 llmint8_status llmint8_workspace_init(void *ws_dev, size_t ws_bytes, void *stream) {
   if (!ws_dev) return LLMINT8_ERR_NULL;
   if (!aligned(ws_dev, 256)) return LLMINT8_ERR_ALIGN;
-  if (ws_bytes < 256) return LLMINT8_ERR_WORKSPACE;
-  return cudaMemsetAsync(ws_dev, 0, 256, as_stream(stream)) == cudaSuccess ? LLMINT8_OK
-                                                                           : LLMINT8_ERR_CUDA;
+  if (ws_bytes < kStateBytes) return LLMINT8_ERR_WORKSPACE;
+  return cudaMemsetAsync(ws_dev, 0, kStateBytes, as_stream(stream)) == cudaSuccess
+             ? LLMINT8_OK
+             : LLMINT8_ERR_CUDA;
 }
 
 size_t llmint8_workspace_size_host(int64_t s, int64_t h, int64_t o) {
@@ -518,7 +648,8 @@ llmint8_status llmint8_prepare_weight(const uint16_t *W_dev, int64_t h, int64_t 
 
 size_t llmint8_quantize_rows_scratch_size(int64_t h) {
   if (h < 0) return 0;
-  return 256 + align256(4 * (size_t)mask_words(h)) + align256(4 * ((size_t)mask_words(h) + 1));
+  return 256 + 2 * align256(4 * (size_t)mask_words(h)) +
+         align256(4 * ((size_t)mask_words(h) + 1));
 }
 
 llmint8_status llmint8_quantize_rows(const uint16_t *X_dev, int64_t s, int64_t h, float alpha,
@@ -543,12 +674,18 @@ llmint8_status llmint8_quantize_rows(const uint16_t *X_dev, int64_t s, int64_t h
   act.s = s;
   act.h = h;
   act.alpha = alpha;
+  const size_t mw_bytes = align256(4 * (size_t)mask_words(h));
   act.block_counter = reinterpret_cast<int32_t *>(sb);
+  act.act_counter = reinterpret_cast<int32_t *>(sb) + 2;
   act.mask = reinterpret_cast<uint32_t *>(sb + 256);
-  act.wprefix = reinterpret_cast<int32_t *>(sb + 256 + align256(4 * (size_t)mask_words(h)));
+  act.wprefix = reinterpret_cast<int32_t *>(sb + 256 + mw_bytes);
+  act.acc_mask = reinterpret_cast<uint32_t *>(sb + 256 + mw_bytes +
+                                              align256(4 * ((size_t)mask_words(h) + 1)));
+  act.act_reset = true;  // caller scratch: state unknown
   act.idx = idx_dev;
   act.count = n_outliers_dev;
   act.flags = flags_dev;
+  act.status = reinterpret_cast<int *>(sb) + 1;
   act.Xq = Xq_dev;
   act.ax = ax_dev;
   int32_t launches = 0;
@@ -654,7 +791,7 @@ std::mutex g_noalloc_mutex;
 // Device address of the scratch array on the current device. In host code
 // the array's name is only a host-side stand-in, so the address is asked of
 // the runtime once per device (with that device current) and cached. The
-// first lookup also clears the status block, asynchronously on `st`.
+// first lookup also clears the state block, asynchronously on `st`.
 llmint8_status noalloc_scratch(cudaStream_t st, void **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
@@ -665,7 +802,7 @@ llmint8_status noalloc_scratch(cudaStream_t st, void **out) {
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
       return LLMINT8_ERR_CUDA;
-    if (cudaMemsetAsync(p, 0, 256, st) != cudaSuccess) return LLMINT8_ERR_CUDA;
+    if (cudaMemsetAsync(p, 0, kStateBytes, st) != cudaSuccess) return LLMINT8_ERR_CUDA;
     slot.ptr = p;
     slot.ready = true;
   }

@@ -14,6 +14,7 @@
 #include <cstdint>
 #include <cuda_fp16.h>
 
+#include "llmint8.h"
 #include "ptx_sm100.cuh"
 
 namespace llmint8 {
@@ -30,43 +31,48 @@ __device__ __forceinline__ int32_t absmax_code(float x, float a) {
   return static_cast<int32_t>(r);
 }
 
-// The same code without a division per element, for a row that shares one
-// scale a > 0 with r ~ 1/a (a few ulps of error are fine). With t = 127|x|
-// (exact in fp32), the candidate n = floor(t*r + 1/2) is within one of the
-// correctly rounded result; the residuals t - (n -+ 1/2) a are computed by one
-// FMA each and are exact in sign, because (n -+ 1/2) has at most 9 significant
-// bits and a at most 11, so the products are exact fp32 values. After the
-// correction (n - 1/2) a <= t < (n + 1/2) a, i.e. n rounds 127|x|/a half away
-// from zero, which is the value absmax_code() produces (its single fp32
-// division cannot move the quotient across a half-integer: the distance of
-// 127x/a from one is at least 2^-12 or q * 2^-19, above the division's error).
-__device__ __forceinline__ int32_t absmax_code_recip(float x, float a, float r) {
-  const float t = 127.0f * fabsf(x);
-  float n = floorf(fmaf(t, r, 0.5f));
-  // (n + 1/2) a > (n - 1/2) a, so at most one of the two corrections applies
-  const float below = fmaf(-(n - 0.5f), a, t) < 0.0f ? 1.0f : 0.0f;
-  const float above = fmaf(-(n + 0.5f), a, t) >= 0.0f ? 1.0f : 0.0f;
-  n = fminf(n + above - below, 127.0f);
-  return static_cast<int32_t>(copysignf(n, x));
-}
-
-// Fast form of absmax_code_recip. With r = 1/a correctly rounded, y =
-// fma(t, r, 1/2) is within 2^-16 of t/a + 1/2 (t/a <= 127: the reciprocal
-// contributes < 2^-17 and the fma rounding <= 2^-18), so when the fractional
-// part of y is at least 2^-15 away from an integer, floor(y) is already
-// floor(t/a + 1/2), the exactly rounded code. Only values that close to a
-// rounding boundary (about 6 in 10^5) take the exact two-residual correction.
-__device__ __forceinline__ int32_t absmax_code_fast(float x, float a, float r) {
-  const float t = 127.0f * fabsf(x);
-  const float y = fmaf(t, r, 0.5f);
-  const float n0 = floorf(y);
-  float n = n0;
-  if (fabsf((y - n0) - 0.5f) > 0.5f - 3.0517578125e-05f) {  // within 2^-15 of an integer
-    const float below = fmaf(-(n0 - 0.5f), a, t) < 0.0f ? 1.0f : 0.0f;
-    const float above = fmaf(-(n0 + 0.5f), a, t) >= 0.0f ? 1.0f : 0.0f;
-    n = fminf(n0 + above - below, 127.0f);
+// Codes for two binary16 values (one 32-bit word) against a row scale a > 0,
+// with r = 1/a correctly rounded and no division or conversion-unit
+// instruction per element; the result equals absmax_code(x, a).
+//  - t = 127|x| exactly: the binary16 magnitude bits shifted into fp32
+//    position encode |x| * 2^-112 (normal and subnormal alike), so one fp32
+//    multiply by 127 * 2^112 gives 127|x| (at most 18 significant bits);
+//  - m = fma(t, r, 1.5 * 2^23) rounds t*r to the nearest integer n, which
+//    then sits in the low mantissa bits of m;
+//  - d = t*r - n (one fma). t*r is within 2^-17 of t/a (t/a <= 127, r has
+//    relative error <= 2^-24), so if |d| < 1/2 - 2^-15, n is t/a rounded.
+//    Otherwise (a near-tie, about 6 values in 10^5) two residuals
+//    t - (n -+ 1/2) a, one FMA each, settle it: they are exact in sign since
+//    (n -+ 1/2) has at most 9 significant bits and a at most 11, so the
+//    products are exact fp32 values. After the correction
+//    (n - 1/2) a <= t < (n + 1/2) a, i.e. n rounds 127|x|/a half away from
+//    zero. That is also absmax_code()'s value: its one fp32 division cannot
+//    move the quotient across a half-integer, whose distance from 127x/a is
+//    at least 2^-12 or q * 2^-19, above the division's error.
+// Returns the two codes (in [-127, 127]) as ints, q0 from the low half.
+__device__ __forceinline__ void absmax_code2_noxu(uint32_t w, float a, float r, int32_t &q0,
+                                                  int32_t &q1) {
+  constexpr float kScale = 127.0f * 5192296858534827628530496329220096.0f;  // 127 * 2^112
+  constexpr float kMagic = 12582912.0f;                                      // 1.5 * 2^23
+  const uint32_t hb[2] = {w & 0xFFFFu, w >> 16};
+  int32_t q[2];
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const float t = __uint_as_float((hb[e] & 0x7FFFu) << 13) * kScale;
+    const float m = fmaf(t, r, kMagic);
+    const float nf = m - kMagic;
+    const float d = fmaf(t, r, -nf);
+    int32_t n = __float_as_int(m) - __float_as_int(kMagic);
+    if (!(fabsf(d) < 0.5f - 3.0517578125e-05f)) {
+      const float below = fmaf(-(nf - 0.5f), a, t) < 0.0f ? 1.0f : 0.0f;
+      const float above = fmaf(-(nf + 0.5f), a, t) >= 0.0f ? 1.0f : 0.0f;
+      n = __float_as_int(fminf(nf + above - below, 127.0f) + kMagic) - __float_as_int(kMagic);
+    }
+    const int32_t neg = -static_cast<int32_t>(hb[e] >> 15);  // 0 or -1
+    q[e] = (n ^ neg) - neg;
   }
-  return static_cast<int32_t>(copysignf(n, x));
+  q0 = q[0];
+  q1 = q[1];
 }
 
 __device__ __forceinline__ float half_bits_to_float(uint32_t b) {
@@ -104,15 +110,20 @@ constexpr int kColsPerBlock = kColThreads * 8;
 
 // Compaction of the bitmask into the ascending outlier list by one block:
 // word_prefix[w] = number of outlier columns before word w, idx[] = the
-// outlier columns, *count = |O|, flags[j] (optional) = bit j.
-template <int kThreads>
-__device__ void compact_outliers_block(const uint32_t *__restrict__ mask, int32_t nwords,
-                                       int32_t h, int32_t *__restrict__ word_prefix,
+// outlier columns, *count = |O|, flags[j] (optional) = bit j, mask_out
+// (optional) = a copy of the bitmask; with `clear` the bitmask itself is
+// zeroed once read. Every thread of the block calls it; its size is a
+// multiple of 32.
+__device__ void compact_outliers_block(uint32_t *__restrict__ mask, int32_t nwords, int32_t h,
+                                       int32_t *__restrict__ word_prefix,
                                        int32_t *__restrict__ idx, int32_t *__restrict__ count,
-                                       uint8_t *__restrict__ flags) {
+                                       uint8_t *__restrict__ flags,
+                                       uint32_t *__restrict__ mask_out = nullptr,
+                                       bool clear = false) {
   __shared__ int32_t warp_sums[32];
+  const int nthreads = static_cast<int>(blockDim.x);
   const int tid = threadIdx.x;
-  const int per = (nwords + kThreads - 1) / kThreads;
+  const int per = (nwords + nthreads - 1) / nthreads;
   const int w0 = tid * per;
   const int w1 = min(nwords, w0 + per);
   int32_t local = 0;
@@ -127,7 +138,7 @@ __device__ void compact_outliers_block(const uint32_t *__restrict__ mask, int32_
   if (lane == 31) warp_sums[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    int32_t v = lane < kThreads / 32 ? warp_sums[lane] : 0;
+    int32_t v = lane < nthreads / 32 ? warp_sums[lane] : 0;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
       const int32_t y = __shfl_up_sync(0xFFFFFFFFu, v, d);
@@ -139,6 +150,8 @@ __device__ void compact_outliers_block(const uint32_t *__restrict__ mask, int32_
   int32_t base = incl - local + (warp > 0 ? warp_sums[warp - 1] : 0);
   for (int w = w0; w < w1; ++w) {
     const uint32_t m = __ldcg(mask + w);
+    if (mask_out) mask_out[w] = m;
+    if (clear) mask[w] = 0u;
     word_prefix[w] = base;
     uint32_t mm = m;
     while (mm) {
@@ -153,7 +166,7 @@ __device__ void compact_outliers_block(const uint32_t *__restrict__ mask, int32_
       }
     }
   }
-  if (tid == kThreads - 1) {
+  if (tid == nthreads - 1) {
     word_prefix[nwords] = base;
     *count = base;
   }
@@ -226,7 +239,7 @@ __global__ void __launch_bounds__(kColThreads)
   __syncthreads();
   if (is_last) {
     __threadfence();
-    compact_outliers_block<kColThreads>(mask, (h + 31) / 32, h, word_prefix, idx, count,
+    compact_outliers_block(mask, (h + 31) / 32, h, word_prefix, idx, count,
                                         flags);
   }
 }
@@ -266,11 +279,7 @@ __device__ __forceinline__ void quantize_chunk(const uint4 v, uint32_t mw, int32
     for (int e = 0; e < 8; ++e) q[e] = 0;
   } else {
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[e]));
-      q[2 * e] = absmax_code_fast(f.x, a, r);
-      q[2 * e + 1] = absmax_code_fast(f.y, a, r);
-    }
+    for (int e = 0; e < 4; ++e) absmax_code2_noxu(w[e], a, r, q[2 * e], q[2 * e + 1]);
     if (mk != 0u) {
 #pragma unroll
       for (int e = 0; e < 8; ++e)
@@ -442,6 +451,385 @@ __global__ void __launch_bounds__(kRowThreads)
   for (int32_t c = lane * 8; c < h; c += 256) {
     const uint4 v = __ldg(reinterpret_cast<const uint4 *>(xr + c));
     quantize_chunk(v, __ldg(mask + (c >> 5)), c, a, r, row, n_out, word_prefix, qr, XO);
+  }
+}
+
+// ------------------------------------------- K1 in one read of X (prefill)
+// Steps 1 and 4 of "The Full LLM.int8() Algorithm" fused over a single read
+// of each row. The outlier set O is a property of all rows, so a row's
+// regular-column absmax is not known when the row is read; what is known is
+// its candidate scale
+//   a'_i = max over { j : |X_ij| < alpha } of |X_ij|.
+// Every regular column has all its values below alpha, so a_i <= a'_i, and
+// a_i == a'_i unless every column attaining a'_i is an outlier column. The
+// codes are written against a'_i; once O is complete, k_act_fixup compares
+// m_i = max over { t : |X_i,O_t| < alpha } |X_i,O_t| with a'_i: m_i < a'_i
+// proves that a regular column attains a'_i (the row's codes and scale are
+// final once its outlier columns are zeroed); m_i == a'_i > 0 sends the row
+// to an exact recomputation. Values >= alpha are coded as 0 here; they all
+// sit in outlier columns, which the fix-up zeroes in every row.
+//
+// A row belongs to a group of `wpr` warps (1 to 4): group g of the grid
+// (g = blockIdx.x * groups + group) takes rows g, g + G, ... (G groups in
+// all). One thread per group streams whole rows into the group's ring of
+// shared-memory stages with bulk copies; the group reduces with shuffles
+// and, for several warps, one named barrier, and quantises the row from
+// shared memory. Outlier column bits gather in a shared bitmask, OR-ed into
+// the global one when the CTA is done; the last CTA compacts it into the
+// outlier list.
+constexpr int kActMaxWarps = 32;
+constexpr int kActMaxGroups = 15;  // named barriers 1..15 (0 is __syncthreads)
+constexpr int kActMaxWpr = 4;
+
+struct ActRowsParams {
+  const uint16_t *X;
+  int64_t s;
+  int32_t h;
+  uint32_t thresh_bits;
+  int32_t groups;        // row groups per CTA
+  int32_t wpr;           // warps per group (blockDim.x = 32 * groups * wpr)
+  int32_t stages;        // stages per group
+  uint32_t stage_bytes;  // 2h rounded up to 128
+  uint64_t timeout_ns;
+  uint32_t *acc_mask;      // accumulation bitmask, all zero on entry and on exit
+  uint32_t *mask;          // receives the call's bitmask
+  int32_t *count;
+  int32_t *block_counter;  // zero on entry and on exit
+  int32_t *word_prefix;
+  int32_t *idx;
+  uint8_t *flags;
+  int8_t *Xq;
+  float *ax;
+  int *status;
+};
+
+// Shared memory of k_act_rows: groups * stages row buffers, the bitmask,
+// one barrier per buffer.
+__host__ __device__ constexpr uint32_t act_mask_offset(int32_t buffers, uint32_t stage_bytes) {
+  return static_cast<uint32_t>(buffers) * stage_bytes;
+}
+__host__ __device__ constexpr uint32_t act_bar_offset(int32_t buffers, uint32_t stage_bytes,
+                                                      int32_t h) {
+  return act_mask_offset(buffers, stage_bytes) + ((static_cast<uint32_t>(h + 31) / 32 + 3u) & ~3u) * 4u;
+}
+__host__ __device__ constexpr uint32_t act_smem_bytes(int32_t buffers, uint32_t stage_bytes,
+                                                      int32_t h) {
+  return act_bar_offset(buffers, stage_bytes, h) + 8u * static_cast<uint32_t>(buffers);
+}
+
+// Running maximum of binary16 magnitudes, two per word, as packed fp16 max
+// with NaN propagation: for non-NaN values it orders exactly like the
+// magnitude bit patterns, and a NaN yields a NaN pattern (above every
+// threshold), which sends the caller to its exact integer path.
+__device__ __forceinline__ uint32_t hmax2_mag(uint32_t acc, uint32_t w) {
+  const __half2 r = __hmax2_nan(*reinterpret_cast<const __half2 *>(&acc),
+                                __habs2(*reinterpret_cast<const __half2 *>(&w)));
+  return *reinterpret_cast<const uint32_t *>(&r);
+}
+
+// Eight codes (bytes, column order) of one 16-byte chunk whose magnitudes
+// are all <= a, with r = RN(127/a) (r = 0 when a == 0). With v = |x| r,
+// which is within 2^-17 of 127|x|/a, two fmas at 128.5 -+ 2^-15 give
+// y = 128 + (1/2 -+ 2^-15 + v) to 2^-17 (y lies in [128, 256), whose
+// spacing is 2^-16), and byte 2 of y's bits is floor(y - 128). When the two
+// bytes agree, z = 127|x|/a + 1/2 lies strictly between the two sums, so
+// that byte is floor(z): the magnitude rounded half away from zero, which
+// is absmax_code()'s result. Otherwise (z within about 2^-15 of an
+// integer) the chunk takes the exact two-residual correction. The sign is
+// applied bytewise: -n as a byte is (0x80 - n) ^ 0x80 for 0 <= n <= 127.
+__device__ __forceinline__ uint32_t gather_byte2(const uint64_t p01, const uint64_t p23) {
+  return prmt(prmt((uint32_t)p01, (uint32_t)(p01 >> 32), 0x0062u),
+              prmt((uint32_t)p23, (uint32_t)(p23 >> 32), 0x0062u), 0x5410u);
+}
+
+// Codes of one chunk (see above). Where the two candidates differ, the
+// result is the lower one or the next integer: it is the next one exactly
+// when 127|x| - (n + 1/2) a >= 0, a residual that one fma gives with its
+// sign exact ((n + 1/2) has at most 9 significant bits, a at most 11, so
+// the product is an exact fp32 value). Lanes whose |x| exceed a (values >=
+// alpha in outlier columns, zeroed later) get unspecified codes; nothing
+// else depends on them.
+__device__ __forceinline__ uint2 quant8_fma(const uint4 v, float a, float r) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  const uint64_t r2 = f32x2_pack(r, r);
+  const uint64_t clo = f32x2_pack(128.5f - 3.0517578125e-05f, 128.5f - 3.0517578125e-05f);
+  const uint64_t chi = f32x2_pack(128.5f + 3.0517578125e-05f, 128.5f + 3.0517578125e-05f);
+  uint64_t lo[4], hi[4], xm[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const uint32_t m = w[e] & 0x7FFF7FFFu;
+    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&m));
+    xm[e] = f32x2_pack(f.x, f.y);
+    lo[e] = f32x2_fma(xm[e], r2, clo);
+    hi[e] = f32x2_fma(xm[e], r2, chi);
+  }
+  // byte 2 of each sum; at most 0x7F for every |x| <= a, and masked so the
+  // unspecified ones cannot carry or borrow across bytes below
+  uint32_t n0 = gather_byte2(lo[0], lo[1]);
+  uint32_t n1 = gather_byte2(lo[2], lo[3]);
+  const bool near = (n0 != gather_byte2(hi[0], hi[1])) | (n1 != gather_byte2(hi[2], hi[3]));
+  n0 &= 0x7F7F7F7Fu;
+  n1 &= 0x7F7F7F7Fu;
+  if (near) {
+    const uint64_t c127 = f32x2_pack(127.0f, 127.0f);
+    const uint64_t cm = f32x2_pack(-127.5f, -127.5f);
+    const uint64_t one = f32x2_pack(1.0f, 1.0f);
+    const uint64_t na = f32x2_pack(-a, -a);
+    uint32_t up[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      // 128 + n (the sum with its fraction bits cleared), then n + 1/2
+      const uint64_t base = lo[e] & 0xFFFF0000FFFF0000ull;
+      const uint64_t half = f32x2_fma(base, one, cm);
+      const uint64_t res = f32x2_fma(half, na, f32x2_mul(xm[e], c127));
+      up[e] = (f32x2_lo(res) >= 0.0f ? 1u : 0u) | (f32x2_hi(res) >= 0.0f ? 0x100u : 0u);
+    }
+    n0 += up[0] | (up[1] << 16);
+    n1 += up[2] | (up[3] << 16);
+  }
+  const uint32_t s0 = prmt(w[0], w[1], 0xFDB9u);  // 0xFF where x < 0
+  const uint32_t s1 = prmt(w[2], w[3], 0xFDB9u);
+  const uint32_t g0 = (0x80808080u - n0) ^ 0x80808080u;
+  const uint32_t g1 = (0x80808080u - n1) ^ 0x80808080u;
+  return make_uint2((g0 & s0) | (n0 & ~s0), (g1 & s1) | (n1 & ~s1));
+}
+
+// Outlier flags of one chunk whose maximum reached the threshold: sets the
+// chunk's bits in the shared bitmask and returns the maximum magnitude bits
+// of its values below the threshold.
+__device__ __noinline__ uint32_t chunk_flags_below(const uint4 v, uint32_t thr, int32_t c,
+                                                   uint32_t *mask_s) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t f = 0, b = 0;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const uint32_t lo = w[e] & 0x7FFFu, hi = (w[e] >> 16) & 0x7FFFu;
+    f |= (lo >= thr ? 1u : 0u) << (2 * e);
+    f |= (hi >= thr ? 1u : 0u) << (2 * e + 1);
+    b = max(b, max(lo < thr ? lo : 0u, hi < thr ? hi : 0u));
+  }
+  atomicOr(mask_s + (c >> 2), f << (8 * (c & 3)));
+  return b;
+}
+
+__global__ void __launch_bounds__(kActMaxWarps * 32) k_act_rows(const ActRowsParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ uint32_t red[kActMaxWarps];
+  __shared__ int is_last;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int wpr = p.wpr, S = p.stages;
+  const int grp = warp / wpr, wig = warp - grp * wpr;  // group, warp in group
+  const uint32_t gbar = 1u + grp, gthreads = 32u * wpr;
+  const int32_t h = p.h;
+  const int32_t nwords = (h + 31) >> 5;
+  const int32_t nchunks = h >> 3;
+  const int32_t buffers = p.groups * S;
+  const uint32_t thr = p.thresh_bits;
+  uint32_t *mask_s = reinterpret_cast<uint32_t *>(smem + act_mask_offset(buffers, p.stage_bytes));
+  const uint32_t bar_g = smem_u32(smem + act_bar_offset(buffers, p.stage_bytes, h)) + 8u * grp * S;
+  const uint32_t stage_s = smem_u32(smem) + static_cast<uint32_t>(grp * S) * p.stage_bytes;
+  const uint8_t *stage_p = smem + static_cast<size_t>(grp * S) * p.stage_bytes;
+  const bool leader = wig == 0 && lane == 0;  // streams the group's rows
+  for (int32_t w = tid; w < nwords; w += blockDim.x) mask_s[w] = 0u;
+  if (leader) {
+    for (int i = 0; i < S; ++i) mbar_init(bar_g + 8u * i, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  grid_dependency_wait();
+  grid_dependency_trigger();
+
+  const int64_t G = static_cast<int64_t>(gridDim.x) * p.groups;
+  const int64_t g = static_cast<int64_t>(blockIdx.x) * p.groups + grp;
+  const int64_t nrows = g < p.s ? (p.s - g + G - 1) / G : 0;
+  const uint32_t row_bytes = 2u * static_cast<uint32_t>(h);
+  uint64_t policy = 0;
+  int64_t issued = 0;  // rows whose copy the leader has issued
+  if (leader) {
+    policy = l2_policy_evict_first();
+    for (; issued < nrows && issued < S; ++issued) {
+      const int64_t row = g + issued * G;
+      mbar_arrive_expect_tx(bar_g + 8u * (uint32_t)issued, row_bytes);
+      bulk_load_1d_hint(stage_s + (uint32_t)issued * p.stage_bytes, p.X + row * h, row_bytes,
+                        bar_g + 8u * (uint32_t)issued, policy);
+    }
+  }
+
+  const int32_t c0 = wig * 32 + lane, cstep = 32 * wpr;  // this thread's chunks
+  int64_t k = 0;
+  int st = 0;
+  uint32_t par = 0;
+  for (; k < nrows; ++k) {
+    const int64_t row = g + k * G;
+    const uint4 *rv = reinterpret_cast<const uint4 *>(stage_p + (size_t)st * p.stage_bytes);
+    const bool ok = mbar_wait_until(bar_g + 8u * st, par, p.timeout_ns);
+    // Step 1 and the candidate scale: per chunk, the packed fp16 maximum of
+    // its magnitudes; a chunk reaching the threshold (or holding a NaN)
+    // takes the exact integer path, which sets its outlier bits.
+    uint32_t run = 0;  // magnitude bits: max over values below the threshold
+    if (ok) {
+      for (int32_t c = c0; c < nchunks; c += cstep) {
+        const uint4 v = rv[c];
+        const uint32_t cm = hmax2_mag(hmax2_mag(hmax2_mag(hmax2_mag(0u, v.x), v.y), v.z), v.w);
+        const uint32_t cmax = max_halves(cm & 0x7FFF7FFFu);
+        run = max(run, cmax < thr ? cmax : chunk_flags_below(v, thr, c, mask_s));
+      }
+    }
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) run = max(run, __shfl_xor_sync(0xFFFFFFFFu, run, d));
+    if (wpr > 1) {
+      if (lane == 0) red[warp] = run;
+      if (named_barrier_or(gbar, gthreads, !ok)) break;
+      for (int i = 0; i < wpr; ++i) run = max(run, red[grp * wpr + i]);
+    } else if (__any_sync(0xFFFFFFFFu, !ok)) {
+      break;
+    }
+    const float a = half_bits_to_float(run);
+    const float r = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
+    if (leader) p.ax[row] = a;
+    // Step 4 against the candidate scale (codes of values >= alpha are
+    // overwritten by the fix-up, which zeroes every outlier column)
+    int8_t *qr = p.Xq + row * h;
+#pragma unroll 2
+    for (int32_t c = c0; c < nchunks; c += cstep)
+      *reinterpret_cast<uint2 *>(qr + 8 * c) = quant8_fma(rv[c], a, r);
+    // every thread of the group is done with this stage (and with red[])
+    if (wpr > 1) named_barrier(gbar, gthreads);
+    else __syncwarp();
+    if (leader && issued < nrows) {  // row k + S into this stage
+      const int64_t nrow = g + issued * G;
+      mbar_arrive_expect_tx(bar_g + 8u * st, row_bytes);
+      bulk_load_1d_hint(stage_s + (uint32_t)st * p.stage_bytes, p.X + nrow * h, row_bytes,
+                        bar_g + 8u * st, policy);
+      ++issued;
+    }
+    if (++st == S) {
+      st = 0;
+      par ^= 1u;
+    }
+  }
+  if (k < nrows && leader) {
+    // a stage never arrived: report it and let the copies in flight land
+    // (bounded) before the shared memory is released
+    atomicOr(p.status, LLMINT8_DEV_TIMEOUT_ROWS);
+    for (int64_t j = k; j < issued; ++j)
+      mbar_wait_until(bar_g + 8u * (uint32_t)(j % S), (uint32_t)((j / S) & 1), p.timeout_ns);
+  }
+  __syncthreads();
+  for (int32_t w = tid; w < nwords; w += blockDim.x) {
+    const uint32_t m = mask_s[w];
+    if (m) atomicOr(p.acc_mask + w, m);
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) is_last = (atomicAdd(p.block_counter, 1) == (int)gridDim.x - 1);
+  __syncthreads();
+  if (is_last) {
+    // every other CTA has flushed its bits; leave the accumulation state
+    // zero for the next call
+    __threadfence();
+    if (tid == 0) *p.block_counter = 0;
+    compact_outliers_block(p.acc_mask, nwords, h, p.word_prefix, p.idx, p.count, p.flags,
+                           p.mask, true);
+  }
+}
+
+// Completes k_act_rows once O is known (and, in the first wo_blocks blocks,
+// builds the fp16 outlier rows of W, Step 2). One warp per row:
+//   XO[i][t] = X[i][O_t]; Xq[i][O_t] = 0;
+//   m_i = max of |X[i][O_t]| below alpha; if m_i == a'_i > 0 the row's
+//   absmax over regular columns is recomputed and the row requantised.
+constexpr int kFixThreads = 256;
+constexpr int kFixRowsPerBlock = kFixThreads / 32;
+constexpr int kFixIdxCache = 64;  // outlier columns a WO block keeps in shared memory
+
+__global__ void __launch_bounds__(kFixThreads)
+    k_act_fixup(const uint16_t *__restrict__ X, int64_t s, int32_t h, uint32_t thresh_bits,
+                const uint32_t *__restrict__ mask, const int32_t *__restrict__ word_prefix,
+                const int32_t *__restrict__ idx, const int32_t *__restrict__ count,
+                int8_t *__restrict__ Xq, float *__restrict__ ax, uint16_t *__restrict__ XO,
+                const int8_t *__restrict__ wq, const float *__restrict__ aw, int32_t o,
+                uint16_t *__restrict__ WO, int32_t wo_blocks) {
+  grid_dependency_wait();
+  grid_dependency_trigger();
+  const int lane = threadIdx.x & 31;
+  // the first outlier columns, |O| and the row's scale are fetched together
+  // (only |O| decides which of them are used), so a row costs two memory
+  // round trips: these loads, then the gathers they address
+  const int32_t j_pre = lane < h ? __ldcg(idx + lane) : 0;
+  if ((int32_t)blockIdx.x < wo_blocks) {
+    // WO[t][j] for every (t, j) pair, j fastest, spread over all wo_blocks
+    // blocks so the one-byte gathers from Wq's rows keep every SM busy
+    __shared__ int32_t sidx[kFixIdxCache];
+    const int32_t n = __ldcg(count);
+    for (int32_t t = threadIdx.x; t < n && t < kFixIdxCache; t += kFixThreads)
+      sidx[t] = __ldcg(idx + t);
+    __syncthreads();
+    const int64_t pairs = static_cast<int64_t>(n) * o;
+    const int64_t stride = static_cast<int64_t>(wo_blocks) * kFixThreads;
+    for (int64_t q0 = static_cast<int64_t>(blockIdx.x) * kFixThreads + threadIdx.x; q0 < pairs;
+         q0 += 4 * stride) {
+      int32_t b[4];
+      float aj[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t q = q0 + u * stride;
+        b[u] = 0;
+        aj[u] = 0.0f;
+        if (q < pairs) {
+          const int32_t t = static_cast<int32_t>(q / o), j = static_cast<int32_t>(q - (int64_t)t * o);
+          const int32_t c = t < kFixIdxCache ? sidx[t] : __ldcg(idx + t);
+          b[u] = wq[static_cast<int64_t>(j) * h + c];
+          aj[u] = __ldg(aw + j);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t q = q0 + u * stride;
+        if (q < pairs)
+          WO[q] = __half_as_ushort(
+              __float2half_rn(__fdiv_rn(static_cast<float>(b[u]) * aj[u], 127.0f)));
+      }
+    }
+    return;
+  }
+  const int64_t row =
+      static_cast<int64_t>(blockIdx.x - wo_blocks) * kFixRowsPerBlock + (threadIdx.x >> 5);
+  if (row >= s) return;
+  const float a0 = __ldcg(ax + row);
+  const int32_t n = __ldcg(count);
+  if (n == 0) return;
+  const uint16_t *xr = X + row * h;
+  int8_t *qr = Xq + row * h;
+  uint32_t mo = 0;
+  for (int32_t t = lane; t < n; t += 32) {
+    const int32_t j = t < 32 ? j_pre : __ldcg(idx + t);
+    const uint32_t hv = xr[j];
+    if (XO) XO[row * n + t] = static_cast<uint16_t>(hv);
+    const uint32_t mag = hv & 0x7FFFu;
+    if (mag < thresh_bits) mo = max(mo, mag);
+  }
+#pragma unroll
+  for (int d = 16; d > 0; d >>= 1) mo = max(mo, __shfl_xor_sync(0xFFFFFFFFu, mo, d));
+  if (!(a0 > 0.0f && half_bits_to_float(mo) == a0)) {
+    for (int32_t t = lane; t < n; t += 32) qr[t < 32 ? j_pre : __ldcg(idx + t)] = 0;
+    return;
+  }
+  // an outlier column attains the candidate scale: exact recomputation
+  uint32_t m2 = 0;
+  for (int32_t c = lane * 8; c < h; c += 256) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(xr + c));
+    m2 = regular_absmax2(m2, v, (__ldcg(mask + (c >> 5)) >> (c & 31)) & 0xFFu);
+  }
+  uint32_t mbits = max_halves(m2);
+#pragma unroll
+  for (int d = 16; d > 0; d >>= 1) mbits = max(mbits, __shfl_xor_sync(0xFFFFFFFFu, mbits, d));
+  const float a = half_bits_to_float(mbits);
+  const float r = a > 0.0f ? __frcp_rn(a) : 0.0f;
+  if (lane == 0) ax[row] = a;
+  for (int32_t c = lane * 8; c < h; c += 256) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(xr + c));
+    quantize_chunk(v, __ldcg(mask + (c >> 5)), c, a, r, row, 0, word_prefix, qr, nullptr);
   }
 }
 

@@ -67,7 +67,8 @@ def test_workspace_size_formula(lib):
     for s, h, o in [(16, 256, 256), (2048, 4096, 4096), (8, 12288, 49152),
                     (3, 272, 784)]:
         nw = (h + 31) // 32
-        exp = (256 + a256(4 * nw) + a256(4 * (nw + 1)) + a256(4 * h)
+        state = 256 + a256(4 * ((133144 + 31) // 32))  # status + accumulation bitmask
+        exp = (state + a256(4 * nw) + a256(4 * (nw + 1)) + a256(4 * h)
                + a256(4 * s) + a256(s * h) + a256(2 * s * h) + a256(2 * h * o)
                + a256(4 * ((o + 127) // 128)) + a256(4 * 16 * o))
         assert lib.llmint8_workspace_size(s, h, o) == exp

@@ -156,6 +156,32 @@ def test_repeated_calls_are_deterministic_and_status_stays_clear():
     assert binding.llmint8_read_device_status(ws) == 0
 
 
+def test_workspace_state_carries_nothing_between_calls():
+    """One workspace, calls with different outlier sets, row counts and
+    paths in turn: each call's outlier set, codes and output are its own."""
+    rng = np.random.default_rng(77)
+    h, o = 1024, 256
+    W = workloads.random_w(rng, h, o)
+    pw, _ = gpu_prepare(W)
+    Wq_ref, aw_ref = oracle.prepare_weight(W)
+    ws = binding.Workspace(300, h, o)
+    xs = [workloads.random_x(rng, 300, h, outlier_cols=(5, 600)),
+          workloads.random_x(rng, 300, h, outlier_cols=(77,)),
+          workloads.random_x(rng, 8, h, outlier_cols=(900,)),   # decode path
+          workloads.random_x(rng, 300, h),                       # no outliers
+          workloads.random_x(rng, 131, h, outlier_cols=(5, 1000))]
+    for X in xs + xs[:2]:
+        out = binding.llmint8_matmul(to_dev(X), pw, 6.0, workspace=ws)
+        n, XO, _ = binding.llmint8_read_outlier_tiles(ws, s=X.shape[0])
+        f_ref, idx_ref, n_ref = oracle.detect_outliers(X, 6.0)
+        assert n == n_ref
+        assert np.array_equal(XO.numpy().view(np.uint16),
+                              np.ascontiguousarray(X[:, idx_ref]).view(np.uint16))
+        ref = oracle.matmul(X, Wq_ref, aw_ref, 6.0)
+        assert_close_fp16(out.cpu().numpy(), ref)
+    assert binding.llmint8_read_device_status(ws) == 0
+
+
 def test_host_buffer_entry_point_matches_device_path():
     X, W, alpha = _small_inputs(SMALL[4])
     s, h = X.shape
