@@ -69,7 +69,10 @@ struct Params {
   const float *ax;        // [s]
   const float *aw;        // [o]
   const uint16_t *XO;     // [s][n_out] fp16
-  const uint16_t *WO;     // [n_out][o] fp16
+  uint16_t *WO;           // [n_out][o] fp16, built here (Step 2, W side)
+  const int8_t *wq;       // [o][h] int8 codes of W
+  const int32_t *idx;     // outlier columns, ascending
+  int32_t *wo_counter;    // CTAs done with their share of WO; zero on entry
   const int32_t *n_out;   // device scalar |O|
   int32_t *ci;            // optional [s][o] int32
   int32_t *status;        // device status word
@@ -220,6 +223,41 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int et = threadIdx.x - EPI_WARP0 * 32;  // 0..127
     const int32_t n_out = *p.n_out;
     const int32_t n_fast = n_out < FAST_OUTLIERS ? n_out : FAST_OUTLIERS;
+    bool wo_ready = n_out == 0;
+    if (n_out > 0) {
+      // Step 2, W side: WO[t][j] = fp16(fp32(fp32(wq[j][O_t]) * aw[j]) / 127)
+      // for this CTA's share of the (t, j) pairs, while the first tile's
+      // mainloop runs; the one-byte gathers are spread over every CTA
+      const int64_t pairs = static_cast<int64_t>(n_out) * p.o;
+      const int64_t stride = static_cast<int64_t>(gridDim.x) * NUM_EPI_THREADS;
+      for (int64_t q0 = static_cast<int64_t>(blockIdx.x) * NUM_EPI_THREADS + et; q0 < pairs;
+           q0 += 4 * stride) {
+        int32_t b[4];
+        float aj[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int64_t q = q0 + u * stride;
+          b[u] = 0;
+          aj[u] = 0.0f;
+          if (q < pairs) {
+            const int32_t t = static_cast<int32_t>(q / p.o);
+            const int32_t j = static_cast<int32_t>(q - static_cast<int64_t>(t) * p.o);
+            b[u] = p.wq[static_cast<int64_t>(j) * p.h + __ldg(p.idx + t)];
+            aj[u] = __ldg(p.aw + j);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int64_t q = q0 + u * stride;
+          if (q < pairs)
+            p.WO[q] = __half_as_ushort(
+                __float2half_rn(__fdiv_rn(static_cast<float>(b[u]) * aj[u], 127.0f)));
+        }
+      }
+      __threadfence();
+      named_barrier(EPI_BARRIER, NUM_EPI_THREADS);
+      if (et == 0) atomicAdd(p.wo_counter, 1);
+    }
     float *sWO = reinterpret_cast<float *>(base + WO_OFF);         // [16][BN] fp32
     float *sAW = reinterpret_cast<float *>(base + AW_OFF);         // [BN]
     uint8_t *sOut = base + OUT_OFF + ew * OUT_STAGE_BYTES;         // [32][128 B]
@@ -232,6 +270,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int32_t n0 = n_blk * BN;
       // (1) column scales and fp16 outlier rows of this tile into shared
       //     memory, while the MMA still works on the accumulator
+      if (!wo_ready) {
+        // every CTA's share of WO is written (bounded wait)
+        bool got = true;
+        if (et == 0) {
+          const uint64_t t0 = global_timer_ns();
+          while (*reinterpret_cast<volatile int32_t *>(p.wo_counter) < (int32_t)gridDim.x) {
+            if (*abort_flag || global_timer_ns() - t0 > p.timeout_ns) {
+              got = false;
+              break;
+            }
+            __nanosleep(128);
+          }
+          if (!got && !*abort_flag) {
+            *abort_flag = 1;
+            atomicOr(p.status, LLMINT8_DEV_TIMEOUT_EPILOGUE);
+          }
+          __threadfence();
+        }
+        if (named_barrier_or(EPI_BARRIER, NUM_EPI_THREADS, !got)) break;
+        wo_ready = true;
+      }
       named_barrier(EPI_BARRIER, NUM_EPI_THREADS);  // previous tile done reading
       for (int i = et; i < BN; i += NUM_EPI_THREADS) {
         const int32_t j = n0 + i;
@@ -242,7 +301,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int c8 = (i % (BN / 8)) * 8;
         const int32_t j = n0 + c8;
         uint4 w8 = make_uint4(0u, 0u, 0u, 0u);
-        if (j < p.o) w8 = __ldg(reinterpret_cast<const uint4 *>(p.WO + (int64_t)t * p.o + j));
+        if (j < p.o) w8 = __ldcg(reinterpret_cast<const uint4 *>(p.WO + (int64_t)t * p.o + j));
         const uint32_t ww[4] = {w8.x, w8.y, w8.z, w8.w};
         float4 *dst = reinterpret_cast<float4 *>(sWO + t * BN + c8);
 #pragma unroll
@@ -313,7 +372,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint16_t *wr = p.WO + (int64_t)t * p.o;
 #pragma unroll
             for (int q = 0; q < 32; ++q) {
-              const float w = (j0 + q < p.o) ? __half2float(__ushort_as_half(wr[j0 + q])) : 0.0f;
+              const float w =
+                  (j0 + q < p.o) ? __half2float(__ushort_as_half(__ldcg(wr + j0 + q))) : 0.0f;
               ef[q] = fmaf(x, w, ef[q]);
             }
           }

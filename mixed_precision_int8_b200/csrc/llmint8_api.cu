@@ -158,11 +158,12 @@ Layout layout_for(int64_t s, int64_t h, int64_t o) {
 
 // status block: [0] device status bits, [1] |O|, [2] column-pass block
 // counter, [3] block counter of the one-read activation pass (zero between
-// calls)
+// calls), [4] CTAs of the GEMM done with their share of WO
 int32_t *status_word(void *ws) { return reinterpret_cast<int32_t *>(ws); }
 int32_t *count_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 1; }
 int32_t *block_counter_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 2; }
 int32_t *act_counter_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 3; }
+int32_t *wo_counter_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 4; }
 
 // --------------------------------------------------------- validation
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -235,6 +236,7 @@ struct ActivationArgs {
   uint32_t *acc_mask;     // one-read pass: accumulation bitmask (zero on entry
   int32_t *act_counter;   // and exit, with its block counter)
   bool act_reset;         // zero them first (their state is not known)
+  int32_t *gemm_counter;  // zeroed for the GEMM that follows (or null)
   uint8_t *flags;
   int8_t *Xq;
   float *ax;
@@ -330,19 +332,12 @@ llmint8_status enqueue_activation_fused(const DeviceInfo &dev, const ActivationA
              st, true, p);
   if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
   *launches += 1;
-  // WO blocks: enough for 16 outlier columns at four pairs per thread, at
-  // most eight per SM (larger |O| loops)
-  int64_t wo_blocks = 0;
-  if (a.WO) {
-    wo_blocks = (16 * a.o + 4 * kFixThreads - 1) / (4 * kFixThreads);
-    wo_blocks = std::min<int64_t>(std::max<int64_t>(wo_blocks, 1), 8 * (int64_t)dev.sm_count);
-  }
-  const int64_t fix_blocks = wo_blocks + (a.s + kFixRowsPerBlock - 1) / kFixRowsPerBlock;
+  const int64_t fix_blocks = (a.s + kFixRowsPerBlock - 1) / kFixRowsPerBlock;
   if (fix_blocks > 0) {
     e = launch(k_act_fixup, dim3((unsigned)fix_blocks), dim3(kFixThreads), 0, st, true, a.X,
                a.s, (int32_t)a.h, p.thresh_bits, (const uint32_t *)a.mask,
                (const int32_t *)a.wprefix, (const int32_t *)a.idx, (const int32_t *)a.count,
-               a.Xq, a.ax, a.XO, a.wq, a.aw, (int32_t)a.o, a.WO, (int32_t)wo_blocks);
+               a.Xq, a.ax, a.XO, a.gemm_counter);
     if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
     *launches += 1;
   }
@@ -369,8 +364,16 @@ llmint8_status enqueue_activation_pass(const DeviceInfo &dev, const ActivationAr
   int64_t reset_blocks = (reset_threads + 255) / 256;
   if (reset_blocks < 1) reset_blocks = 1;
   if (reset_blocks > 4 * (int64_t)dev.sm_count) reset_blocks = 4 * (int64_t)dev.sm_count;
+  // prefill: the one extra word zeroed is the GEMM's WO counter (the GEMM
+  // builds the fp16 outlier rows of W itself)
+  int32_t *zb = a.zero_buf;
+  int64_t zn = a.zero_n;
+  if (!zb && a.gemm_counter) {
+    zb = a.gemm_counter;
+    zn = 1;
+  }
   cudaError_t e = launch(k_reset_mask, dim3((unsigned)reset_blocks), dim3(256), 0, st, false,
-                         a.mask, nwords, a.count, a.block_counter, a.zero_buf, a.zero_n);
+                         a.mask, nwords, a.count, a.block_counter, zb, zn);
   if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
   const int gx = (int)((a.h + kColsPerBlock - 1) / kColsPerBlock);
   const int64_t want_blocks = 4 * (int64_t)dev.sm_count;
@@ -384,7 +387,7 @@ llmint8_status enqueue_activation_pass(const DeviceInfo &dev, const ActivationAr
              a.idx, a.flags);
   if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
   const int64_t nv = (a.h + 1023) / 1024;
-  const int64_t wo_blocks_reg = a.WO ? (a.o + kRowRegThreads - 1) / kRowRegThreads : 0;
+  const int64_t wo_blocks_reg = 0;  // WO is built by the GEMM
   if (nv <= 16 && a.s + wo_blocks_reg <= (int64_t)INT32_MAX) {
     if (nv <= 1) e = launch_rows<1>(a, wo_blocks_reg, st);
     else if (nv <= 2) e = launch_rows<2>(a, wo_blocks_reg, st);
@@ -394,7 +397,7 @@ llmint8_status enqueue_activation_pass(const DeviceInfo &dev, const ActivationAr
     else e = launch_rows<16>(a, wo_blocks_reg, st);
   } else {
     const int64_t rb = (a.s + kRowsPerBlock - 1) / kRowsPerBlock;
-    const int64_t wob = a.WO ? (a.o + kRowThreads - 1) / kRowThreads : 0;
+    const int64_t wob = 0;  // WO is built by the GEMM
     e = launch(k_rows_and_outlier_w_any, dim3((unsigned)(rb + wob)), dim3(kRowThreads), 0, st,
                true, a.X, a.s, hh, (const uint32_t *)a.mask, (const int32_t *)a.wprefix,
                (const int32_t *)a.count, a.Xq, a.ax, a.XO, a.wq, a.aw, (int32_t)a.o,
@@ -475,6 +478,7 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
   act.acc_mask = reinterpret_cast<uint32_t *>(wsb + L.acc);
   act.act_counter = act_counter_word(ws);
   act.act_reset = false;  // the workspace keeps them zero between calls
+  act.gemm_counter = use_decode ? nullptr : wo_counter_word(ws);
   act.flags = nullptr;
   act.status = status;
   act.Xq = xq;
@@ -560,6 +564,9 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
     p.aw = w->aw_dev;
     p.XO = xo;
     p.WO = wo;
+    p.wq = w->wq_dev;
+    p.idx = idx;
+    p.wo_counter = wo_counter_word(ws);
     p.n_out = count;
     p.ci = opts ? opts->ci_dev : nullptr;
     p.status = status;

@@ -734,102 +734,107 @@ __global__ void __launch_bounds__(kActMaxWarps * 32) k_act_rows(const ActRowsPar
   }
 }
 
-// Completes k_act_rows once O is known (and, in the first wo_blocks blocks,
-// builds the fp16 outlier rows of W, Step 2). One warp per row:
+// Completes k_act_rows once O is known. One warp per row:
 //   XO[i][t] = X[i][O_t]; Xq[i][O_t] = 0;
 //   m_i = max of |X[i][O_t]| below alpha; if m_i == a'_i > 0 the row's
-//   absmax over regular columns is recomputed and the row requantised.
+//   absmax over regular columns is recomputed and the row requantised by
+//   the whole block (every thread loads its chunks of the row at once).
+// Block 0 also zeroes *gemm_counter (used by the GEMM that follows).
 constexpr int kFixThreads = 256;
 constexpr int kFixRowsPerBlock = kFixThreads / 32;
-constexpr int kFixIdxCache = 64;  // outlier columns a WO block keeps in shared memory
 
 __global__ void __launch_bounds__(kFixThreads)
     k_act_fixup(const uint16_t *__restrict__ X, int64_t s, int32_t h, uint32_t thresh_bits,
                 const uint32_t *__restrict__ mask, const int32_t *__restrict__ word_prefix,
                 const int32_t *__restrict__ idx, const int32_t *__restrict__ count,
                 int8_t *__restrict__ Xq, float *__restrict__ ax, uint16_t *__restrict__ XO,
-                const int8_t *__restrict__ wq, const float *__restrict__ aw, int32_t o,
-                uint16_t *__restrict__ WO, int32_t wo_blocks) {
+                int32_t *__restrict__ gemm_counter) {
+  __shared__ int redo[kFixRowsPerBlock];
+  __shared__ uint32_t red[kFixThreads / 32];
   grid_dependency_wait();
   grid_dependency_trigger();
-  const int lane = threadIdx.x & 31;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (blockIdx.x == 0 && tid == 0 && gemm_counter) *gemm_counter = 0;
   // the first outlier columns, |O| and the row's scale are fetched together
   // (only |O| decides which of them are used), so a row costs two memory
   // round trips: these loads, then the gathers they address
   const int32_t j_pre = lane < h ? __ldcg(idx + lane) : 0;
-  if ((int32_t)blockIdx.x < wo_blocks) {
-    // WO[t][j] for every (t, j) pair, j fastest, spread over all wo_blocks
-    // blocks so the one-byte gathers from Wq's rows keep every SM busy
-    __shared__ int32_t sidx[kFixIdxCache];
-    const int32_t n = __ldcg(count);
-    for (int32_t t = threadIdx.x; t < n && t < kFixIdxCache; t += kFixThreads)
-      sidx[t] = __ldcg(idx + t);
-    __syncthreads();
-    const int64_t pairs = static_cast<int64_t>(n) * o;
-    const int64_t stride = static_cast<int64_t>(wo_blocks) * kFixThreads;
-    for (int64_t q0 = static_cast<int64_t>(blockIdx.x) * kFixThreads + threadIdx.x; q0 < pairs;
-         q0 += 4 * stride) {
-      int32_t b[4];
-      float aj[4];
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * kFixRowsPerBlock + warp;
+  const bool row_ok = row < s;
+  const float a0 = row_ok ? __ldcg(ax + row) : 0.0f;
+  const int32_t n = __ldcg(count);
+  if (n == 0) return;  // uniform over the grid
+  bool need = false;
+  if (row_ok) {
+    const uint16_t *xr = X + row * h;
+    uint32_t mo = 0;
+    for (int32_t t = lane; t < n; t += 32) {
+      const int32_t j = t < 32 ? j_pre : __ldcg(idx + t);
+      const uint32_t hv = xr[j];
+      if (XO) XO[row * n + t] = static_cast<uint16_t>(hv);
+      const uint32_t mag = hv & 0x7FFFu;
+      if (mag < thresh_bits) mo = max(mo, mag);
+    }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int64_t q = q0 + u * stride;
-        b[u] = 0;
-        aj[u] = 0.0f;
-        if (q < pairs) {
-          const int32_t t = static_cast<int32_t>(q / o), j = static_cast<int32_t>(q - (int64_t)t * o);
-          const int32_t c = t < kFixIdxCache ? sidx[t] : __ldcg(idx + t);
-          b[u] = wq[static_cast<int64_t>(j) * h + c];
-          aj[u] = __ldg(aw + j);
-        }
+    for (int d = 16; d > 0; d >>= 1) mo = max(mo, __shfl_xor_sync(0xFFFFFFFFu, mo, d));
+    need = a0 > 0.0f && half_bits_to_float(mo) == a0;
+    if (!need) {
+      int8_t *qr = Xq + row * h;
+      for (int32_t t = lane; t < n; t += 32) qr[t < 32 ? j_pre : __ldcg(idx + t)] = 0;
+    }
+  }
+  if (lane == 0) redo[warp] = need ? 1 : 0;
+  if (!__syncthreads_or(need)) return;
+  // an outlier column attains a row's candidate scale: exact recomputation
+  // of that row by the whole block
+  const int32_t nchunks = h >> 3;
+  for (int w = 0; w < kFixRowsPerBlock; ++w) {
+    if (!redo[w]) continue;
+    const int64_t r = static_cast<int64_t>(blockIdx.x) * kFixRowsPerBlock + w;
+    const uint16_t *xr = X + r * h;
+    uint32_t m2 = 0;
+    for (int32_t c0 = tid; c0 < nchunks; c0 += 8 * kFixThreads) {
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int32_t c = c0 + u * kFixThreads;
+        v[u] = c < nchunks ? __ldg(reinterpret_cast<const uint4 *>(xr) + c) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int64_t q = q0 + u * stride;
-        if (q < pairs)
-          WO[q] = __half_as_ushort(
-              __float2half_rn(__fdiv_rn(static_cast<float>(b[u]) * aj[u], 127.0f)));
+      for (int u = 0; u < 8; ++u) {
+        const int32_t c = c0 + u * kFixThreads;
+        if (c < nchunks)
+          m2 = regular_absmax2(m2, v[u], (__ldcg(mask + (c >> 2)) >> (8 * (c & 3))) & 0xFFu);
       }
     }
-    return;
-  }
-  const int64_t row =
-      static_cast<int64_t>(blockIdx.x - wo_blocks) * kFixRowsPerBlock + (threadIdx.x >> 5);
-  if (row >= s) return;
-  const float a0 = __ldcg(ax + row);
-  const int32_t n = __ldcg(count);
-  if (n == 0) return;
-  const uint16_t *xr = X + row * h;
-  int8_t *qr = Xq + row * h;
-  uint32_t mo = 0;
-  for (int32_t t = lane; t < n; t += 32) {
-    const int32_t j = t < 32 ? j_pre : __ldcg(idx + t);
-    const uint32_t hv = xr[j];
-    if (XO) XO[row * n + t] = static_cast<uint16_t>(hv);
-    const uint32_t mag = hv & 0x7FFFu;
-    if (mag < thresh_bits) mo = max(mo, mag);
-  }
+    uint32_t mbits = max_halves(m2);
 #pragma unroll
-  for (int d = 16; d > 0; d >>= 1) mo = max(mo, __shfl_xor_sync(0xFFFFFFFFu, mo, d));
-  if (!(a0 > 0.0f && half_bits_to_float(mo) == a0)) {
-    for (int32_t t = lane; t < n; t += 32) qr[t < 32 ? j_pre : __ldcg(idx + t)] = 0;
-    return;
-  }
-  // an outlier column attains the candidate scale: exact recomputation
-  uint32_t m2 = 0;
-  for (int32_t c = lane * 8; c < h; c += 256) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(xr + c));
-    m2 = regular_absmax2(m2, v, (__ldcg(mask + (c >> 5)) >> (c & 31)) & 0xFFu);
-  }
-  uint32_t mbits = max_halves(m2);
+    for (int d = 16; d > 0; d >>= 1) mbits = max(mbits, __shfl_xor_sync(0xFFFFFFFFu, mbits, d));
+    if (lane == 0) red[warp] = mbits;
+    __syncthreads();
+    mbits = red[0];
 #pragma unroll
-  for (int d = 16; d > 0; d >>= 1) mbits = max(mbits, __shfl_xor_sync(0xFFFFFFFFu, mbits, d));
-  const float a = half_bits_to_float(mbits);
-  const float r = a > 0.0f ? __frcp_rn(a) : 0.0f;
-  if (lane == 0) ax[row] = a;
-  for (int32_t c = lane * 8; c < h; c += 256) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(xr + c));
-    quantize_chunk(v, __ldcg(mask + (c >> 5)), c, a, r, row, 0, word_prefix, qr, nullptr);
+    for (int i = 1; i < kFixThreads / 32; ++i) mbits = max(mbits, red[i]);
+    const float a = half_bits_to_float(mbits);
+    const float rr = a > 0.0f ? __frcp_rn(a) : 0.0f;
+    if (tid == 0) ax[r] = a;
+    int8_t *qr = Xq + r * h;
+    for (int32_t c0 = tid; c0 < nchunks; c0 += 8 * kFixThreads) {
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int32_t c = c0 + u * kFixThreads;
+        v[u] = c < nchunks ? __ldg(reinterpret_cast<const uint4 *>(xr) + c) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int32_t c = c0 + u * kFixThreads;
+        if (c < nchunks)
+          quantize_chunk(v[u], __ldcg(mask + (c >> 2)), 8 * c, a, rr, r, 0, word_prefix, qr,
+                         nullptr);
+      }
+    }
+    __syncthreads();  // red[] is reused by the next row
   }
 }
 
