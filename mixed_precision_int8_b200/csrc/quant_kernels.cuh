@@ -920,6 +920,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
                      int32_t *__restrict__ count, float *__restrict__ ax,
                      int8_t *__restrict__ Xq, uint16_t *__restrict__ XO) {
   __shared__ float row_a[kSmallMaxRows], row_r[kSmallMaxRows];
+  __shared__ uint32_t row_m[kSmallMaxRows];
   __shared__ int32_t s_prefix[kDecodeColsPerBlock / 32];
   __shared__ int32_t red_before[kDecodeThreads / 32], red_total[kDecodeThreads / 32];
   grid_dependency_wait();
@@ -927,22 +928,50 @@ __global__ void __launch_bounds__(kDecodeThreads)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int32_t nwords = (h + 31) >> 5;
   const int32_t w_begin = blockIdx.x * (kDecodeColsPerBlock / 32);
+  // Every load of this kernel is issued before any result is used: the
+  // block's columns of X (independent of the column pass), the partial row
+  // maxima and the bitmask words, four per thread at a time.
+  const int32_t c = blockIdx.x * kDecodeColsPerBlock + tid * 8;
+  uint4 v[kSmallMaxRows];
+#pragma unroll
+  for (int i = 0; i < kSmallMaxRows; ++i)
+    if (i < s && c < h) v[i] = __ldg(reinterpret_cast<const uint4 *>(X + (int64_t)i * h + c));
+  const uint32_t mw = c < h ? __ldg(mask + (c >> 5)) : 0u;
+  const int32_t pw = w_begin + lane;  // this block's words (warp 0)
+  const uint32_t pw_bits = (warp == 0 && pw < nwords) ? __ldg(mask + pw) : 0u;
+  if (tid < kSmallMaxRows) row_m[tid] = 0u;
+  __syncthreads();
   // row scales: maximum over every column block's partial maximum
-  if (tid < s) {
-    uint32_t m = 0;
-    for (int32_t b = 0; b < col_blocks; ++b)
-      m = max(m, __ldg(partial_max + (int64_t)b * kSmallMaxRows + tid));
-    const float a = half_bits_to_float(m);
-    row_a[tid] = a;
-    row_r[tid] = a > 0.0f ? __frcp_rn(a) : 0.0f;
-    if (blockIdx.x == 0) ax[tid] = a;
+  const int32_t npm = col_blocks * kSmallMaxRows;
+  for (int32_t q0 = tid; q0 < npm; q0 += 4 * kDecodeThreads) {
+    uint32_t m[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int32_t q = q0 + u * kDecodeThreads;
+      m[u] = q < npm ? __ldg(partial_max + q) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int32_t q = q0 + u * kDecodeThreads;
+      if (q < npm && (q % kSmallMaxRows) < s && m[u]) atomicMax(row_m + (q % kSmallMaxRows), m[u]);
+    }
   }
   // outlier columns before this block, and in total
   int32_t before = 0, total = 0;
-  for (int32_t w = tid; w < nwords; w += kDecodeThreads) {
-    const int32_t pc = __popc(__ldg(mask + w));
-    total += pc;
-    if (w < w_begin) before += pc;
+  for (int32_t w0 = tid; w0 < nwords; w0 += 4 * kDecodeThreads) {
+    uint32_t bits[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int32_t w = w0 + u * kDecodeThreads;
+      bits[u] = w < nwords ? __ldg(mask + w) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int32_t w = w0 + u * kDecodeThreads;
+      const int32_t pc = __popc(bits[u]);
+      total += pc;
+      if (w < w_begin) before += pc;
+    }
   }
 #pragma unroll
   for (int d = 16; d > 0; d >>= 1) {
@@ -954,6 +983,12 @@ __global__ void __launch_bounds__(kDecodeThreads)
     red_total[warp] = total;
   }
   __syncthreads();
+  if (tid < s) {
+    const float a = half_bits_to_float(row_m[tid]);
+    row_a[tid] = a;
+    row_r[tid] = a > 0.0f ? __frcp_rn(a) : 0.0f;
+    if (blockIdx.x == 0) ax[tid] = a;
+  }
   before = 0;
   total = 0;
 #pragma unroll
@@ -963,8 +998,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
   }
   // prefix counts of this block's 32 mask words (one warp)
   if (warp == 0) {
-    const int32_t w = w_begin + lane;
-    const int32_t pc = (w < nwords) ? __popc(__ldg(mask + w)) : 0;
+    const int32_t pc = __popc(pw_bits);
     int32_t incl = pc;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
@@ -973,19 +1007,13 @@ __global__ void __launch_bounds__(kDecodeThreads)
     }
     const int32_t pre = before + incl - pc;
     s_prefix[lane] = pre;
-    if (w < nwords) word_prefix[w] = pre;
-    if (w == nwords - 1) word_prefix[nwords] = pre + pc;
+    if (pw < nwords) word_prefix[pw] = pre;
+    if (pw == nwords - 1) word_prefix[nwords] = pre + pc;
   }
   if (blockIdx.x == 0 && tid == 0) *count = total;
   __syncthreads();
   // codes and the fp16 outlier columns of this block's columns, all rows
-  const int32_t c = blockIdx.x * kDecodeColsPerBlock + tid * 8;
   if (c >= h) return;
-  const uint32_t mw = __ldg(mask + (c >> 5));
-  uint4 v[kSmallMaxRows];
-#pragma unroll
-  for (int i = 0; i < kSmallMaxRows; ++i)
-    if (i < s) v[i] = __ldg(reinterpret_cast<const uint4 *>(X + (int64_t)i * h + c));
   const int32_t *pre_local = s_prefix - w_begin;  // indexed by global word
 #pragma unroll
   for (int i = 0; i < kSmallMaxRows; ++i)
