@@ -171,9 +171,10 @@ LLMINT8_API llmint8_status llmint8_quantize_rows(const uint16_t *X_dev, int64_t 
  * outlier row of W recovered from the int8 weight (the prepared weight is
  * the only copy of W the library holds). Ci is exact; the fp16 outlier
  * product and the dequantisation use fp32 arithmetic. ws_dev must hold
- * llmint8_workspace_size(s, h, o) bytes; it may be reused across calls on
- * the same stream, not shared by calls that can overlap. |O| stays on the
- * device: the call never synchronises. */
+ * llmint8_workspace_size(s, h, o) bytes and have been cleared once with
+ * llmint8_workspace_init; it may be reused across calls on the same stream
+ * (with any s, h, o it is large enough for), not shared by calls that can
+ * overlap. |O| stays on the device: the call never synchronises. */
 LLMINT8_API llmint8_status llmint8_matmul(const uint16_t *X_dev, int64_t s,
                               const llmint8_weight *w, float alpha,
                               uint16_t *out_dev, void *ws_dev, size_t ws_bytes,
@@ -198,7 +199,8 @@ LLMINT8_API llmint8_status llmint8_matmul_host(const uint16_t *X_host, int64_t s
 /* The fp16 outlier tiles of the last llmint8_matmul on this workspace:
  * copies n_outliers (to *n_out_host), XO (fp16 [s][n], to XO_host if
  * non-NULL) and WO (fp16 [n][o], to WO_host if non-NULL) from the workspace
- * to host memory sized for n = h. Synchronises `stream`. Testing aid. */
+ * to host memory sized for n = h. s, h, o must be those of that call (the
+ * workspace layout depends on them). Synchronises `stream`. Testing aid. */
 LLMINT8_API llmint8_status llmint8_read_outlier_tiles(const void *ws_dev, size_t ws_bytes,
                                           int64_t s, int64_t h, int64_t o,
                                           int32_t *n_out_host,
