@@ -82,6 +82,7 @@ typedef enum {
 #define LLMINT8_DEV_TIMEOUT_EPILOGUE 0x4  /* epilogue gave up waiting */
 #define LLMINT8_DEV_TIMEOUT_DRAIN 0x8     /* drain after an abort timed out */
 #define LLMINT8_DEV_TIMEOUT_ROWS 0x10     /* activation row stream gave up waiting */
+#define LLMINT8_DEV_TIMEOUT_SELFTEST 0x20 /* llmint8_wait_selftest's waits ran out */
 
 /* A prepared (offline-quantised) weight. Buffers are caller-owned device
  * memory: wq_dev is int8 [o][h] (the reduction index k contiguous, i.e. the
@@ -212,6 +213,18 @@ LLMINT8_API llmint8_status llmint8_read_outlier_tiles(const void *ws_dev, size_t
  * set (bits also stored in *bits_out when non-NULL), else LLMINT8_OK. */
 LLMINT8_API llmint8_status llmint8_read_device_status(void *ws_dev, size_t ws_bytes,
                                           int32_t *bits_out, void *stream);
+
+/* Testing aid for the bounded waits every kernel of this library uses:
+ * enqueues one small kernel whose two waits can never be satisfied — an
+ * mbarrier phase that nothing completes, and a word of the workspace's
+ * state block that nothing sets (zeroed here first) — each limited to
+ * limit_ns nanoseconds (1e3 <= limit_ns <= 1e10, else LLMINT8_ERR_ARG).
+ * Both give up, the kernel sets LLMINT8_DEV_TIMEOUT_SELFTEST in the status
+ * word and returns, and the CUDA context stays usable. ws_dev is a matmul
+ * workspace (at least LLMINT8_WORKSPACE_STATE_BYTES). Asynchronous on
+ * `stream`; read the result with llmint8_read_device_status. */
+LLMINT8_API llmint8_status llmint8_wait_selftest(void *ws_dev, size_t ws_bytes,
+                                     uint64_t limit_ns, void *stream);
 
 /* Allocation-free form of llmint8_matmul (the pages have no counterpart: it
  * is a deployment convenience, not part of the method).

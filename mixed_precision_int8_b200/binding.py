@@ -80,6 +80,7 @@ def load_library():
         "llmint8_decode_max_rows": ([], _c_i64),
         "llmint8_matmul_noalloc": ([_vp, _c_i64, ctypes.POINTER(llmint8_weight),
                                     _c_f32, _vp, _vp], _c_i32),
+        "llmint8_wait_selftest": ([_vp, _sz, ctypes.c_uint64, _vp], _c_i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -95,7 +96,7 @@ EXPORTED = ("llmint8_status_string", "llmint8_workspace_size",
             "llmint8_quantize_rows", "llmint8_matmul", "llmint8_matmul_ex",
             "llmint8_matmul_host", "llmint8_read_outlier_tiles",
             "llmint8_read_device_status", "llmint8_decode_max_rows",
-            "llmint8_matmul_noalloc")
+            "llmint8_matmul_noalloc", "llmint8_wait_selftest")
 
 
 def status_string(code: int) -> str:
@@ -278,6 +279,13 @@ def llmint8_read_outlier_tiles(workspace: Workspace, s: Optional[int] = None,
         _ptr(XO), _ptr(WO), _stream(stream)))
     k = n.value
     return k, XO[: s * k].view(s, k), WO[: k * o].view(k, o)
+
+
+def llmint8_wait_selftest(workspace: Workspace, limit_ns: int = 2_000_000,
+                          stream=None) -> None:
+    """Enqueue the bounded-wait self-test (its waits run out by design)."""
+    _check("llmint8_wait_selftest", load_library().llmint8_wait_selftest(
+        _ptr(workspace.buf), workspace.nbytes, int(limit_ns), _stream(stream)))
 
 
 def llmint8_read_device_status(workspace: Workspace, stream=None) -> int:

@@ -164,6 +164,7 @@ int32_t *count_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 1; }
 int32_t *block_counter_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 2; }
 int32_t *act_counter_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 3; }
 int32_t *wo_counter_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 4; }
+constexpr int kSelftestWord = 8;  // a status-block word no kernel sets
 
 // --------------------------------------------------------- validation
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -775,6 +776,22 @@ llmint8_status llmint8_read_device_status(void *ws_dev, size_t ws_bytes, int32_t
     return LLMINT8_ERR_CUDA;
   if (bits_out) *bits_out = bits;
   return bits ? LLMINT8_ERR_DEVICE_STATUS : LLMINT8_OK;
+}
+
+llmint8_status llmint8_wait_selftest(void *ws_dev, size_t ws_bytes, uint64_t limit_ns,
+                                     void *stream) {
+  if (!ws_dev) return LLMINT8_ERR_NULL;
+  if (!aligned(ws_dev, 256)) return LLMINT8_ERR_ALIGN;
+  if (ws_bytes < kStateBytes) return LLMINT8_ERR_WORKSPACE;
+  if (limit_ns < 1000ull || limit_ns > 10000000000ull) return LLMINT8_ERR_ARG;
+  DeviceInfo *dev = nullptr;
+  llmint8_status rc = device_info(&dev);
+  if (rc) return rc;
+  cudaStream_t st = as_stream(stream);
+  int32_t *never = reinterpret_cast<int32_t *>(ws_dev) + kSelftestWord;
+  if (cudaMemsetAsync(never, 0, 4, st) != cudaSuccess) return LLMINT8_ERR_CUDA;
+  k_wait_selftest<<<1, 32, 0, st>>>(status_word(ws_dev), never, limit_ns);
+  return last_launch();
 }
 
 }  // extern "C"

@@ -1022,6 +1022,29 @@ __global__ void __launch_bounds__(kDecodeThreads)
                      XO);
 }
 
+// ------------------------------------------------------- wait self-test
+// Two waits that nothing can satisfy, each bounded like every wait of the
+// library: an mbarrier phase nobody arrives at, and a word nobody sets.
+// Both run out; the status word records it and the kernel returns.
+__global__ void k_wait_selftest(int *__restrict__ status, const int *never_set,
+                                uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const bool phase_done = mbar_wait_until(smem_u32(&bar), 0u, limit_ns);
+  bool flag_seen = false;
+  const uint64_t t0 = global_timer_ns();
+  while (!(flag_seen = (*reinterpret_cast<const volatile int *>(never_set) != 0))) {
+    if (global_timer_ns() - t0 > limit_ns) break;
+    __nanosleep(1000);
+  }
+  if (threadIdx.x == 0 && !(phase_done && flag_seen))
+    atomicOr(status, LLMINT8_DEV_TIMEOUT_SELFTEST);
+}
+
 // ------------------------------------------------------------------- K0
 // Offline weight preparation. Column absmax as binary16 magnitude bits
 // (atomicMax over row blocks), then codes written transposed ([o][h]) through

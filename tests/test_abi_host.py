@@ -88,6 +88,15 @@ def _weight(h, o, wq=FAKE, aw=FAKE):
     return binding.llmint8_weight(h, o, wq, aw)
 
 
+def test_wait_selftest_validates_its_arguments_on_the_host(lib):
+    state = 17152  # LLMINT8_WORKSPACE_STATE_BYTES
+    assert lib.llmint8_wait_selftest(None, state, 10**6, None) == -1
+    assert lib.llmint8_wait_selftest(ctypes.c_void_p((1 << 20) + 8), state, 10**6, None) == -3
+    assert lib.llmint8_wait_selftest(FAKE, state - 1, 10**6, None) == -4
+    assert lib.llmint8_wait_selftest(FAKE, state, 10, None) == -7
+    assert lib.llmint8_wait_selftest(FAKE, state, 10**11, None) == -7
+
+
 @needs_no_gpu
 @pytest.mark.parametrize("h,o", [(8, 256), (100, 256), (133160, 256),
                                  (256, 8), (256, 100)])

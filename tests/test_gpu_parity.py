@@ -182,6 +182,22 @@ def test_workspace_state_carries_nothing_between_calls():
     assert binding.llmint8_read_device_status(ws) == 0
 
 
+def test_bounded_waits_run_out_report_and_leave_the_context_usable():
+    """The wait self-test's mbarrier phase and flag are never satisfied: both
+    waits give up after their limit, the status word says so, and the next
+    call on the same workspace and stream runs normally."""
+    X, W, alpha = _small_inputs(SMALL[0])
+    pw, _ = gpu_prepare(W)
+    ws = binding.Workspace(X.shape[0], pw.h, pw.o)
+    binding.llmint8_wait_selftest(ws, limit_ns=2_000_000)
+    bits = binding.llmint8_read_device_status(ws)
+    assert bits == 0x20  # LLMINT8_DEV_TIMEOUT_SELFTEST, nothing else
+    Wq_ref, aw_ref = oracle.prepare_weight(W)
+    out = binding.llmint8_matmul(to_dev(X), pw, alpha, workspace=ws)
+    assert_close_fp16(out.cpu().numpy(), oracle.matmul(X, Wq_ref, aw_ref, alpha))
+    assert binding.llmint8_read_device_status(ws) == 0
+
+
 def test_host_buffer_entry_point_matches_device_path():
     X, W, alpha = _small_inputs(SMALL[4])
     s, h = X.shape
