@@ -42,7 +42,7 @@ def _load():
     lib.oracle_quantize_rows.argtypes = [vp, i64, i64, vp, vp, i64, vp, vp]
     lib.oracle_int8_gemm.argtypes = [vp, i64, i64, vp, i64, vp, i64, vp]
     lib.oracle_outlier_weights.argtypes = [vp, vp, i64, i64, vp, i32, vp]
-    lib.oracle_matmul.argtypes = [vp, i64, i64, vp, vp, i64, f32, vp, i64,
+    lib.oracle_matmul.argtypes = [vp, i64, i64, vp, vp, i64, vp, f32, vp, i64,
                                   vp, i64, vp, vp]
     lib.oracle_num_threads.argtypes = []
     for fn in ("oracle_prepare_weight", "oracle_detect_outliers",
@@ -165,11 +165,13 @@ def outlier_weights(Wq: np.ndarray, aw: np.ndarray,
 
 def matmul(X: np.ndarray, Wq: np.ndarray, aw: np.ndarray, alpha: float,
            rows: Optional[Sequence[int]] = None,
-           cols: Optional[Sequence[int]] = None, want_ci: bool = False):
+           cols: Optional[Sequence[int]] = None, want_ci: bool = False,
+           W16: Optional[np.ndarray] = None):
     """Full LLM.int8() output (float16) for the chosen rows x cols.
 
-    Returns out [nr, nc] float16, plus Ci int32 of the same shape when
-    ``want_ci``.
+    With ``W16`` (the fp16 weight [h, o]) the outlier rows of W are its own
+    fp16 values; without it they are recovered from Wq and aw. Returns out
+    [nr, nc] float16, plus Ci int32 of the same shape when ``want_ci``.
     """
     Xb = _bits(X)
     s, h = Xb.shape
@@ -183,8 +185,13 @@ def matmul(X: np.ndarray, Wq: np.ndarray, aw: np.ndarray, alpha: float,
     nc = o if c is None else c.shape[0]
     out = np.empty((nr, nc), dtype=np.uint16)
     Ci = np.empty((nr, nc), dtype=np.int32) if want_ci else None
-    _check(_load().oracle_matmul(_ptr(Xb), s, h, _ptr(Wq), _ptr(aw), o, alpha,
-                                 _ptr(r), nr, _ptr(c), nc, _ptr(out), _ptr(Ci)),
+    w16 = None
+    if W16 is not None:
+        w16 = _bits(W16)
+        assert w16.shape == (h, o)
+    _check(_load().oracle_matmul(_ptr(Xb), s, h, _ptr(Wq), _ptr(aw), o, _ptr(w16),
+                                 alpha, _ptr(r), nr, _ptr(c), nc, _ptr(out),
+                                 _ptr(Ci)),
            "matmul")
     out = out.view(np.float16)
     return (out, Ci) if want_ci else out

@@ -300,7 +300,10 @@ int oracle_outlier_weights(const int8_t *Wq, const float *aw, int64_t h,
  * columns `cols` (NULL = all), given the prepared weight (Wq [o][h], aw [o]).
  *
  *   1. O from all s rows of X (|x| >= alpha).
- *   2. XO = X[:, O]; WO from Wq as in oracle_outlier_weights.
+ *   2. XO = X[:, O]; WO from Wq as in oracle_outlier_weights, or, when the
+ *      caller's fp16 weight W16 ([h][o], nullable) is given, the outlier rows
+ *      of W themselves, WO[t][j] = W16[O_t][j] ([P4] "Mixed-Precision
+ *      Decomposition": the outlier part of W stays in fp16).
  *   3. E[i][j] = sum_t XO[i][t] * WO[t][j]                 (fp64)
  *   4. ax, Xq as in oracle_quantize_rows; Ci exact;
  *      D[i][j] = Ci[i][j] * ax[i] * aw[j] / (127 * 127)     (fp64)
@@ -309,9 +312,9 @@ int oracle_outlier_weights(const int8_t *Wq, const float *aw, int64_t h,
  * out is [nrows][ncols] binary16; Ci_out (nullable) receives the int32
  * accumulators of the same outputs. */
 int oracle_matmul(const uint16_t *X, int64_t s, int64_t h, const int8_t *Wq,
-                  const float *aw, int64_t o, float alpha, const int64_t *rows,
-                  int64_t nrows, const int64_t *cols, int64_t ncols,
-                  uint16_t *out, int32_t *Ci_out)
+                  const float *aw, int64_t o, const uint16_t *W16, float alpha,
+                  const int64_t *rows, int64_t nrows, const int64_t *cols,
+                  int64_t ncols, uint16_t *out, int32_t *Ci_out)
 {
     if (s < 0 || h < 0 || o < 0 || !out || (!X && s * h > 0) ||
         (!Wq && h * o > 0) || (!aw && o > 0))
@@ -344,9 +347,15 @@ int oracle_matmul(const uint16_t *X, int64_t s, int64_t h, const int8_t *Wq,
         rc = ORACLE_ERR_ARG;
         goto done;
     }
-    rc = oracle_outlier_weights(Wq, aw, h, o, idx, n, WO);
-    if (rc)
-        goto done;
+    if (W16) {
+        for (int32_t t = 0; t < n; ++t)
+            for (int64_t j = 0; j < o; ++j)
+                WO[t * o + j] = W16[(int64_t)idx[t] * o + j];
+    } else {
+        rc = oracle_outlier_weights(Wq, aw, h, o, idx, n, WO);
+        if (rc)
+            goto done;
+    }
     /* Step 4: codes and exact integer product */
     rc = oracle_quantize_rows(X, s, h, flags, rows, nrows, Xq, ax);
     if (rc)

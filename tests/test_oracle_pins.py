@@ -286,6 +286,36 @@ def test_alpha_zero_is_a_plain_fp16_product_of_the_outlier_rows():
                           ref.astype(np.float16).view(np.uint16))
 
 
+def test_exact_fp16_outlier_rows_with_alpha_zero_give_the_fp16_product():
+    # [P4] "Mixed-Precision Decomposition": the outlier part of W stays in
+    # fp16. Given the caller's fp16 W and alpha = 0, every column is an
+    # outlier column, the int8 part vanishes and the output is X . W itself
+    # (a textbook product, rounded once). h != o catches a transposed read.
+    X = workloads.random_x(RNG, 10, 64, outlier_cols=(1,))
+    W = workloads.random_w(RNG, 64, 24)
+    Wq, aw = oracle.prepare_weight(W)
+    out, Ci = oracle.matmul(X, Wq, aw, 0.0, want_ci=True, W16=W)
+    assert np.all(Ci == 0)
+    ref = X.astype(np.float64) @ W.astype(np.float64)
+    assert np.array_equal(out.view(np.uint16),
+                          ref.astype(np.float16).view(np.uint16))
+
+
+def test_exact_fp16_outlier_rows_change_nothing_without_outliers():
+    # With no outlier column the fp16 weight is never read: the output equals
+    # the recovered-rows output bit for bit; with outliers it differs.
+    X = workloads.random_x(RNG, 16, 128, scale=1.0)
+    W = workloads.random_w(RNG, 128, 40)
+    Wq, aw = oracle.prepare_weight(W)
+    a = oracle.matmul(X, Wq, aw, 6.0)
+    b = oracle.matmul(X, Wq, aw, 6.0, W16=W)
+    assert np.array_equal(a.view(np.uint16), b.view(np.uint16))
+    Xo = workloads.random_x(RNG, 16, 128, outlier_cols=(3, 70), lo=20.0, hi=60.0)
+    a = oracle.matmul(Xo, Wq, aw, 6.0)
+    b = oracle.matmul(Xo, Wq, aw, 6.0, W16=W)
+    assert not np.array_equal(a.view(np.uint16), b.view(np.uint16))
+
+
 def test_no_outlier_input_is_pure_vector_wise_int8():
     # With max |X| < alpha the outlier set is empty, so alpha has no further
     # effect: any alpha above max |X| gives the same output as alpha = +inf.
