@@ -93,6 +93,13 @@ typedef struct {
     int64_t o;
     int8_t *wq_dev;
     float *aw_dev;
+    /* Optional (NULL: off): the caller's fp16 weight W [h][o] (16-byte
+     * aligned), kept alive by the caller while the weight is in use. When
+     * set, the fp16 outlier rows of W are W's own values, WO[t][j] =
+     * W[O_t][j] ("Mixed-Precision Decomposition": the outlier part of W stays
+     * in fp16), instead of being recovered from wq. prepare_weight ignores
+     * it. */
+    const uint16_t *w16_dev;
 } llmint8_weight;
 
 /* Optional extras for llmint8_matmul_ex (all fields may be zero/NULL).

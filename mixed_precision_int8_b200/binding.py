@@ -29,7 +29,8 @@ _vp, _sz = ctypes.c_void_p, ctypes.c_size_t
 
 
 class llmint8_weight(ctypes.Structure):
-    _fields_ = [("h", _c_i64), ("o", _c_i64), ("wq_dev", _vp), ("aw_dev", _vp)]
+    _fields_ = [("h", _c_i64), ("o", _c_i64), ("wq_dev", _vp), ("aw_dev", _vp),
+                ("w16_dev", _vp)]
 
 
 class llmint8_matmul_opts(ctypes.Structure):
@@ -125,13 +126,18 @@ def _f16_dev(t: torch.Tensor, name: str):
 
 
 class PreparedWeight:
-    """Device buffers of a prepared weight: wq int8 [o,h], aw float32 [o]."""
+    """Device buffers of a prepared weight: wq int8 [o,h], aw float32 [o],
+    and optionally the fp16 weight itself (w16 [h,o], kept referenced here)
+    whose outlier rows then serve as the fp16 outlier rows of W."""
 
-    def __init__(self, wq: torch.Tensor, aw: torch.Tensor):
+    def __init__(self, wq: torch.Tensor, aw: torch.Tensor,
+                 w16: Optional[torch.Tensor] = None):
         self.wq = wq
         self.aw = aw
+        self.w16 = w16
         self.o, self.h = wq.shape
-        self.c = llmint8_weight(self.h, self.o, wq.data_ptr(), aw.data_ptr())
+        self.c = llmint8_weight(self.h, self.o, wq.data_ptr(), aw.data_ptr(),
+                                w16.data_ptr() if w16 is not None else None)
 
 
 class Workspace:
@@ -157,13 +163,17 @@ def llmint8_decode_max_rows() -> int:
     return int(load_library().llmint8_decode_max_rows())
 
 
-def llmint8_prepare_weight(W: torch.Tensor, stream=None) -> PreparedWeight:
-    """W fp16 [h,o] on the GPU -> PreparedWeight (int8 [o,h] codes + scales)."""
+def llmint8_prepare_weight(W: torch.Tensor, stream=None,
+                           keep_fp16: bool = False) -> PreparedWeight:
+    """W fp16 [h,o] on the GPU -> PreparedWeight (int8 [o,h] codes + scales).
+
+    With keep_fp16 the weight keeps W (a reference, not a copy) and the
+    layer's fp16 outlier rows of W are W's own values."""
     _f16_dev(W, "W")
     h, o = W.shape
     wq = torch.empty((o, h), dtype=torch.int8, device=W.device)
     aw = torch.empty((o,), dtype=torch.float32, device=W.device)
-    pw = PreparedWeight(wq, aw)
+    pw = PreparedWeight(wq, aw, W if keep_fp16 else None)
     _check("llmint8_prepare_weight", load_library().llmint8_prepare_weight(
         _ptr(W), h, o, ctypes.byref(pw.c), _stream(stream)))
     return pw

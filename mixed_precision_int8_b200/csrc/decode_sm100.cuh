@@ -75,6 +75,7 @@ struct Params {
   const int32_t *word_prefix;  // outlier columns before each mask word
   const uint16_t *XO;     // [s][n_out] fp16
   uint16_t *WO;           // [n_out][o] fp16, written here
+  const uint16_t *w16;    // optional fp16 W [h][o]: WO rows are its own rows
   const int32_t *n_out;
   uint16_t *out;
   int32_t *ci;            // optional exact accumulators [s][o]
@@ -314,11 +315,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const int r = lane + 32 * q;
                 const int64_t j = m_blk * BM + r;
                 if (j < p.o) {
-                  const int8_t code = static_cast<int8_t>(
-                      box[r * BOX_K + ((((cb >> 4) ^ (r & 7)) << 4) | (cb & 15))]);
-                  const float prod = static_cast<float>(code) * aw_rows[q];
-                  p.WO[(int64_t)rank * p.o + j] =
-                      __half_as_ushort(__float2half_rn(__fdiv_rn(prod, 127.0f)));
+                  if (p.w16) {  // the caller's fp16 row of W
+                    p.WO[(int64_t)rank * p.o + j] =
+                        __ldg(p.w16 + (int64_t)(k0 + cc) * p.o + j);
+                  } else {
+                    const int8_t code = static_cast<int8_t>(
+                        box[r * BOX_K + ((((cb >> 4) ^ (r & 7)) << 4) | (cb & 15))]);
+                    const float prod = static_cast<float>(code) * aw_rows[q];
+                    p.WO[(int64_t)rank * p.o + j] =
+                        __half_as_ushort(__float2half_rn(__fdiv_rn(prod, 127.0f)));
+                  }
                 }
               }
               ++rank;

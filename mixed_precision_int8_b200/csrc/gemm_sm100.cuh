@@ -71,6 +71,7 @@ struct Params {
   const uint16_t *XO;     // [s][n_out] fp16
   uint16_t *WO;           // [n_out][o] fp16, built here (Step 2, W side)
   const int8_t *wq;       // [o][h] int8 codes of W
+  const uint16_t *w16;    // optional fp16 W [h][o]: WO rows are its own rows
   const int32_t *idx;     // outlier columns, ascending
   int32_t *wo_counter;    // CTAs done with their share of WO; zero on entry
   const int32_t *n_out;   // device scalar |O|
@@ -226,12 +227,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     bool wo_ready = n_out == 0;
     if (n_out > 0) {
       // Step 2, W side: WO[t][j] = fp16(fp32(fp32(wq[j][O_t]) * aw[j]) / 127)
-      // for this CTA's share of the (t, j) pairs, while the first tile's
-      // mainloop runs; the one-byte gathers are spread over every CTA
+      // (or W[O_t][j] itself when the fp16 weight is given) for this CTA's
+      // share of the (t, j) pairs, while the first tile's mainloop runs; the
+      // one-byte gathers are spread over every CTA
       const int64_t pairs = static_cast<int64_t>(n_out) * p.o;
       const int64_t stride = static_cast<int64_t>(gridDim.x) * NUM_EPI_THREADS;
-      for (int64_t q0 = static_cast<int64_t>(blockIdx.x) * NUM_EPI_THREADS + et; q0 < pairs;
-           q0 += 4 * stride) {
+      if (p.w16) {
+        for (int64_t q = static_cast<int64_t>(blockIdx.x) * NUM_EPI_THREADS + et; q < pairs;
+             q += stride) {
+          const int32_t t = static_cast<int32_t>(q / p.o);
+          const int32_t j = static_cast<int32_t>(q - static_cast<int64_t>(t) * p.o);
+          p.WO[q] = __ldg(p.w16 + static_cast<int64_t>(__ldg(p.idx + t)) * p.o + j);
+        }
+      }
+      for (int64_t q0 = static_cast<int64_t>(blockIdx.x) * NUM_EPI_THREADS + et;
+           !p.w16 && q0 < pairs; q0 += 4 * stride) {
         int32_t b[4];
         float aj[4];
 #pragma unroll

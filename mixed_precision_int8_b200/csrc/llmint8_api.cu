@@ -413,7 +413,9 @@ llmint8_status validate_weight(const llmint8_weight *w) {
   if (!w || !w->wq_dev || !w->aw_dev) return LLMINT8_ERR_NULL;
   llmint8_status st = check_hw(w->h, w->o);
   if (st) return st;
-  if (!aligned(w->wq_dev, 16) || !aligned(w->aw_dev, 16)) return LLMINT8_ERR_ALIGN;
+  if (!aligned(w->wq_dev, 16) || !aligned(w->aw_dev, 16) ||
+      (w->w16_dev && !aligned(w->w16_dev, 16)))
+    return LLMINT8_ERR_ALIGN;
   return LLMINT8_OK;
 }
 
@@ -536,6 +538,7 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
     p.word_prefix = wprefix;
     p.XO = xo;
     p.WO = wo;
+    p.w16 = w->w16_dev;
     p.n_out = count;
     p.out = out;
     p.ci = opts ? opts->ci_dev : nullptr;
@@ -566,6 +569,7 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
     p.XO = xo;
     p.WO = wo;
     p.wq = w->wq_dev;
+    p.w16 = w->w16_dev;
     p.idx = idx;
     p.wo_counter = wo_counter_word(ws);
     p.n_out = count;

@@ -31,9 +31,9 @@ def to_dev(a: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a)).cuda()
 
 
-def gpu_prepare(W: np.ndarray):
+def gpu_prepare(W: np.ndarray, keep_fp16: bool = False):
     Wd = to_dev(W)
-    pw = binding.llmint8_prepare_weight(Wd)
+    pw = binding.llmint8_prepare_weight(Wd, keep_fp16=keep_fp16)
     return pw, Wd
 
 

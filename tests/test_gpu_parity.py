@@ -126,6 +126,41 @@ def test_matmul_small_cases(case):
     assert np.array_equal(WO.numpy().view(np.uint16), WO_ref.view(np.uint16))
 
 
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: f"{c[0]}x{c[1]}x{c[2]}a{c[4]}")
+def test_matmul_small_cases_with_fp16_outlier_rows(case):
+    """The caller's fp16 W supplies the outlier rows of W: output against the
+    oracle in the same mode, and the WO tiles equal W's rows bit for bit."""
+    X, W, alpha = _small_inputs(case, seed=5)
+    s = X.shape[0]
+    pw, Wd = gpu_prepare(W, keep_fp16=True)
+    Wq_ref, aw_ref = oracle.prepare_weight(W)
+    ref, ci_ref = oracle.matmul(X, Wq_ref, aw_ref, alpha, want_ci=True, W16=W)
+    for path in ([1, 2] if s <= 16 else [1]):
+        out, ci, ws = gpu_matmul(X, pw, alpha, path=path, want_ci=True)
+        assert np.array_equal(ci, ci_ref), f"int32 accumulators, path {path}"
+        assert_close_fp16(out, ref, f"out path {path}")
+        f_ref, idx_ref, n_ref = oracle.detect_outliers(X, alpha)
+        n, _, WO = binding.llmint8_read_outlier_tiles(ws)
+        assert n == n_ref
+        assert np.array_equal(WO.numpy().view(np.uint16),
+                              np.ascontiguousarray(W[idx_ref, :]).view(np.uint16)), path
+
+
+@pytest.mark.parametrize("name", ["opt6.7b_attn_prefill", "opt175b_decode"])
+def test_workload_matmul_with_fp16_outlier_rows(name):
+    wl, X, cols, W = workloads.make_inputs(name)
+    pw, Wd = gpu_prepare(W, keep_fp16=True)
+    rows = sample_rows(wl.s, 48)
+    c = sample_cols(wl.o, 512)
+    Wq_ref, aw_ref = oracle_prepared(W, c)
+    ref = oracle.matmul(X, Wq_ref, aw_ref, wl.alpha, rows=rows,
+                        W16=np.ascontiguousarray(W[:, c]))
+    out, _, _ = gpu_matmul(X, pw, wl.alpha)
+    assert_close_fp16(out[np.ix_(rows, c)], ref)
+    del Wd, pw
+    torch.cuda.empty_cache()
+
+
 def test_matmul_zero_rows_and_zero_weight_columns():
     rng = np.random.default_rng(9)
     X = workloads.random_x(rng, 20, 256, outlier_cols=(4, 77), row_frac=1.0)
