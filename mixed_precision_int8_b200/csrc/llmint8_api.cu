@@ -513,7 +513,8 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
                             threshold_bits(alpha), mask, partial, col_blocks, act.zero_buf,
                             act.zero_n);
     if (e0 != cudaSuccess) return LLMINT8_ERR_CUDA;
-    e0 = launch(k_decode_rowpass, dim3((unsigned)col_blocks), dim3(kDecodeThreads), 0, st, true,
+    e0 = launch(k_decode_rowpass, dim3((unsigned)col_blocks, (unsigned)s), dim3(kDecodeThreads), 0,
+                st, true,
                 X, (int32_t)s, (int32_t)h, (const uint32_t *)mask, (const uint32_t *)partial,
                 col_blocks, wprefix, count, ax, xq, xo);
     if (e0 != cudaSuccess) return LLMINT8_ERR_CUDA;

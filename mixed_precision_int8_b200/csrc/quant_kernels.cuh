@@ -913,50 +913,41 @@ __global__ void __launch_bounds__(kDecodeThreads)
   }
 }
 
+// One block per (1024-column block, row): blockIdx.y is the row, so every
+// thread quantises one 16-byte chunk and the s rows of a column block run
+// side by side. Each block reduces the row's partial maxima and the prefix
+// counts it needs itself (a few hundred words, all loaded before use).
 __global__ void __launch_bounds__(kDecodeThreads)
     k_decode_rowpass(const uint16_t *__restrict__ X, int32_t s, int32_t h,
                      const uint32_t *__restrict__ mask, const uint32_t *__restrict__ partial_max,
                      int32_t col_blocks, int32_t *__restrict__ word_prefix,
                      int32_t *__restrict__ count, float *__restrict__ ax,
                      int8_t *__restrict__ Xq, uint16_t *__restrict__ XO) {
-  __shared__ float row_a[kSmallMaxRows], row_r[kSmallMaxRows];
-  __shared__ uint32_t row_m[kSmallMaxRows];
   __shared__ int32_t s_prefix[kDecodeColsPerBlock / 32];
   __shared__ int32_t red_before[kDecodeThreads / 32], red_total[kDecodeThreads / 32];
+  __shared__ uint32_t red_max[kDecodeThreads / 32];
   grid_dependency_wait();
   grid_dependency_trigger();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int32_t row = blockIdx.y;
   const int32_t nwords = (h + 31) >> 5;
   const int32_t w_begin = blockIdx.x * (kDecodeColsPerBlock / 32);
-  // Every load of this kernel is issued before any result is used: the
-  // block's columns of X (independent of the column pass), the partial row
-  // maxima and the bitmask words, four per thread at a time.
   const int32_t c = blockIdx.x * kDecodeColsPerBlock + tid * 8;
-  uint4 v[kSmallMaxRows];
-#pragma unroll
-  for (int i = 0; i < kSmallMaxRows; ++i)
-    if (i < s && c < h) v[i] = __ldg(reinterpret_cast<const uint4 *>(X + (int64_t)i * h + c));
+  // every load first: this thread's chunk of the row (independent of the
+  // column pass), its mask word, the block's mask words (warp 0), the row's
+  // partial maxima and all mask words for the prefix counts
+  uint4 v = make_uint4(0u, 0u, 0u, 0u);
+  if (c < h) v = __ldg(reinterpret_cast<const uint4 *>(X + (int64_t)row * h + c));
   const uint32_t mw = c < h ? __ldg(mask + (c >> 5)) : 0u;
-  const int32_t pw = w_begin + lane;  // this block's words (warp 0)
+  const int32_t pw = w_begin + lane;
   const uint32_t pw_bits = (warp == 0 && pw < nwords) ? __ldg(mask + pw) : 0u;
-  if (tid < kSmallMaxRows) row_m[tid] = 0u;
-  __syncthreads();
-  // row scales: maximum over every column block's partial maximum
-  const int32_t npm = col_blocks * kSmallMaxRows;
-  for (int32_t q0 = tid; q0 < npm; q0 += 4 * kDecodeThreads) {
-    uint32_t m[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int32_t q = q0 + u * kDecodeThreads;
-      m[u] = q < npm ? __ldg(partial_max + q) : 0u;
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int32_t q = q0 + u * kDecodeThreads;
-      if (q < npm && (q % kSmallMaxRows) < s && m[u]) atomicMax(row_m + (q % kSmallMaxRows), m[u]);
-    }
+  uint32_t m = 0;
+  for (int32_t q0 = tid; q0 < col_blocks; q0 += 2 * kDecodeThreads) {
+    const int32_t q1 = q0 + kDecodeThreads;
+    const uint32_t m0 = __ldg(partial_max + (int64_t)q0 * kSmallMaxRows + row);
+    const uint32_t m1 = q1 < col_blocks ? __ldg(partial_max + (int64_t)q1 * kSmallMaxRows + row) : 0u;
+    m = max(m, max(m0, m1));
   }
-  // outlier columns before this block, and in total
   int32_t before = 0, total = 0;
   for (int32_t w0 = tid; w0 < nwords; w0 += 4 * kDecodeThreads) {
     uint32_t bits[4];
@@ -967,35 +958,35 @@ __global__ void __launch_bounds__(kDecodeThreads)
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int32_t w = w0 + u * kDecodeThreads;
       const int32_t pc = __popc(bits[u]);
       total += pc;
-      if (w < w_begin) before += pc;
+      if (w0 + u * kDecodeThreads < w_begin) before += pc;
     }
   }
 #pragma unroll
   for (int d = 16; d > 0; d >>= 1) {
     before += __shfl_xor_sync(0xFFFFFFFFu, before, d);
     total += __shfl_xor_sync(0xFFFFFFFFu, total, d);
+    m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, d));
   }
   if (lane == 0) {
     red_before[warp] = before;
     red_total[warp] = total;
+    red_max[warp] = m;
   }
   __syncthreads();
-  if (tid < s) {
-    const float a = half_bits_to_float(row_m[tid]);
-    row_a[tid] = a;
-    row_r[tid] = a > 0.0f ? __frcp_rn(a) : 0.0f;
-    if (blockIdx.x == 0) ax[tid] = a;
-  }
   before = 0;
   total = 0;
+  m = 0;
 #pragma unroll
   for (int w = 0; w < kDecodeThreads / 32; ++w) {
     before += red_before[w];
     total += red_total[w];
+    m = max(m, red_max[w]);
   }
+  // row scale (maximum over every column block's partial maximum)
+  const float a = half_bits_to_float(m);
+  if (blockIdx.x == 0 && tid == 0) ax[row] = a;
   // prefix counts of this block's 32 mask words (one warp)
   if (warp == 0) {
     const int32_t pc = __popc(pw_bits);
@@ -1007,19 +998,36 @@ __global__ void __launch_bounds__(kDecodeThreads)
     }
     const int32_t pre = before + incl - pc;
     s_prefix[lane] = pre;
-    if (pw < nwords) word_prefix[pw] = pre;
-    if (pw == nwords - 1) word_prefix[nwords] = pre + pc;
+    if (row == 0) {
+      if (pw < nwords) word_prefix[pw] = pre;
+      if (pw == nwords - 1) word_prefix[nwords] = pre + pc;
+    }
   }
-  if (blockIdx.x == 0 && tid == 0) *count = total;
+  if (row == 0 && blockIdx.x == 0 && tid == 0) *count = total;
   __syncthreads();
-  // codes and the fp16 outlier columns of this block's columns, all rows
   if (c >= h) return;
-  const int32_t *pre_local = s_prefix - w_begin;  // indexed by global word
+  // codes of this chunk (outlier columns zeroed) and its fp16 outlier entries
+  const float r = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
+  uint2 q = quant8_fma(v, a, r);
+  const uint32_t mk = (mw >> (c & 31)) & 0xFFu;
+  if (mk) {
+    const uint32_t keep_lo = ((mk & 0x1u) ? 0u : 0x000000FFu) | ((mk & 0x2u) ? 0u : 0x0000FF00u) |
+                             ((mk & 0x4u) ? 0u : 0x00FF0000u) | ((mk & 0x8u) ? 0u : 0xFF000000u);
+    const uint32_t keep_hi = ((mk & 0x10u) ? 0u : 0x000000FFu) | ((mk & 0x20u) ? 0u : 0x0000FF00u) |
+                             ((mk & 0x40u) ? 0u : 0x00FF0000u) | ((mk & 0x80u) ? 0u : 0xFF000000u);
+    q.x &= keep_lo;
+    q.y &= keep_hi;
+    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+    const int32_t *pre_local = s_prefix - w_begin;  // indexed by global word
 #pragma unroll
-  for (int i = 0; i < kSmallMaxRows; ++i)
-    if (i < s)
-      quantize_chunk(v[i], mw, c, row_a[i], row_r[i], i, total, pre_local, Xq + (int64_t)i * h,
-                     XO);
+    for (int e = 0; e < 8; ++e) {
+      if ((mk >> e) & 1u) {
+        const uint32_t hv = (e & 1) ? (w4[e >> 1] >> 16) : (w4[e >> 1] & 0xFFFFu);
+        XO[(int64_t)row * total + outlier_rank(pre_local, mw, c, e)] = static_cast<uint16_t>(hv);
+      }
+    }
+  }
+  *reinterpret_cast<uint2 *>(Xq + (int64_t)row * h + c) = q;
 }
 
 // ------------------------------------------------------- wait self-test
