@@ -345,15 +345,6 @@ llmint8_status enqueue_activation_fused(const DeviceInfo &dev, const ActivationA
   return last_launch();
 }
 
-template <int NV>
-cudaError_t launch_rows(const ActivationArgs &a, int64_t wo_blocks, cudaStream_t st) {
-  return launch(k_rows_and_outlier_w<NV>, dim3((unsigned)(a.s + wo_blocks)),
-                dim3(kRowRegThreads), 0, st, true, a.X, a.s, (int32_t)a.h,
-                (const uint32_t *)a.mask, (const int32_t *)a.wprefix, (const int32_t *)a.count,
-                a.Xq, a.ax, a.XO, a.wq, a.aw, (int32_t)a.o, (const int32_t *)a.idx, a.WO,
-                (int32_t)wo_blocks);
-}
-
 llmint8_status enqueue_activation_pass(const DeviceInfo &dev, const ActivationArgs &a,
                                        cudaStream_t st, int32_t *launches) {
   ActPlan plan;
@@ -381,31 +372,22 @@ llmint8_status enqueue_activation_pass(const DeviceInfo &dev, const ActivationAr
   int64_t gy_target = (want_blocks + gx - 1) / gx;
   int64_t rpb = (a.s + gy_target - 1) / gy_target;
   rpb = (rpb + 7) / 8 * 8;  // whole batches of eight rows in flight per thread
+  if (rpb < 8) rpb = 8;     // (s == 0: one empty block row still compacts)
   if ((a.s + rpb - 1) / rpb > 65535) rpb = (a.s + 65534) / 65535;
-  const int gy = (int)((a.s + rpb - 1) / rpb);
+  const int gy = (int)std::max<int64_t>(1, (a.s + rpb - 1) / rpb);
   e = launch(k_outlier_columns, dim3(gx, gy), dim3(kColThreads), 0, st, true, a.X, a.s, hh,
              threshold_bits(a.alpha), (int32_t)rpb, a.mask, a.count, a.block_counter, a.wprefix,
              a.idx, a.flags);
   if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
-  const int64_t nv = (a.h + 1023) / 1024;
-  const int64_t wo_blocks_reg = 0;  // WO is built by the GEMM
-  if (nv <= 16 && a.s + wo_blocks_reg <= (int64_t)INT32_MAX) {
-    if (nv <= 1) e = launch_rows<1>(a, wo_blocks_reg, st);
-    else if (nv <= 2) e = launch_rows<2>(a, wo_blocks_reg, st);
-    else if (nv <= 4) e = launch_rows<4>(a, wo_blocks_reg, st);
-    else if (nv <= 8) e = launch_rows<8>(a, wo_blocks_reg, st);
-    else if (nv <= 12) e = launch_rows<12>(a, wo_blocks_reg, st);
-    else e = launch_rows<16>(a, wo_blocks_reg, st);
-  } else {
-    const int64_t rb = (a.s + kRowsPerBlock - 1) / kRowsPerBlock;
-    const int64_t wob = 0;  // WO is built by the GEMM
-    e = launch(k_rows_and_outlier_w_any, dim3((unsigned)(rb + wob)), dim3(kRowThreads), 0, st,
-               true, a.X, a.s, hh, (const uint32_t *)a.mask, (const int32_t *)a.wprefix,
-               (const int32_t *)a.count, a.Xq, a.ax, a.XO, a.wq, a.aw, (int32_t)a.o,
-               (const int32_t *)a.idx, a.WO, (int32_t)wob);
+  *launches += 2;
+  const int64_t rb = (a.s + kRowsPerBlock - 1) / kRowsPerBlock;
+  if (rb > 0) {
+    e = launch(k_rows_any, dim3((unsigned)rb), dim3(kRowThreads), 0, st, true, a.X, a.s, hh,
+               (const uint32_t *)a.mask, (const int32_t *)a.wprefix, (const int32_t *)a.count,
+               a.Xq, a.ax, a.XO);
+    if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+    *launches += 1;
   }
-  if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
-  *launches += 3;
   return last_launch();
 }
 

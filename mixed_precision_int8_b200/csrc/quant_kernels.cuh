@@ -31,50 +31,6 @@ __device__ __forceinline__ int32_t absmax_code(float x, float a) {
   return static_cast<int32_t>(r);
 }
 
-// Codes for two binary16 values (one 32-bit word) against a row scale a > 0,
-// with r = 1/a correctly rounded and no division or conversion-unit
-// instruction per element; the result equals absmax_code(x, a).
-//  - t = 127|x| exactly: the binary16 magnitude bits shifted into fp32
-//    position encode |x| * 2^-112 (normal and subnormal alike), so one fp32
-//    multiply by 127 * 2^112 gives 127|x| (at most 18 significant bits);
-//  - m = fma(t, r, 1.5 * 2^23) rounds t*r to the nearest integer n, which
-//    then sits in the low mantissa bits of m;
-//  - d = t*r - n (one fma). t*r is within 2^-17 of t/a (t/a <= 127, r has
-//    relative error <= 2^-24), so if |d| < 1/2 - 2^-15, n is t/a rounded.
-//    Otherwise (a near-tie, about 6 values in 10^5) two residuals
-//    t - (n -+ 1/2) a, one FMA each, settle it: they are exact in sign since
-//    (n -+ 1/2) has at most 9 significant bits and a at most 11, so the
-//    products are exact fp32 values. After the correction
-//    (n - 1/2) a <= t < (n + 1/2) a, i.e. n rounds 127|x|/a half away from
-//    zero. That is also absmax_code()'s value: its one fp32 division cannot
-//    move the quotient across a half-integer, whose distance from 127x/a is
-//    at least 2^-12 or q * 2^-19, above the division's error.
-// Returns the two codes (in [-127, 127]) as ints, q0 from the low half.
-__device__ __forceinline__ void absmax_code2_noxu(uint32_t w, float a, float r, int32_t &q0,
-                                                  int32_t &q1) {
-  constexpr float kScale = 127.0f * 5192296858534827628530496329220096.0f;  // 127 * 2^112
-  constexpr float kMagic = 12582912.0f;                                      // 1.5 * 2^23
-  const uint32_t hb[2] = {w & 0xFFFFu, w >> 16};
-  int32_t q[2];
-#pragma unroll
-  for (int e = 0; e < 2; ++e) {
-    const float t = __uint_as_float((hb[e] & 0x7FFFu) << 13) * kScale;
-    const float m = fmaf(t, r, kMagic);
-    const float nf = m - kMagic;
-    const float d = fmaf(t, r, -nf);
-    int32_t n = __float_as_int(m) - __float_as_int(kMagic);
-    if (!(fabsf(d) < 0.5f - 3.0517578125e-05f)) {
-      const float below = fmaf(-(nf - 0.5f), a, t) < 0.0f ? 1.0f : 0.0f;
-      const float above = fmaf(-(nf + 0.5f), a, t) >= 0.0f ? 1.0f : 0.0f;
-      n = __float_as_int(fminf(nf + above - below, 127.0f) + kMagic) - __float_as_int(kMagic);
-    }
-    const int32_t neg = -static_cast<int32_t>(hb[e] >> 15);  // 0 or -1
-    q[e] = (n ^ neg) - neg;
-  }
-  q0 = q[0];
-  q1 = q[1];
-}
-
 __device__ __forceinline__ float half_bits_to_float(uint32_t b) {
   return __half2float(__ushort_as_half(static_cast<unsigned short>(b)));
 }
@@ -248,57 +204,12 @@ __global__ void __launch_bounds__(kColThreads)
 //   ax[i]    = max over regular columns of |X[i][j]|            (exact)
 //   Xq[i][j] = code(X[i][j], ax[i]) on regular columns, 0 on outlier ones
 //   XO[i][t] = X[i][O_t]  (fp16, row stride |O|; optional)
-// and, in the same launch, the W half of Step 2 (k_rows_and_outlier_w).
 
 // Outlier position of column c + e (its rank among the outlier columns).
 __device__ __forceinline__ int32_t outlier_rank(const int32_t *word_prefix, uint32_t mask_word,
                                                 int32_t c, int e) {
   const int bit = (c & 31) + e;
   return word_prefix[c >> 5] + __popc(mask_word & ((1u << bit) - 1u));
-}
-
-// Four codes (low bytes of a..d) packed into one word, byte 0 = a.
-__device__ __forceinline__ uint32_t pack4_bytes(int32_t a, int32_t b, int32_t c, int32_t d) {
-  const uint32_t ab = __byte_perm((uint32_t)a, (uint32_t)b, 0x0040);
-  const uint32_t cd = __byte_perm((uint32_t)c, (uint32_t)d, 0x0040);
-  return __byte_perm(ab, cd, 0x5410);
-}
-
-// Codes for one 16-byte chunk (8 columns starting at c) of row `row`, whose
-// scale is a (r ~ 1/a; a == 0 gives zero codes).
-__device__ __forceinline__ void quantize_chunk(const uint4 v, uint32_t mw, int32_t c, float a,
-                                               float r, int64_t row, int32_t n_out,
-                                               const int32_t *word_prefix,
-                                               int8_t *__restrict__ qr,
-                                               uint16_t *__restrict__ XO) {
-  const uint32_t mk = (mw >> (c & 31)) & 0xFFu;
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  int32_t q[8];
-  if (a == 0.0f) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) q[e] = 0;
-  } else {
-#pragma unroll
-    for (int e = 0; e < 4; ++e) absmax_code2_noxu(w[e], a, r, q[2 * e], q[2 * e + 1]);
-    if (mk != 0u) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e)
-        if ((mk >> e) & 1u) q[e] = 0;
-    }
-  }
-  uint2 packed;
-  packed.x = pack4_bytes(q[0], q[1], q[2], q[3]);
-  packed.y = pack4_bytes(q[4], q[5], q[6], q[7]);
-  *reinterpret_cast<uint2 *>(qr + c) = packed;
-  if (mk != 0u && XO != nullptr) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      if ((mk >> e) & 1u) {
-        const uint32_t hv = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
-        XO[row * n_out + outlier_rank(word_prefix, mw, c, e)] = static_cast<uint16_t>(hv);
-      }
-    }
-  }
 }
 
 // Running per-halfword maximum of the magnitude bits of the regular columns
@@ -320,139 +231,6 @@ __device__ __forceinline__ uint32_t regular_absmax2(uint32_t m2, const uint4 v, 
 }
 
 __device__ __forceinline__ uint32_t max_halves(uint32_t m2) { return max(m2 & 0xFFFFu, m2 >> 16); }
-
-// K2: WO[t][j] = fp16(fp32(fp32(wq[j][O_t]) * aw[j]) / 127) for one column j
-// and every outlier t. The column of the int8 weight is a strided gather (one
-// byte per 32-byte sector), so eight loads are kept in flight per thread.
-__device__ __forceinline__ void outlier_weight_rows(const int8_t *__restrict__ wq,
-                                                    const float *__restrict__ aw, int32_t h,
-                                                    int32_t o, const int32_t *__restrict__ idx,
-                                                    int32_t n, int32_t j,
-                                                    uint16_t *__restrict__ WO) {
-  if (j >= o) return;
-  const float a = __ldg(aw + j);
-  const int8_t *wr = wq + static_cast<int64_t>(j) * h;
-  for (int32_t t0 = 0; t0 < n; t0 += 8) {
-    int32_t b[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) b[u] = (t0 + u < n) ? wr[__ldg(idx + t0 + u)] : 0;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if (t0 + u < n) {
-        const float prod = static_cast<float>(b[u]) * a;
-        WO[static_cast<int64_t>(t0 + u) * o + j] =
-            __half_as_ushort(__float2half_rn(__fdiv_rn(prod, 127.0f)));
-      }
-    }
-  }
-}
-
-constexpr int kRowRegThreads = 128;  // one block per row, row held in registers
-
-// Blocks [0, wo_blocks) build the fp16 outlier rows of W for 128 columns
-// each (first, so their gather latency overlaps the rows); blocks
-// [wo_blocks, wo_blocks + s) quantise one row each, the row held in
-// registers (NV 16-byte chunks per thread, h <= NV * 1024).
-template <int NV>
-__global__ void __launch_bounds__(kRowRegThreads)
-    k_rows_and_outlier_w(const uint16_t *__restrict__ X, int64_t s, int32_t h,
-                         const uint32_t *__restrict__ mask,
-                         const int32_t *__restrict__ word_prefix,
-                         const int32_t *__restrict__ count, int8_t *__restrict__ Xq,
-                         float *__restrict__ ax, uint16_t *__restrict__ XO,
-                         const int8_t *__restrict__ wq, const float *__restrict__ aw, int32_t o,
-                         const int32_t *__restrict__ idx, uint16_t *__restrict__ WO,
-                         int32_t wo_blocks) {
-  __shared__ uint32_t red[kRowRegThreads / 32];
-  grid_dependency_wait();
-  grid_dependency_trigger();
-  const int tid = threadIdx.x;
-  if ((int32_t)blockIdx.x < wo_blocks) {
-    const int32_t j = (int32_t)blockIdx.x * kRowRegThreads + tid;
-    outlier_weight_rows(wq, aw, h, o, idx, *count, j, WO);
-    return;
-  }
-  const int64_t row = (int64_t)blockIdx.x - wo_blocks;
-  const uint16_t *xr = X + row * h;
-  uint4 v[NV];
-  uint32_t mw[NV];
-#pragma unroll
-  for (int u = 0; u < NV; ++u) {
-    const int32_t c = (u * kRowRegThreads + tid) * 8;
-    if (c < h) {
-      v[u] = __ldg(reinterpret_cast<const uint4 *>(xr + c));
-      mw[u] = __ldg(mask + (c >> 5));
-    }
-  }
-  uint32_t m2 = 0;
-#pragma unroll
-  for (int u = 0; u < NV; ++u) {
-    const int32_t c = (u * kRowRegThreads + tid) * 8;
-    if (c < h) m2 = regular_absmax2(m2, v[u], (mw[u] >> (c & 31)) & 0xFFu);
-  }
-  uint32_t mbits = max_halves(m2);
-#pragma unroll
-  for (int d = 16; d > 0; d >>= 1) mbits = max(mbits, __shfl_xor_sync(0xFFFFFFFFu, mbits, d));
-  if ((tid & 31) == 0) red[tid >> 5] = mbits;
-  __syncthreads();
-#pragma unroll
-  for (int w = 0; w < kRowRegThreads / 32; ++w) mbits = max(mbits, red[w]);
-  const float a = half_bits_to_float(mbits);
-  const float r = a > 0.0f ? __frcp_rn(a) : 0.0f;
-  if (tid == 0) ax[row] = a;
-  const int32_t n_out = (XO != nullptr) ? *count : 0;
-  int8_t *qr = Xq + row * h;
-#pragma unroll
-  for (int u = 0; u < NV; ++u) {
-    const int32_t c = (u * kRowRegThreads + tid) * 8;
-    if (c < h) quantize_chunk(v[u], mw[u], c, a, r, row, n_out, word_prefix, qr, XO);
-  }
-}
-
-// Any h: one warp per row, the row read twice (second time from L1/L2);
-// the first wo_blocks blocks build the fp16 outlier rows of W.
-constexpr int kRowThreads = 256;
-constexpr int kRowsPerBlock = kRowThreads / 32;
-
-__global__ void __launch_bounds__(kRowThreads)
-    k_rows_and_outlier_w_any(const uint16_t *__restrict__ X, int64_t s, int32_t h,
-                             const uint32_t *__restrict__ mask,
-                             const int32_t *__restrict__ word_prefix,
-                             const int32_t *__restrict__ count, int8_t *__restrict__ Xq,
-                             float *__restrict__ ax, uint16_t *__restrict__ XO,
-                             const int8_t *__restrict__ wq, const float *__restrict__ aw,
-                             int32_t o, const int32_t *__restrict__ idx,
-                             uint16_t *__restrict__ WO, int32_t wo_blocks) {
-  grid_dependency_wait();
-  grid_dependency_trigger();
-  if ((int32_t)blockIdx.x < wo_blocks) {
-    const int32_t j = (int32_t)blockIdx.x * kRowThreads + threadIdx.x;
-    outlier_weight_rows(wq, aw, h, o, idx, *count, j, WO);
-    return;
-  }
-  const int lane = threadIdx.x & 31;
-  const int64_t row =
-      static_cast<int64_t>(blockIdx.x - wo_blocks) * kRowsPerBlock + (threadIdx.x >> 5);
-  if (row >= s) return;
-  const uint16_t *xr = X + row * h;
-  uint32_t m2 = 0;
-  for (int32_t c = lane * 8; c < h; c += 256) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(xr + c));
-    m2 = regular_absmax2(m2, v, (__ldg(mask + (c >> 5)) >> (c & 31)) & 0xFFu);
-  }
-  uint32_t mbits = max_halves(m2);
-#pragma unroll
-  for (int d = 16; d > 0; d >>= 1) mbits = max(mbits, __shfl_xor_sync(0xFFFFFFFFu, mbits, d));
-  const float a = half_bits_to_float(mbits);
-  const float r = a > 0.0f ? __frcp_rn(a) : 0.0f;
-  if (lane == 0) ax[row] = a;
-  const int32_t n_out = (XO != nullptr) ? *count : 0;
-  int8_t *qr = Xq + row * h;
-  for (int32_t c = lane * 8; c < h; c += 256) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(xr + c));
-    quantize_chunk(v, __ldg(mask + (c >> 5)), c, a, r, row, n_out, word_prefix, qr, XO);
-  }
-}
 
 // ------------------------------------------- K1 in one read of X (prefill)
 // Steps 1 and 4 of "The Full LLM.int8() Algorithm" fused over a single read
@@ -592,6 +370,37 @@ __device__ __forceinline__ uint2 quant8_fma(const uint4 v, float a, float r) {
   const uint32_t g0 = (0x80808080u - n0) ^ 0x80808080u;
   const uint32_t g1 = (0x80808080u - n1) ^ 0x80808080u;
   return make_uint2((g0 & s0) | (n0 & ~s0), (g1 & s1) | (n1 & ~s1));
+}
+
+// Codes for one 16-byte chunk (8 columns starting at c) of row `row`, with
+// r = RN(127/a): quant8_fma, outlier columns zeroed, and (if XO) the fp16
+// values of the chunk's outlier columns written to XO[row][rank].
+__device__ __forceinline__ void quantize_chunk(const uint4 v, uint32_t mw, int32_t c, float a,
+                                               float r, int64_t row, int32_t n_out,
+                                               const int32_t *word_prefix,
+                                               int8_t *__restrict__ qr,
+                                               uint16_t *__restrict__ XO) {
+  const uint32_t mk = (mw >> (c & 31)) & 0xFFu;
+  uint2 q = quant8_fma(v, a, r);
+  if (mk != 0u) {
+    uint32_t keep[2] = {0u, 0u};
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (!((mk >> e) & 1u)) keep[e >> 2] |= 0xFFu << (8 * (e & 3));
+    q.x &= keep[0];
+    q.y &= keep[1];
+    if (XO != nullptr) {
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        if ((mk >> e) & 1u) {
+          const uint32_t hv = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
+          XO[row * n_out + outlier_rank(word_prefix, mw, c, e)] = static_cast<uint16_t>(hv);
+        }
+      }
+    }
+  }
+  *reinterpret_cast<uint2 *>(qr + c) = q;
 }
 
 // Outlier flags of one chunk whose maximum reached the threshold: sets the
@@ -816,7 +625,7 @@ __global__ void __launch_bounds__(kFixThreads)
 #pragma unroll
     for (int i = 1; i < kFixThreads / 32; ++i) mbits = max(mbits, red[i]);
     const float a = half_bits_to_float(mbits);
-    const float rr = a > 0.0f ? __frcp_rn(a) : 0.0f;
+    const float rr = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
     if (tid == 0) ax[r] = a;
     int8_t *qr = Xq + r * h;
     for (int32_t c0 = tid; c0 < nchunks; c0 += 8 * kFixThreads) {
@@ -835,6 +644,41 @@ __global__ void __launch_bounds__(kFixThreads)
       }
     }
     __syncthreads();  // red[] is reused by the next row
+  }
+}
+
+// Rows too long for a shared-memory stage of k_act_rows: one warp per row
+// after the column pass, the row read twice (the second time from L2).
+constexpr int kRowThreads = 256;
+constexpr int kRowsPerBlock = kRowThreads / 32;
+
+__global__ void __launch_bounds__(kRowThreads)
+    k_rows_any(const uint16_t *__restrict__ X, int64_t s, int32_t h,
+               const uint32_t *__restrict__ mask, const int32_t *__restrict__ word_prefix,
+               const int32_t *__restrict__ count, int8_t *__restrict__ Xq,
+               float *__restrict__ ax, uint16_t *__restrict__ XO) {
+  grid_dependency_wait();
+  grid_dependency_trigger();
+  const int lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerBlock + (threadIdx.x >> 5);
+  if (row >= s) return;
+  const uint16_t *xr = X + row * h;
+  uint32_t m2 = 0;
+  for (int32_t c = lane * 8; c < h; c += 256) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(xr + c));
+    m2 = regular_absmax2(m2, v, (__ldg(mask + (c >> 5)) >> (c & 31)) & 0xFFu);
+  }
+  uint32_t mbits = max_halves(m2);
+#pragma unroll
+  for (int d = 16; d > 0; d >>= 1) mbits = max(mbits, __shfl_xor_sync(0xFFFFFFFFu, mbits, d));
+  const float a = half_bits_to_float(mbits);
+  const float r = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
+  if (lane == 0) ax[row] = a;
+  const int32_t n_out = (XO != nullptr) ? *count : 0;
+  int8_t *qr = Xq + row * h;
+  for (int32_t c = lane * 8; c < h; c += 256) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(xr + c));
+    quantize_chunk(v, __ldg(mask + (c >> 5)), c, a, r, row, n_out, word_prefix, qr, XO);
   }
 }
 

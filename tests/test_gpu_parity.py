@@ -161,6 +161,36 @@ def test_workload_matmul_with_fp16_outlier_rows(name):
     torch.cuda.empty_cache()
 
 
+# rows too long for a shared-memory stage of the one-read pass (2h bytes plus
+# its bitmask above the per-CTA budget): the column-pass + row-pass kernels
+LONG_H = 108544
+
+
+def test_long_rows_quantize_bit_exact_and_empty_input():
+    rng = np.random.default_rng(31)
+    X = workloads.random_x(rng, 40, LONG_H, outlier_cols=(5, 70000, LONG_H - 1))
+    _check_quantize_rows(X, 6.0)
+    # s = 0: nothing to quantise, an empty outlier set
+    Xq, ax, flags, idx, n = binding.llmint8_quantize_rows(
+        torch.empty((0, LONG_H), dtype=torch.float16, device="cuda"), 6.0)
+    torch.cuda.synchronize()
+    assert int(n.item()) == 0 and int(flags.sum().item()) == 0
+
+
+@pytest.mark.parametrize("s", [40, 8])
+def test_long_rows_matmul(s):
+    rng = np.random.default_rng(32 + s)
+    X = workloads.random_x(rng, s, LONG_H, outlier_cols=(3, 54321))
+    W = workloads.random_w(rng, LONG_H, 256, sigma=0.01)
+    pw, _ = gpu_prepare(W)
+    Wq_ref, aw_ref = oracle.prepare_weight(W)
+    rows = sample_rows(s, 12)
+    ref, ci_ref = oracle.matmul(X, Wq_ref, aw_ref, 6.0, rows=rows, want_ci=True)
+    out, ci, _ = gpu_matmul(X, pw, 6.0, want_ci=True)
+    assert np.array_equal(ci[rows], ci_ref)
+    assert_close_fp16(out[rows], ref)
+
+
 def test_matmul_zero_rows_and_zero_weight_columns():
     rng = np.random.default_rng(9)
     X = workloads.random_x(rng, 20, 256, outlier_cols=(4, 77), row_frac=1.0)
