@@ -8,19 +8,21 @@
 //   out[i][j] = fp16( Ci[i][j] * (ax[i] / 16129) * aw[j]
 //                     + sum_t XO[i][t] * WO[t][j] )          fp32
 //
-// Structure (one persistent CTA per SM, 256 threads):
+// Structure (one persistent CTA per SM, 384 threads; setmaxnreg moves
+// registers from the first warpgroup to the two epilogue warpgroups):
 //   warp 0      TMA producer: Xq and Wq tiles (128-byte swizzle) into a
 //               4-stage shared-memory ring, completion on mbarriers
 //   warp 1      one thread issues tcgen05.mma.kind::i8 (M=128, N=256, K=32)
 //               into a TMEM accumulator; tcgen05.commit frees ring slots
 //   warp 2      allocates / frees the 512 TMEM columns (2 accumulators)
-//   warps 4-7   epilogue: stage the tile's column scales and fp16 outlier
-//               rows (as fp32) in shared memory while the MMA runs, then
-//               tcgen05.ld the int32 accumulator (each warp owns 32 TMEM
-//               lanes = 32 output rows), dequantise and add the outlier
-//               product with packed f32x2 FMAs on CUDA cores, and write fp16
-//               through a 128B-swizzled staging block with TMA stores; the
-//               other accumulator is being filled by the MMA meanwhile.
+//   warps 4-11  epilogue: before the first tile, a share of the fp16 outlier
+//               rows of W; per tile, the column scales and outlier rows (as
+//               fp32) staged in shared memory while the MMA runs, then each
+//               warp tcgen05.lds its half of the columns of its 32 TMEM lanes
+//               (= 32 output rows), dequantises and adds the outlier product
+//               with packed f32x2 FMAs on CUDA cores, and writes fp16 through
+//               a 64B-swizzled 32x32 staging block with TMA stores; the other
+//               accumulator is being filled by the MMA meanwhile.
 // Every wait is bounded by the global timer; on a timeout the CTA records a
 // status bit, drains its in-flight copies and MMAs, frees TMEM and returns.
 #pragma once
@@ -43,16 +45,18 @@ constexpr uint32_t A_STAGE_BYTES = BM * BK;
 constexpr uint32_t B_STAGE_BYTES = BN * BK;
 constexpr int NUM_ACC = 2;
 constexpr uint32_t TMEM_COLS = 512;  // NUM_ACC * BN int32 columns
-constexpr int NUM_THREADS = 256;
+constexpr int NUM_THREADS = 384;
 constexpr int EPI_WARP0 = 4;
-constexpr int NUM_EPI_THREADS = 128;
-constexpr int EPI_BARRIER = 1;       // named barrier of the 4 epilogue warps
-constexpr int OUT_BOX_COLS = 64;     // fp16 columns per TMA store (128 bytes)
+constexpr int NUM_EPI_THREADS = 256;  // 8 warps: two per TMEM lane quarter
+constexpr int EPI_BARRIER = 1;       // named barrier of the epilogue warps
+constexpr int OUT_BOX_COLS = 32;     // fp16 columns per TMA store (64 bytes)
 constexpr uint32_t OUT_STAGE_BYTES = 32 * OUT_BOX_COLS * 2;  // per epilogue warp
+constexpr int REGS_LOW = 56;         // producer / MMA warpgroup after setmaxnreg
+constexpr int REGS_HIGH = 216;       // epilogue warpgroups after setmaxnreg
 constexpr int FAST_OUTLIERS = 16;    // outlier rows kept in shared memory
 constexpr uint32_t RING_BYTES = STAGES * (A_STAGE_BYTES + B_STAGE_BYTES);
 constexpr uint32_t OUT_OFF = RING_BYTES;
-constexpr uint32_t WO_OFF = OUT_OFF + 4 * OUT_STAGE_BYTES;  // fp32 [FAST_OUTLIERS][BN]
+constexpr uint32_t WO_OFF = OUT_OFF + 8 * OUT_STAGE_BYTES;  // fp32 [FAST_OUTLIERS][BN]
 constexpr uint32_t AW_OFF = WO_OFF + FAST_OUTLIERS * BN * 4;
 constexpr uint32_t BAR_OFF = AW_OFF + BN * 4;
 constexpr size_t SMEM_BYTES = 1024 + BAR_OFF + 256;
@@ -137,7 +141,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   grid_dependency_wait();
 
   const int32_t num_tiles = p.num_m_blocks * p.num_n_blocks;
-
+  if (warp < EPI_WARP0) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_LOW));
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------ TMA producer
     uint32_t stage = 0, phase = 0;
@@ -218,9 +223,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_wait_bounded(drain_bar, 0, &never, p.status, LLMINT8_DEV_TIMEOUT_DRAIN,
                         p.timeout_ns);
     }
-  } else if (warp >= EPI_WARP0) {
+  }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_HIGH));
     // --------------------------------------------------------- epilogue
-    const int ew = warp - EPI_WARP0;  // TMEM lane quarter of this warp
+    const int ew = warp & 3;          // TMEM lane quarter of this warp
+    const int hc = (warp - EPI_WARP0) >> 2;  // which half of the tile's columns
     const int et = threadIdx.x - EPI_WARP0 * 32;  // 0..127
     const int32_t n_out = *p.n_out;
     const int32_t n_fast = n_out < FAST_OUTLIERS ? n_out : FAST_OUTLIERS;
@@ -270,7 +278,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     float *sWO = reinterpret_cast<float *>(base + WO_OFF);         // [16][BN] fp32
     float *sAW = reinterpret_cast<float *>(base + AW_OFF);         // [BN]
-    uint8_t *sOut = base + OUT_OFF + ew * OUT_STAGE_BYTES;         // [32][128 B]
+    uint8_t *sOut = base + OUT_OFF + (warp - EPI_WARP0) * OUT_STAGE_BYTES;  // [32][64 B]
     const uint32_t sOut_addr = smem_u32(sOut);
     int32_t it = 0;
     for (int32_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
@@ -337,14 +345,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                            LLMINT8_DEV_TIMEOUT_EPILOGUE, p.timeout_ns);
       if (named_barrier_or(EPI_BARRIER, NUM_EPI_THREADS, !ready)) break;
       tc_fence_after();
-      const uint32_t t_row = tmem_base + ((uint32_t)(ew * 32) << 16) + acc * BN;
+      const uint32_t t_row = tmem_base + ((uint32_t)(ew * 32) << 16) + acc * BN + hc * (BN / 2);
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = 0; c < BN / 64; ++c) {
         uint32_t v[32];
         __syncwarp();
         tmem_ld_32x32b_x32(t_row + c * 32, v);
         tmem_ld_wait();
-        if (c == BN / 32 - 1) {
+        if (c == BN / 64 - 1) {
           // the accumulator is fully read: hand it back to the MMA warp
           tc_fence_before();
           mbar_arrive(tempty_bar(acc));
@@ -358,7 +366,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int t = 0; t < FAST_OUTLIERS; ++t) {
           if (t < n_fast) {
             const uint64_t x2 = f32x2_pack(xo[t], xo[t]);
-            const float4 *wrow = reinterpret_cast<const float4 *>(sWO + t * BN + c * 32);
+            const float4 *wrow =
+                reinterpret_cast<const float4 *>(sWO + t * BN + hc * (BN / 2) + c * 32);
 #pragma unroll
             for (int q4 = 0; q4 < 8; ++q4) {
               const float4 w = wrow[q4];
@@ -367,7 +376,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
         }
-        const int32_t j0 = n0 + c * 32;
+        const int32_t j0 = n0 + hc * (BN / 2) + c * 32;
         if (n_out > FAST_OUTLIERS) {
           // outlier columns beyond the shared-memory fast path (|O| > 16)
           float ef[32];
@@ -394,7 +403,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t h2[16];  // fp16 pairs of the 32 outputs
 #pragma unroll
         for (int q4 = 0; q4 < 8; ++q4) {
-          const float4 a4 = *reinterpret_cast<const float4 *>(sAW + c * 32 + 4 * q4);
+          const float4 a4 = *reinterpret_cast<const float4 *>(sAW + hc * (BN / 2) + c * 32 + 4 * q4);
           const uint64_t sv0 = f32x2_mul(rs2, f32x2_pack(a4.x, a4.y));
           const uint64_t sv1 = f32x2_mul(rs2, f32x2_pack(a4.z, a4.w));
           const uint64_t c0 = f32x2_pack((float)(int32_t)v[4 * q4], (float)(int32_t)v[4 * q4 + 1]);
@@ -405,23 +414,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           h2[2 * q4] = f2h2(f32x2_lo(r0), f32x2_hi(r0));
           h2[2 * q4 + 1] = f2h2(f32x2_lo(r1), f32x2_hi(r1));
         }
-        // stage 32 fp16 (64 bytes) of this row into the 128B-swizzled block
-        // of 64 columns; chunk k of row r lives at 16-byte slot k ^ (r & 7)
-        const int half = c & 1;
-        if (half == 0) {
-          if (lane == 0) bulk_wait_group_read0();  // previous store has read it
-          __syncwarp();
-        }
+        // stage 32 fp16 (64 bytes) of this row into the 64B-swizzled 32x32
+        // block; chunk k of row r lives at 16-byte slot k ^ ((r / 2) % 4)
+        if (lane == 0) bulk_wait_group_read0();  // the previous store has read it
+        __syncwarp();
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8) {
-          const int chunk = half * 4 + q8;
           const uint4 h8 = make_uint4(h2[4 * q8], h2[4 * q8 + 1], h2[4 * q8 + 2], h2[4 * q8 + 3]);
-          *reinterpret_cast<uint4 *>(sOut + lane * 128 + ((chunk ^ (lane & 7)) * 16)) = h8;
+          *reinterpret_cast<uint4 *>(sOut + lane * 64 + ((q8 ^ ((lane >> 1) & 3)) * 16)) = h8;
         }
-        if (half == 1) {
-          fence_proxy_async_smem();
-          __syncwarp();
-          const int32_t bx = n0 + (c - 1) * 32, by = m_blk * BM + ew * 32;
+        fence_proxy_async_smem();
+        __syncwarp();
+        {
+          const int32_t bx = j0, by = m_blk * BM + ew * 32;
           if (lane == 0 && bx < p.o && by < p.s) {  // partial boxes are clipped by TMA
             tma_store_2d(&tmOut, sOut_addr, bx, by);
             bulk_commit_group();

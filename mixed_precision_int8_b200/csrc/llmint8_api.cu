@@ -107,6 +107,7 @@ bool make_tmap_i8(CUtensorMap *map, const void *ptr, uint64_t inner, uint64_t ro
 // [box_rows][box_inner] blocks staged with the 128-byte swizzle.
 bool make_tmap_f16(CUtensorMap *map, void *ptr, uint64_t inner, uint64_t rows,
                    uint32_t box_inner, uint32_t box_rows) {
+  const CUtensorMapSwizzle swz = box_inner * 2 == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, rows};
@@ -114,7 +115,7 @@ bool make_tmap_f16(CUtensorMap *map, void *ptr, uint64_t inner, uint64_t rows,
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, ptr, dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
