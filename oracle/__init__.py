@@ -38,15 +38,19 @@ def _load():
     lib.oracle_quantize_value.argtypes = [f32, f32]
     lib.oracle_quantize_value.restype = ctypes.c_int
     lib.oracle_prepare_weight.argtypes = [vp, i64, i64, vp, vp]
+    lib.oracle_prepare_weight_mode.argtypes = [vp, i64, i64, ctypes.c_int, vp, vp]
+    lib.oracle_quantize_rows_mode.argtypes = [vp, i64, i64, vp, vp, i64,
+                                              ctypes.c_int, vp, vp]
     lib.oracle_detect_outliers.argtypes = [vp, i64, i64, f32, vp, vp, vp]
     lib.oracle_quantize_rows.argtypes = [vp, i64, i64, vp, vp, i64, vp, vp]
     lib.oracle_int8_gemm.argtypes = [vp, i64, i64, vp, i64, vp, i64, vp]
     lib.oracle_outlier_weights.argtypes = [vp, vp, i64, i64, vp, i32, vp]
-    lib.oracle_matmul.argtypes = [vp, i64, i64, vp, vp, i64, vp, f32, vp, i64,
-                                  vp, i64, vp, vp]
+    lib.oracle_matmul.argtypes = [vp, i64, i64, vp, vp, i64, vp, f32,
+                                  ctypes.c_int, vp, i64, vp, i64, vp, vp]
     lib.oracle_num_threads.argtypes = []
-    for fn in ("oracle_prepare_weight", "oracle_detect_outliers",
-               "oracle_quantize_rows", "oracle_int8_gemm",
+    for fn in ("oracle_prepare_weight", "oracle_prepare_weight_mode",
+               "oracle_detect_outliers", "oracle_quantize_rows",
+               "oracle_quantize_rows_mode", "oracle_int8_gemm",
                "oracle_outlier_weights", "oracle_matmul",
                "oracle_num_threads"):
         getattr(lib, fn).restype = ctypes.c_int
@@ -93,13 +97,16 @@ def quantize_value(x: float, a: float) -> int:
     return int(_load().oracle_quantize_value(float(x), float(a)))
 
 
-def prepare_weight(W: np.ndarray):
-    """W float16 [h,o] -> (Wq int8 [o,h], aw float32 [o])."""
+def prepare_weight(W: np.ndarray, tensor: bool = False):
+    """W float16 [h,o] -> (Wq int8 [o,h], aw float32 [o]).
+
+    tensor: one absmax constant for the whole weight (every aw[j] equal)."""
     Wb = _bits(W)
     h, o = Wb.shape
     Wq = np.empty((o, h), dtype=np.int8)
     aw = np.empty((o,), dtype=np.float32)
-    _check(_load().oracle_prepare_weight(_ptr(Wb), h, o, _ptr(Wq), _ptr(aw)),
+    _check(_load().oracle_prepare_weight_mode(_ptr(Wb), h, o, int(bool(tensor)),
+                                              _ptr(Wq), _ptr(aw)),
            "prepare_weight")
     return Wq, aw
 
@@ -119,8 +126,10 @@ def detect_outliers(X: np.ndarray, alpha: float):
 
 
 def quantize_rows(X: np.ndarray, flags: np.ndarray,
-                  rows: Optional[Sequence[int]] = None):
-    """Row scales and codes for the given rows -> (Xq int8 [r,h], ax f32 [r])."""
+                  rows: Optional[Sequence[int]] = None, tensor: bool = False):
+    """Row scales and codes for the given rows -> (Xq int8 [r,h], ax f32 [r]).
+
+    tensor: one absmax constant for all of X (every ax[r] equal)."""
     Xb = _bits(X)
     s, h = Xb.shape
     flags = np.ascontiguousarray(flags, dtype=np.uint8)
@@ -128,8 +137,8 @@ def quantize_rows(X: np.ndarray, flags: np.ndarray,
     nr = s if r is None else r.shape[0]
     Xq = np.empty((nr, h), dtype=np.int8)
     ax = np.empty((nr,), dtype=np.float32)
-    _check(_load().oracle_quantize_rows(_ptr(Xb), s, h, _ptr(flags), _ptr(r),
-                                        nr, _ptr(Xq), _ptr(ax)),
+    _check(_load().oracle_quantize_rows_mode(_ptr(Xb), s, h, _ptr(flags), _ptr(r),
+                                             nr, int(bool(tensor)), _ptr(Xq), _ptr(ax)),
            "quantize_rows")
     return Xq, ax
 
@@ -166,11 +175,14 @@ def outlier_weights(Wq: np.ndarray, aw: np.ndarray,
 def matmul(X: np.ndarray, Wq: np.ndarray, aw: np.ndarray, alpha: float,
            rows: Optional[Sequence[int]] = None,
            cols: Optional[Sequence[int]] = None, want_ci: bool = False,
-           W16: Optional[np.ndarray] = None):
+           W16: Optional[np.ndarray] = None, x_tensor: bool = False):
     """Full LLM.int8() output (float16) for the chosen rows x cols.
 
     With ``W16`` (the fp16 weight [h, o]) the outlier rows of W are its own
-    fp16 values; without it they are recovered from Wq and aw. Returns out
+    fp16 values; without it they are recovered from Wq and aw. With
+    ``x_tensor`` X is quantised with one constant for the whole tensor (the
+    tensor-wise baseline; pair it with a ``prepare_weight(W, tensor=True)``
+    weight for tensor-wise W). Returns out
     [nr, nc] float16, plus Ci int32 of the same shape when ``want_ci``.
     """
     Xb = _bits(X)
@@ -190,8 +202,8 @@ def matmul(X: np.ndarray, Wq: np.ndarray, aw: np.ndarray, alpha: float,
         w16 = _bits(W16)
         assert w16.shape == (h, o)
     _check(_load().oracle_matmul(_ptr(Xb), s, h, _ptr(Wq), _ptr(aw), o, _ptr(w16),
-                                 alpha, _ptr(r), nr, _ptr(c), nc, _ptr(out),
-                                 _ptr(Ci)),
+                                 alpha, int(bool(x_tensor)), _ptr(r), nr, _ptr(c), nc,
+                                 _ptr(out), _ptr(Ci)),
            "matmul")
     out = out.view(np.float16)
     return (out, Ci) if want_ci else out

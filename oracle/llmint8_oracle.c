@@ -145,8 +145,11 @@ int oracle_quantize_value(float x, float a)
  * h rows: aw[j] = max_k |W[k][j]|; Wq[j][k] = Q(W[k][j], aw[j]).
  * W is [h][o] row-major binary16; Wq is stored transposed, [o][h]
  * (the reduction dimension k contiguous); aw is [o] fp32. */
-int oracle_prepare_weight(const uint16_t *W, int64_t h, int64_t o,
-                          int8_t *Wq, float *aw)
+/* With `tensor` set, the baseline of [P4] "Quantization Primitives" (absmax
+ * over the whole tensor, the Table 1 "Int8 absmax" / row-wise weight side):
+ * one constant, the largest |W| of all, for every column. */
+int oracle_prepare_weight_mode(const uint16_t *W, int64_t h, int64_t o,
+                               int tensor, int8_t *Wq, float *aw)
 {
     if (!W || !Wq || !aw || h < 0 || o < 0)
         return ORACLE_ERR_ARG;
@@ -159,6 +162,14 @@ int oracle_prepare_weight(const uint16_t *W, int64_t h, int64_t o,
         }
         aw[j] = (float)m; /* a binary16 value: exact in fp32 */
     }
+    if (tensor) {
+        float m = 0.0f;
+        for (int64_t j = 0; j < o; ++j)
+            if (aw[j] > m)
+                m = aw[j];
+        for (int64_t j = 0; j < o; ++j)
+            aw[j] = m;
+    }
 #pragma omp parallel for schedule(static)
     for (int64_t j = 0; j < o; ++j) {
         for (int64_t k = 0; k < h; ++k) {
@@ -167,6 +178,12 @@ int oracle_prepare_weight(const uint16_t *W, int64_t h, int64_t o,
         }
     }
     return ORACLE_OK;
+}
+
+int oracle_prepare_weight(const uint16_t *W, int64_t h, int64_t o,
+                          int8_t *Wq, float *aw)
+{
+    return oracle_prepare_weight_mode(W, h, o, 0, Wq, aw);
 }
 
 /* ------------------------------------------------------ Step 1: detection */
@@ -207,26 +224,43 @@ int oracle_detect_outliers(const uint16_t *X, int64_t s, int64_t h,
  * |X[i][j]| (0 when there is none), Xq[i][j] = Q(X[i][j], ax[i]) on
  * non-outlier columns and 0 on outlier columns. Rows are taken from `rows`
  * (nrows of them; all rows when rows == NULL); output row r is rows[r]. */
-int oracle_quantize_rows(const uint16_t *X, int64_t s, int64_t h,
-                         const uint8_t *flags, const int64_t *rows,
-                         int64_t nrows, int8_t *Xq, float *ax)
+/* Largest |X[i][j]| over the non-outlier columns of row i. */
+static double regular_absmax(const uint16_t *X, int64_t h, const uint8_t *flags, int64_t i)
+{
+    double m = 0.0;
+    for (int64_t j = 0; j < h; ++j) {
+        if (flags[j])
+            continue;
+        double v = fabs(oracle_half_to_double(X[i * h + j]));
+        if (v > m)
+            m = v;
+    }
+    return m;
+}
+
+/* With `tensor` set, the tensor-wise baseline of [P4] "Quantization
+ * Primitives" on the activation side: one constant for all of X (the
+ * largest regular |X| of every row), so ax[r] is that constant for every
+ * row. */
+int oracle_quantize_rows_mode(const uint16_t *X, int64_t s, int64_t h,
+                              const uint8_t *flags, const int64_t *rows,
+                              int64_t nrows, int tensor, int8_t *Xq, float *ax)
 {
     if ((!X && s * h > 0) || !flags || !ax || s < 0 || h < 0)
         return ORACLE_ERR_ARG;
     if (!rows)
         nrows = s;
+    double all = 0.0;
+    if (tensor)
+        for (int64_t i = 0; i < s; ++i) {
+            double m = regular_absmax(X, h, flags, i);
+            if (m > all)
+                all = m;
+        }
 #pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < nrows; ++r) {
         int64_t i = rows ? rows[r] : r;
-        double m = 0.0;
-        for (int64_t j = 0; j < h; ++j) {
-            if (flags[j])
-                continue;
-            double v = fabs(oracle_half_to_double(X[i * h + j]));
-            if (v > m)
-                m = v;
-        }
-        ax[r] = (float)m;
+        ax[r] = (float)(tensor ? all : regular_absmax(X, h, flags, i));
         if (Xq) {
             for (int64_t j = 0; j < h; ++j) {
                 float x = (float)oracle_half_to_double(X[i * h + j]);
@@ -236,6 +270,13 @@ int oracle_quantize_rows(const uint16_t *X, int64_t s, int64_t h,
         }
     }
     return ORACLE_OK;
+}
+
+int oracle_quantize_rows(const uint16_t *X, int64_t s, int64_t h,
+                         const uint8_t *flags, const int64_t *rows,
+                         int64_t nrows, int8_t *Xq, float *ax)
+{
+    return oracle_quantize_rows_mode(X, s, h, flags, rows, nrows, 0, Xq, ax);
 }
 
 /* ------------------------------------------------ Step 4: int8 x int8 sum */
@@ -309,12 +350,16 @@ int oracle_outlier_weights(const int8_t *Wq, const float *aw, int64_t h,
  *      D[i][j] = Ci[i][j] * ax[i] * aw[j] / (127 * 127)     (fp64)
  *   5. out[i][j] = fp16(D[i][j] + E[i][j])                  (one rounding)
  *
+ * With x_tensor, step 4 uses one constant for all of X (the tensor-wise
+ * baseline, see oracle_quantize_rows_mode); a tensor-wise W is a prepared
+ * weight from oracle_prepare_weight_mode.
+ *
  * out is [nrows][ncols] binary16; Ci_out (nullable) receives the int32
  * accumulators of the same outputs. */
 int oracle_matmul(const uint16_t *X, int64_t s, int64_t h, const int8_t *Wq,
                   const float *aw, int64_t o, const uint16_t *W16, float alpha,
-                  const int64_t *rows, int64_t nrows, const int64_t *cols,
-                  int64_t ncols, uint16_t *out, int32_t *Ci_out)
+                  int x_tensor, const int64_t *rows, int64_t nrows,
+                  const int64_t *cols, int64_t ncols, uint16_t *out, int32_t *Ci_out)
 {
     if (s < 0 || h < 0 || o < 0 || !out || (!X && s * h > 0) ||
         (!Wq && h * o > 0) || (!aw && o > 0))
@@ -357,7 +402,7 @@ int oracle_matmul(const uint16_t *X, int64_t s, int64_t h, const int8_t *Wq,
             goto done;
     }
     /* Step 4: codes and exact integer product */
-    rc = oracle_quantize_rows(X, s, h, flags, rows, nrows, Xq, ax);
+    rc = oracle_quantize_rows_mode(X, s, h, flags, rows, nrows, x_tensor, Xq, ax);
     if (rc)
         goto done;
     rc = oracle_int8_gemm(Xq, nrows, h, Wq, o, cols, ncols, Ci);

@@ -178,6 +178,43 @@ def test_prepare_weight_layout_scale_and_codes():
     assert np.array_equal(Wq[j].ravel().astype(np.int64), exact)
 
 
+def test_tensor_wise_and_row_wise_codes_of_the_golden_rows():
+    g = load_golden("tensorwise_example.txt")
+    X = np.array([[float(v) for v in g["row1"]], [float(v) for v in g["row2"]]],
+                 dtype=np.float16)
+    flags = np.zeros(4, dtype=np.uint8)
+    Xq, ax = oracle.quantize_rows(X, flags, tensor=True)
+    assert ax.tolist() == [float(g["tensor_scale"][0])] * 2
+    assert Xq[0].tolist() == [int(v) for v in g["tensor_codes1"]]
+    assert Xq[1].tolist() == [int(v) for v in g["tensor_codes2"]]
+    Xq, ax = oracle.quantize_rows(X, flags)
+    assert ax.tolist() == [float(v) for v in g["row_scales"]]
+    assert Xq[0].tolist() == [int(v) for v in g["tensor_codes1"]]
+    assert Xq[1].tolist() == [int(v) for v in g["row_codes2"]]
+    # one scale for all rows: any row subset sees the whole tensor's constant
+    Xq, ax = oracle.quantize_rows(X, flags, rows=[1], tensor=True)
+    assert ax.tolist() == [3.0] and Xq[0].tolist() == [int(v) for v in g["tensor_codes2"]]
+
+
+def test_tensor_wise_equals_row_wise_when_every_row_shares_its_absmax():
+    X = workloads.random_x(RNG, 12, 96, outlier_cols=(7,), row_frac=1.0)
+    X[:, 3] = 4.5  # below alpha, above every N(0,1) draw here: every row's max
+    flags, _, _ = oracle.detect_outliers(X, 6.0)
+    a = oracle.quantize_rows(X, flags)
+    b = oracle.quantize_rows(X, flags, tensor=True)
+    assert np.all(a[1] == 4.5)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_tensor_wise_weight_uses_the_global_absmax():
+    W = workloads.random_w(RNG, 150, 40)
+    Wq, aw = oracle.prepare_weight(W, tensor=True)
+    m = np.abs(W.astype(np.float32)).max()
+    assert np.all(aw == m)
+    exact = _exact_codes(W.T.ravel(), np.full(W.size, m, dtype=np.float16))
+    assert np.array_equal(Wq.ravel().astype(np.int64), exact)
+
+
 # ----------------------------------------------------------- detection
 
 def test_detection_threshold_is_inclusive():
