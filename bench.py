@@ -44,6 +44,8 @@ METRIC = "LLM.int8() matmul effective TOPS"
 UNIT = "TOPS"
 DEFAULT_WORKLOAD = "opt6.7b_attn_prefill"
 FLUSH_BYTES = 512 << 20
+# scale granularity flags -> LLMINT8_SCALE_VECTORWISE (0) / TENSORWISE (1)
+SCALE_MODES = {"row": 0, "column": 0, "tensor": 1}
 KERNEL_SOURCES = ["mixed_precision_int8_b200/csrc/gemm_sm100.cuh",
                   "mixed_precision_int8_b200/csrc/decode_sm100.cuh",
                   "mixed_precision_int8_b200/csrc/quant_kernels.cuh",
@@ -151,7 +153,7 @@ class ClockSampler:
 
 # ------------------------------------------------------------ CPU oracle
 
-def cpu_oracle_run(wl, X, Wq, aw, budget_s: float):
+def cpu_oracle_run(wl, X, Wq, aw, budget_s: float, x_tensor: bool = False):
     """Time the oracle on a row sample sized to about budget_s seconds.
 
     The sample is grown by 4x until a run takes a quarter of the budget (the
@@ -164,7 +166,7 @@ def cpu_oracle_run(wl, X, Wq, aw, budget_s: float):
     def timed(n):
         rows = np.sort(order[:n])
         t = time.perf_counter()
-        oracle.matmul(X, Wq, aw, wl.alpha, rows=rows)
+        oracle.matmul(X, Wq, aw, wl.alpha, rows=rows, x_tensor=x_tensor)
         return time.perf_counter() - t
 
     n = min(wl.s, 4)
@@ -239,7 +241,8 @@ def run_ours(args, world, rank, local):
     s, h, o = wl.s, wl.h, wl.o
     Xd = torch.from_numpy(X).to(dev)
     Wd = torch.from_numpy(W).to(dev)
-    pw = binding.llmint8_prepare_weight(Wd)
+    x_mode = SCALE_MODES[args.x_scale]
+    pw = binding.llmint8_prepare_weight(Wd, w_scale=SCALE_MODES[args.w_scale])
     torch.cuda.synchronize()
     del Wd
     out = torch.empty((s, o), dtype=torch.float16, device=dev)
@@ -250,7 +253,7 @@ def run_ours(args, world, rank, local):
 
     def step(ev=None):
         binding.llmint8_matmul(Xd, pw, wl.alpha, out=out, workspace=ws,
-                               events=ev)
+                               events=ev, x_scale=x_mode)
 
     for _ in range(Wm):
         flush.fill_(1)
@@ -300,7 +303,7 @@ def run_ours(args, world, rank, local):
     outh = torch.empty((s, o), dtype=torch.float16).pin_memory()
     wsh = binding.Workspace(s, h, o, device=dev, host=True)
     for _ in range(max(1, Wm)):
-        binding.llmint8_matmul_host(Xh, pw, wl.alpha, outh, wsh)
+        binding.llmint8_matmul_host(Xh, pw, wl.alpha, outh, wsh, x_scale=x_mode)
     e_ms = []
     barrier(world)
     torch.cuda.synchronize()
@@ -309,7 +312,7 @@ def run_ours(args, world, rank, local):
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        binding.llmint8_matmul_host(Xh, pw, wl.alpha, outh, wsh)
+        binding.llmint8_matmul_host(Xh, pw, wl.alpha, outh, wsh, x_scale=x_mode)
         b.record(stream)
         b.synchronize()
         e_ms.append(a.elapsed_time(b))
@@ -351,6 +354,7 @@ def run_ours(args, world, rank, local):
         "config": {"workload": wl.name, "s": s, "h": h, "o": o,
                    "alpha": wl.alpha, "outlier_cols": int(len(cols)),
                    "parallelism": f"replicas x{world}" if world > 1 else "single",
+                   "scales": {"x": args.x_scale, "w": args.w_scale},
                    "l2": "flushed (512 MB write) before every timed step"},
         "e2e": {"value": e2e_value, "unit": UNIT,
                 "h2d_bytes_per_step": 2 * s * h,
@@ -365,7 +369,8 @@ def run_ours(args, world, rank, local):
         import oracle
         Wq = pw.wq.cpu().numpy()
         aw = pw.aw.cpu().numpy()
-        line["cpu_baseline"] = cpu_oracle_run(wl, X, Wq, aw, args.cpu_seconds)
+        line["cpu_baseline"] = cpu_oracle_run(wl, X, Wq, aw, args.cpu_seconds,
+                                              x_tensor=args.x_scale == "tensor")
     return line
 
 
@@ -376,14 +381,15 @@ def run_reference(args, world, rank, local):
         return None
     import oracle
     wl, X, cols, W = workloads.make_inputs(args.workload)
-    Wq, aw = oracle.prepare_weight(W)
+    Wq, aw = oracle.prepare_weight(W, tensor=args.w_scale == "tensor")
+    x_tensor = args.x_scale == "tensor"
     per_step = max(0.2, args.cpu_seconds / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
-        cpu_oracle_run(wl, X, Wq, aw, per_step)
+        cpu_oracle_run(wl, X, Wq, aw, per_step, x_tensor)
     vals, samples = [], []
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        r = cpu_oracle_run(wl, X, Wq, aw, per_step)
+        r = cpu_oracle_run(wl, X, Wq, aw, per_step, x_tensor)
         vals.append(r["value"])
         samples.append(r["sample"])
     el = time.perf_counter() - t0
@@ -396,7 +402,8 @@ def run_reference(args, world, rank, local):
         "vs_baseline": None, "dtype": "i8 codes, fp64 accumulation",
         "data": "synthetic (seeded, OPT-shaped outliers)",
         "config": {"workload": wl.name, "s": wl.s, "h": wl.h, "o": wl.o,
-                   "alpha": wl.alpha, "parallelism": "single"},
+                   "alpha": wl.alpha, "parallelism": "single",
+                   "scales": {"x": args.x_scale, "w": args.w_scale}},
         "cpu_baseline": {"value": value, "unit": UNIT,
                          "cores": oracle.num_threads(), "kind": "oracle",
                          "sample": f"per step: {samples[-1]}; "
@@ -416,6 +423,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--x-scale", default="row", choices=["row", "tensor"],
+                    help="absmax per row of X (the method) or one per tensor")
+    ap.add_argument("--w-scale", default="column", choices=["column", "tensor"],
+                    help="absmax per column of W (the method) or one per tensor")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

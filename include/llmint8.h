@@ -110,14 +110,26 @@ typedef struct {
  *      of Step 4 (testing; costs an extra 4*s*o bytes of stores).
  *  path: 0 = automatic, 1 = force the prefill GEMM kernel, 2 = force the
  *      decode (s <= 16) kernel; 2 with s > 16 is LLMINT8_ERR_ARG.
- *  launches (out): number of kernels this call enqueued. */
+ *  launches (out): number of kernels this call enqueued.
+ *  x_scale: LLMINT8_SCALE_VECTORWISE (0, the method: one absmax per row of
+ *      X) or LLMINT8_SCALE_TENSORWISE (one absmax for all of X, the largest
+ *      row scale, so every ax[i] is that constant); anything else is
+ *      LLMINT8_ERR_ARG. Outlier columns are split off in both modes. */
 typedef struct {
     void *gemm_event_start;
     void *gemm_event_stop;
     int32_t *ci_dev;
     int32_t path;
     int32_t launches;
+    int32_t x_scale;
 } llmint8_matmul_opts;
+
+/* Scale granularity ("Quantization Primitives": absmax over a whole tensor;
+ * "Vector-wise Quantization": one constant per row of X and per column of
+ * W). The tensor-wise modes are the Table 1 baselines ("Int8 absmax"), kept
+ * for comparison; vector-wise is the method. */
+#define LLMINT8_SCALE_VECTORWISE 0
+#define LLMINT8_SCALE_TENSORWISE 1
 
 /* Human-readable name of a status code (static storage). */
 LLMINT8_API const char *llmint8_status_string(llmint8_status st);
@@ -155,6 +167,14 @@ LLMINT8_API llmint8_status llmint8_prepare_weight(const uint16_t *W_dev, int64_t
                                       int64_t o, llmint8_weight *out,
                                       void *stream);
 
+/* llmint8_prepare_weight with a scale granularity: w_scale =
+ * LLMINT8_SCALE_VECTORWISE is llmint8_prepare_weight; TENSORWISE sets every
+ * aw[j] to max_{k,j} |W[k][j]| and quantises all of W against it. Any other
+ * w_scale is LLMINT8_ERR_ARG. */
+LLMINT8_API llmint8_status llmint8_prepare_weight_ex(const uint16_t *W_dev, int64_t h,
+                                         int64_t o, int32_t w_scale,
+                                         llmint8_weight *out, void *stream);
+
 /* Steps 1 and 4 (activation side) on their own, for testing:
  *   flags_dev[j]  = 1 if column j is an outlier column, else 0   (u8 [h])
  *   idx_dev[0..n) = outlier columns in ascending order           (i32 [h])
@@ -171,6 +191,17 @@ LLMINT8_API llmint8_status llmint8_quantize_rows(const uint16_t *X_dev, int64_t 
                                      int32_t *idx_dev, int32_t *n_outliers_dev,
                                      void *scratch_dev, size_t scratch_bytes,
                                      void *stream);
+
+/* llmint8_quantize_rows with a scale granularity: x_scale =
+ * LLMINT8_SCALE_TENSORWISE makes every ax[i] the largest of the row scales
+ * above and quantises all rows against it (outlier columns still 0);
+ * VECTORWISE is llmint8_quantize_rows; anything else is LLMINT8_ERR_ARG. */
+LLMINT8_API llmint8_status llmint8_quantize_rows_ex(const uint16_t *X_dev, int64_t s,
+                                        int64_t h, float alpha, int32_t x_scale,
+                                        int8_t *Xq_dev, float *ax_dev,
+                                        uint8_t *flags_dev, int32_t *idx_dev,
+                                        int32_t *n_outliers_dev, void *scratch_dev,
+                                        size_t scratch_bytes, void *stream);
 
 /* The whole layer, Steps 1-5: out_dev (fp16 [s][o]) = LLM.int8()(X_dev, w).
  *   out[i][j] = fp16( Ci[i][j] * ax[i] * aw[j] / (127*127)
@@ -203,6 +234,14 @@ LLMINT8_API llmint8_status llmint8_matmul_host(const uint16_t *X_host, int64_t s
                                    const llmint8_weight *w, float alpha,
                                    uint16_t *out_host, void *ws_dev,
                                    size_t ws_bytes, void *stream);
+
+/* llmint8_matmul_host with the extras of llmint8_matmul_opts (opts may be
+ * NULL; the same fields and errors as llmint8_matmul_ex). */
+LLMINT8_API llmint8_status llmint8_matmul_host_ex(const uint16_t *X_host, int64_t s,
+                                      const llmint8_weight *w, float alpha,
+                                      uint16_t *out_host, void *ws_dev,
+                                      size_t ws_bytes, llmint8_matmul_opts *opts,
+                                      void *stream);
 
 /* The fp16 outlier tiles of the last llmint8_matmul on this workspace:
  * copies n_outliers (to *n_out_host), XO (fp16 [s][n], to XO_host if

@@ -23,6 +23,8 @@ STATUS_NAMES = {0: "OK", -1: "ERR_NULL", -2: "ERR_SHAPE", -3: "ERR_ALIGN",
                 -4: "ERR_WORKSPACE", -5: "ERR_CUDA", -6: "ERR_DEVICE_STATUS",
                 -7: "ERR_ARG", -8: "ERR_UNSUPPORTED", -9: "ERR_TOO_LARGE"}
 NOALLOC_MAX_SCRATCH_BYTES = 64 << 20  # LLMINT8_NOALLOC_MAX_SCRATCH_BYTES
+SCALE_VECTORWISE = 0  # LLMINT8_SCALE_VECTORWISE: per row of X / column of W
+SCALE_TENSORWISE = 1  # LLMINT8_SCALE_TENSORWISE: one constant per tensor
 
 _c_i64, _c_i32, _c_f32 = ctypes.c_int64, ctypes.c_int32, ctypes.c_float
 _vp, _sz = ctypes.c_void_p, ctypes.c_size_t
@@ -35,7 +37,8 @@ class llmint8_weight(ctypes.Structure):
 
 class llmint8_matmul_opts(ctypes.Structure):
     _fields_ = [("gemm_event_start", _vp), ("gemm_event_stop", _vp),
-                ("ci_dev", _vp), ("path", _c_i32), ("launches", _c_i32)]
+                ("ci_dev", _vp), ("path", _c_i32), ("launches", _c_i32),
+                ("x_scale", _c_i32)]
 
 
 class Llmint8Error(RuntimeError):
@@ -65,7 +68,11 @@ def load_library():
         "llmint8_workspace_init": ([_vp, _sz, _vp], _c_i32),
         "llmint8_prepare_weight": ([_vp, _c_i64, _c_i64,
                                     ctypes.POINTER(llmint8_weight), _vp], _c_i32),
+        "llmint8_prepare_weight_ex": ([_vp, _c_i64, _c_i64, _c_i32,
+                                       ctypes.POINTER(llmint8_weight), _vp], _c_i32),
         "llmint8_quantize_rows_scratch_size": ([_c_i64], _sz),
+        "llmint8_quantize_rows_ex": ([_vp, _c_i64, _c_i64, _c_f32, _c_i32, _vp,
+                                      _vp, _vp, _vp, _vp, _vp, _sz, _vp], _c_i32),
         "llmint8_quantize_rows": ([_vp, _c_i64, _c_i64, _c_f32, _vp, _vp, _vp,
                                    _vp, _vp, _vp, _sz, _vp], _c_i32),
         "llmint8_matmul": ([_vp, _c_i64, ctypes.POINTER(llmint8_weight), _c_f32,
@@ -75,6 +82,9 @@ def load_library():
                                ctypes.POINTER(llmint8_matmul_opts), _vp], _c_i32),
         "llmint8_matmul_host": ([_vp, _c_i64, ctypes.POINTER(llmint8_weight),
                                  _c_f32, _vp, _vp, _sz, _vp], _c_i32),
+        "llmint8_matmul_host_ex": ([_vp, _c_i64, ctypes.POINTER(llmint8_weight),
+                                    _c_f32, _vp, _vp, _sz,
+                                    ctypes.POINTER(llmint8_matmul_opts), _vp], _c_i32),
         "llmint8_read_outlier_tiles": ([_vp, _sz, _c_i64, _c_i64, _c_i64, _vp,
                                         _vp, _vp, _vp], _c_i32),
         "llmint8_read_device_status": ([_vp, _sz, _vp, _vp], _c_i32),
@@ -97,7 +107,9 @@ EXPORTED = ("llmint8_status_string", "llmint8_workspace_size",
             "llmint8_quantize_rows", "llmint8_matmul", "llmint8_matmul_ex",
             "llmint8_matmul_host", "llmint8_read_outlier_tiles",
             "llmint8_read_device_status", "llmint8_decode_max_rows",
-            "llmint8_matmul_noalloc", "llmint8_wait_selftest")
+            "llmint8_matmul_noalloc", "llmint8_wait_selftest",
+            "llmint8_prepare_weight_ex", "llmint8_quantize_rows_ex",
+            "llmint8_matmul_host_ex")
 
 
 def status_string(code: int) -> str:
@@ -164,23 +176,28 @@ def llmint8_decode_max_rows() -> int:
 
 
 def llmint8_prepare_weight(W: torch.Tensor, stream=None,
-                           keep_fp16: bool = False) -> PreparedWeight:
+                           keep_fp16: bool = False,
+                           w_scale: int = SCALE_VECTORWISE) -> PreparedWeight:
     """W fp16 [h,o] on the GPU -> PreparedWeight (int8 [o,h] codes + scales).
 
     With keep_fp16 the weight keeps W (a reference, not a copy) and the
-    layer's fp16 outlier rows of W are W's own values."""
+    layer's fp16 outlier rows of W are W's own values. w_scale =
+    SCALE_TENSORWISE gives every column the one absmax of all of W."""
     _f16_dev(W, "W")
     h, o = W.shape
     wq = torch.empty((o, h), dtype=torch.int8, device=W.device)
     aw = torch.empty((o,), dtype=torch.float32, device=W.device)
     pw = PreparedWeight(wq, aw, W if keep_fp16 else None)
-    _check("llmint8_prepare_weight", load_library().llmint8_prepare_weight(
-        _ptr(W), h, o, ctypes.byref(pw.c), _stream(stream)))
+    _check("llmint8_prepare_weight_ex", load_library().llmint8_prepare_weight_ex(
+        _ptr(W), h, o, int(w_scale), ctypes.byref(pw.c), _stream(stream)))
     return pw
 
 
-def llmint8_quantize_rows(X: torch.Tensor, alpha: float = 6.0, stream=None):
+def llmint8_quantize_rows(X: torch.Tensor, alpha: float = 6.0, stream=None,
+                          x_scale: int = SCALE_VECTORWISE):
     """Steps 1 and 4 (activation side) -> (Xq, ax, flags, idx, n_outliers).
+
+    x_scale = SCALE_TENSORWISE quantises all rows against one constant.
 
     n_outliers is a 1-element device tensor (it is never read back here);
     idx holds valid entries in its first n_outliers slots.
@@ -196,9 +213,9 @@ def llmint8_quantize_rows(X: torch.Tensor, alpha: float = 6.0, stream=None):
     n = torch.empty((1,), dtype=torch.int32, device=dev)
     nb = int(lib.llmint8_quantize_rows_scratch_size(h))
     scratch = torch.empty(max(nb, 256), dtype=torch.uint8, device=dev)
-    _check("llmint8_quantize_rows", lib.llmint8_quantize_rows(
-        _ptr(X), s, h, float(alpha), _ptr(Xq), _ptr(ax), _ptr(flags), _ptr(idx),
-        _ptr(n), _ptr(scratch), nb, _stream(stream)))
+    _check("llmint8_quantize_rows_ex", lib.llmint8_quantize_rows_ex(
+        _ptr(X), s, h, float(alpha), int(x_scale), _ptr(Xq), _ptr(ax),
+        _ptr(flags), _ptr(idx), _ptr(n), _ptr(scratch), nb, _stream(stream)))
     return Xq, ax, flags, idx, n
 
 
@@ -206,12 +223,14 @@ def llmint8_matmul(X: torch.Tensor, w: PreparedWeight, alpha: float = 6.0,
                    out: Optional[torch.Tensor] = None,
                    workspace: Optional[Workspace] = None,
                    ci: Optional[torch.Tensor] = None, path: int = 0,
-                   events=None, stream=None) -> torch.Tensor:
+                   events=None, stream=None,
+                   x_scale: int = SCALE_VECTORWISE) -> torch.Tensor:
     """C = LLM.int8()(X, W): X fp16 [s,h] on the GPU -> fp16 [s,o].
 
     ci (optional, int32 [s,o]) receives the exact int32 accumulators; path
     forces the prefill (1) or decode (2) kernel; events = (start, stop)
-    torch.cuda.Event pair recorded around the GEMM kernel.
+    torch.cuda.Event pair recorded around the GEMM kernel; x_scale =
+    SCALE_TENSORWISE quantises X with one constant for the whole tensor.
     """
     _f16_dev(X, "X")
     s, h = X.shape
@@ -223,6 +242,7 @@ def llmint8_matmul(X: torch.Tensor, w: PreparedWeight, alpha: float = 6.0,
         workspace = Workspace(s, h, w.o, device=X.device)
     opts = llmint8_matmul_opts()
     opts.path = int(path)
+    opts.x_scale = int(x_scale)
     if ci is not None:
         if ci.dtype != torch.int32 or ci.shape != (s, w.o):
             raise ValueError("ci must be int32 [s,o]")
@@ -263,14 +283,17 @@ def llmint8_matmul_noalloc(X: torch.Tensor, w: PreparedWeight,
 
 def llmint8_matmul_host(X_host: torch.Tensor, w: PreparedWeight,
                         alpha: float, out_host: torch.Tensor,
-                        workspace: Workspace, stream=None) -> torch.Tensor:
+                        workspace: Workspace, stream=None,
+                        x_scale: int = SCALE_VECTORWISE) -> torch.Tensor:
     """End-to-end form: host fp16 X in, host fp16 C out (synchronises)."""
     if X_host.is_cuda or out_host.is_cuda:
         raise ValueError("X_host and out_host must be host tensors")
     s, h = X_host.shape
-    _check("llmint8_matmul_host", load_library().llmint8_matmul_host(
+    opts = llmint8_matmul_opts()
+    opts.x_scale = int(x_scale)
+    _check("llmint8_matmul_host_ex", load_library().llmint8_matmul_host_ex(
         _ptr(X_host), s, ctypes.byref(w.c), float(alpha), _ptr(out_host),
-        _ptr(workspace.buf), workspace.nbytes, _stream(stream)))
+        _ptr(workspace.buf), workspace.nbytes, ctypes.byref(opts), _stream(stream)))
     return out_host
 
 

@@ -165,6 +165,7 @@ int32_t *count_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 1; }
 int32_t *block_counter_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 2; }
 int32_t *act_counter_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 3; }
 int32_t *wo_counter_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 4; }
+float *tensor_scale_word(void *ws) { return reinterpret_cast<float *>(ws) + 5; }
 constexpr int kSelftestWord = 8;  // a status-block word no kernel sets
 
 // --------------------------------------------------------- validation
@@ -346,6 +347,23 @@ llmint8_status enqueue_activation_fused(const DeviceInfo &dev, const ActivationA
   return last_launch();
 }
 
+// Tensor-wise activation scale, after the activation pass has left the
+// bitmask and the row scales: one constant (the largest row scale) for all
+// rows, and every row's codes again against it.
+llmint8_status enqueue_tensor_scale(const ActivationArgs &a, float *scale, cudaStream_t st,
+                                    int32_t *launches) {
+  cudaError_t e = launch(k_tensor_scale, dim3(1), dim3(1024), 0, st, true,
+                         (const float *)a.ax, a.s, scale);
+  if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+  const int64_t rb = (a.s + kRowsPerBlock - 1) / kRowsPerBlock;
+  e = launch(k_rows_tensor_scale, dim3((unsigned)rb), dim3(kRowThreads), 0, st, true, a.X, a.s,
+             (int32_t)a.h, (const uint32_t *)a.mask, (const int32_t *)a.wprefix,
+             (const float *)scale, a.Xq, a.ax);
+  if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+  *launches += 2;
+  return LLMINT8_OK;
+}
+
 llmint8_status enqueue_activation_pass(const DeviceInfo &dev, const ActivationArgs &a,
                                        cudaStream_t st, int32_t *launches) {
   ActPlan plan;
@@ -412,6 +430,9 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
   if ((rc = check_alpha(alpha))) return rc;
   const int path = opts ? opts->path : 0;
   if (path < 0 || path > 2 || (path == 2 && s > kDecodeMaxRows)) return LLMINT8_ERR_ARG;
+  const int x_scale = opts ? opts->x_scale : LLMINT8_SCALE_VECTORWISE;
+  if (x_scale != LLMINT8_SCALE_VECTORWISE && x_scale != LLMINT8_SCALE_TENSORWISE)
+    return LLMINT8_ERR_ARG;
   if (s == 0) return LLMINT8_OK;
   if (!X || !out || !ws) return LLMINT8_ERR_NULL;
   if (!aligned(X, 16) || !aligned(out, 16) || !aligned(ws, 256)) return LLMINT8_ERR_ALIGN;
@@ -505,6 +526,9 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
   } else if ((rc = enqueue_activation_pass(*dev, act, st, &launches))) {
     return rc;
   }
+  if (x_scale == LLMINT8_SCALE_TENSORWISE &&
+      (rc = enqueue_tensor_scale(act, tensor_scale_word(ws), st, &launches)))
+    return rc;
   const bool timed = opts && (opts->gemm_event_start || opts->gemm_event_stop);
   if (opts && opts->gemm_event_start)
     cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->gemm_event_start), st);
@@ -617,6 +641,13 @@ int64_t llmint8_decode_max_rows(void) { return kDecodeMaxRows; }
 
 llmint8_status llmint8_prepare_weight(const uint16_t *W_dev, int64_t h, int64_t o,
                                       llmint8_weight *out, void *stream) {
+  return llmint8_prepare_weight_ex(W_dev, h, o, LLMINT8_SCALE_VECTORWISE, out, stream);
+}
+
+llmint8_status llmint8_prepare_weight_ex(const uint16_t *W_dev, int64_t h, int64_t o,
+                                         int32_t w_scale, llmint8_weight *out, void *stream) {
+  if (w_scale != LLMINT8_SCALE_VECTORWISE && w_scale != LLMINT8_SCALE_TENSORWISE)
+    return LLMINT8_ERR_ARG;
   if (!W_dev || !out || !out->wq_dev || !out->aw_dev) return LLMINT8_ERR_NULL;
   llmint8_status rc = check_hw(h, o);
   if (rc) return rc;
@@ -635,6 +666,7 @@ llmint8_status llmint8_prepare_weight(const uint16_t *W_dev, int64_t h, int64_t 
   if (rpb < 8) rpb = 8;
   const int gy = (int)((h + rpb - 1) / rpb);
   k_weight_colmax<<<dim3(gx, gy), 256, 0, st>>>(W_dev, hh, oo, (int32_t)rpb, awb);
+  if (w_scale == LLMINT8_SCALE_TENSORWISE) k_bits_to_tensor_max<<<1, 1024, 0, st>>>(awb, o);
   k_weight_codes<<<dim3((unsigned)((o + kWqTile - 1) / kWqTile),
                         (unsigned)((h + kWqTile - 1) / kWqTile)),
                    256, 0, st>>>(W_dev, hh, oo, awb, out->wq_dev);
@@ -652,6 +684,18 @@ llmint8_status llmint8_quantize_rows(const uint16_t *X_dev, int64_t s, int64_t h
                                      int8_t *Xq_dev, float *ax_dev, uint8_t *flags_dev,
                                      int32_t *idx_dev, int32_t *n_outliers_dev,
                                      void *scratch_dev, size_t scratch_bytes, void *stream) {
+  return llmint8_quantize_rows_ex(X_dev, s, h, alpha, LLMINT8_SCALE_VECTORWISE, Xq_dev, ax_dev,
+                                  flags_dev, idx_dev, n_outliers_dev, scratch_dev, scratch_bytes,
+                                  stream);
+}
+
+llmint8_status llmint8_quantize_rows_ex(const uint16_t *X_dev, int64_t s, int64_t h, float alpha,
+                                        int32_t x_scale, int8_t *Xq_dev, float *ax_dev,
+                                        uint8_t *flags_dev, int32_t *idx_dev,
+                                        int32_t *n_outliers_dev, void *scratch_dev,
+                                        size_t scratch_bytes, void *stream) {
+  if (x_scale != LLMINT8_SCALE_VECTORWISE && x_scale != LLMINT8_SCALE_TENSORWISE)
+    return LLMINT8_ERR_ARG;
   if (h < 16 || h > kMaxH || (h % 16) != 0) return LLMINT8_ERR_SHAPE;
   if (s < 0 || s > (int64_t)INT32_MAX) return LLMINT8_ERR_SHAPE;
   llmint8_status rc = check_alpha(alpha);
@@ -685,7 +729,14 @@ llmint8_status llmint8_quantize_rows(const uint16_t *X_dev, int64_t s, int64_t h
   act.Xq = Xq_dev;
   act.ax = ax_dev;
   int32_t launches = 0;
-  return enqueue_activation_pass(*dev, act, as_stream(stream), &launches);
+  cudaStream_t st = as_stream(stream);
+  if ((rc = enqueue_activation_pass(*dev, act, st, &launches))) return rc;
+  if (x_scale == LLMINT8_SCALE_TENSORWISE && s > 0) {
+    if ((rc = enqueue_tensor_scale(act, reinterpret_cast<float *>(sb) + 4, st, &launches)))
+      return rc;
+    return last_launch();
+  }
+  return LLMINT8_OK;
 }
 
 llmint8_status llmint8_matmul(const uint16_t *X_dev, int64_t s, const llmint8_weight *w,
@@ -705,6 +756,13 @@ llmint8_status llmint8_matmul_ex(const uint16_t *X_dev, int64_t s, const llmint8
 llmint8_status llmint8_matmul_host(const uint16_t *X_host, int64_t s, const llmint8_weight *w,
                                    float alpha, uint16_t *out_host, void *ws_dev, size_t ws_bytes,
                                    void *stream) {
+  return llmint8_matmul_host_ex(X_host, s, w, alpha, out_host, ws_dev, ws_bytes, nullptr, stream);
+}
+
+llmint8_status llmint8_matmul_host_ex(const uint16_t *X_host, int64_t s, const llmint8_weight *w,
+                                      float alpha, uint16_t *out_host, void *ws_dev,
+                                      size_t ws_bytes, llmint8_matmul_opts *opts, void *stream) {
+  if (opts) opts->launches = 0;
   llmint8_status rc = validate_weight(w);
   if (rc) return rc;
   if (s < 0 || s > (int64_t)INT32_MAX) return LLMINT8_ERR_SHAPE;
@@ -720,7 +778,7 @@ llmint8_status llmint8_matmul_host(const uint16_t *X_host, int64_t s, const llmi
   uint16_t *od = reinterpret_cast<uint16_t *>(wsb + L.ostage);
   if (cudaMemcpyAsync(xd, X_host, 2 * (size_t)s * w->h, cudaMemcpyHostToDevice, st) != cudaSuccess)
     return LLMINT8_ERR_CUDA;
-  if ((rc = matmul_impl(xd, s, w, alpha, od, ws_dev, ws_bytes, nullptr, st, true))) return rc;
+  if ((rc = matmul_impl(xd, s, w, alpha, od, ws_dev, ws_bytes, opts, st, true))) return rc;
   if (cudaMemcpyAsync(out_host, od, 2 * (size_t)s * w->o, cudaMemcpyDeviceToHost, st) !=
       cudaSuccess)
     return LLMINT8_ERR_CUDA;

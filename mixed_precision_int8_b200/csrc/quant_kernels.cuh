@@ -874,6 +874,69 @@ __global__ void __launch_bounds__(kDecodeThreads)
   *reinterpret_cast<uint2 *>(Xq + (int64_t)row * h + c) = q;
 }
 
+// ------------------------------------------ tensor-wise scale baselines
+// The Table 1 baselines of "Quantization Primitives": absmax over a whole
+// tensor instead of per row (X) or per column (W). Both run on the same
+// kernels as the vector-wise method; only the scales change.
+
+// One block: every one of the n magnitude words becomes their maximum
+// (prepare_weight's column maxima -> one constant for the whole weight).
+__global__ void __launch_bounds__(1024) k_bits_to_tensor_max(uint32_t *__restrict__ bits,
+                                                             int64_t n) {
+  __shared__ uint32_t red[32];
+  uint32_t m = 0;
+  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) m = max(m, bits[i]);
+#pragma unroll
+  for (int d = 16; d > 0; d >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, d));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  m = 0;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = max(m, red[w]);
+  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) bits[i] = m;
+}
+
+// One block: *scale = max over the s row scales (each the absmax of a
+// row's regular columns): the activation tensor's one constant.
+__global__ void __launch_bounds__(1024) k_tensor_scale(const float *__restrict__ ax, int64_t s,
+                                                       float *__restrict__ scale) {
+  __shared__ float red[32];
+  grid_dependency_wait();
+  grid_dependency_trigger();
+  float m = 0.0f;
+  for (int64_t i = threadIdx.x; i < s; i += blockDim.x) m = fmaxf(m, ax[i]);
+#pragma unroll
+  for (int d = 16; d > 0; d >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, d));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, red[w]);
+    *scale = m;
+  }
+}
+
+// One warp per row: codes of the regular columns against the tensor's one
+// constant (outlier columns stay 0); ax[row] becomes that constant.
+__global__ void __launch_bounds__(kRowThreads)
+    k_rows_tensor_scale(const uint16_t *__restrict__ X, int64_t s, int32_t h,
+                        const uint32_t *__restrict__ mask, const int32_t *__restrict__ word_prefix,
+                        const float *__restrict__ scale, int8_t *__restrict__ Xq,
+                        float *__restrict__ ax) {
+  grid_dependency_wait();
+  grid_dependency_trigger();
+  const int lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerBlock + (threadIdx.x >> 5);
+  if (row >= s) return;
+  const float a = *scale;
+  const float r = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
+  if (lane == 0) ax[row] = a;
+  const uint16_t *xr = X + row * h;
+  int8_t *qr = Xq + row * h;
+  for (int32_t c = lane * 8; c < h; c += 256) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(xr + c));
+    quantize_chunk(v, __ldcg(mask + (c >> 5)), c, a, r, row, 0, word_prefix, qr, nullptr);
+  }
+}
+
 // ------------------------------------------------------- wait self-test
 // Two waits that nothing can satisfy, each bounded like every wait of the
 // library: an mbarrier phase nobody arrives at, and a word nobody sets.

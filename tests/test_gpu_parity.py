@@ -161,6 +161,88 @@ def test_workload_matmul_with_fp16_outlier_rows(name):
     torch.cuda.empty_cache()
 
 
+# Tensor-wise baselines ("Quantization Primitives"; Table 1 "Int8 absmax"):
+# one absmax for all of X and/or all of W, on the same kernels.
+TENSOR_CASES = [SMALL[i] for i in (0, 2, 4, 5, 6, 9, 11, 12)]
+VW, TW = binding.SCALE_VECTORWISE, binding.SCALE_TENSORWISE
+
+
+@pytest.mark.parametrize("case", TENSOR_CASES, ids=lambda c: f"{c[0]}x{c[1]}x{c[2]}a{c[4]}")
+def test_quantize_rows_tensorwise_bit_exact(case):
+    X, _, alpha = _small_inputs(case, seed=11)
+    if X.shape[0] > 2:
+        X[1] = 0  # an all-zero row takes the tensor constant too
+    Xq, ax, flags, idx, n = binding.llmint8_quantize_rows(to_dev(X), alpha, x_scale=TW)
+    torch.cuda.synchronize()
+    f_ref, _, n_ref = oracle.detect_outliers(X, alpha)
+    assert int(n.item()) == n_ref
+    assert np.array_equal(flags.cpu().numpy(), f_ref)
+    Xq_ref, ax_ref = oracle.quantize_rows(X, f_ref, tensor=True)
+    assert np.array_equal(ax.cpu().numpy(), ax_ref)
+    assert np.array_equal(Xq.cpu().numpy(), Xq_ref)
+
+
+@pytest.mark.parametrize("case", TENSOR_CASES, ids=lambda c: f"{c[0]}x{c[1]}x{c[2]}")
+def test_prepare_weight_tensorwise_bit_exact(case):
+    _, W, _ = _small_inputs(case, seed=12)
+    W[:, 1] = 0
+    pw = binding.llmint8_prepare_weight(to_dev(W), w_scale=TW)
+    torch.cuda.synchronize()
+    Wq_ref, aw_ref = oracle.prepare_weight(W, tensor=True)
+    assert np.array_equal(pw.aw.cpu().numpy(), aw_ref)
+    assert np.array_equal(pw.wq.cpu().numpy(), Wq_ref)
+
+
+@pytest.mark.parametrize("modes", [(TW, VW), (VW, TW), (TW, TW)], ids=["xT", "wT", "xTwT"])
+@pytest.mark.parametrize("case", TENSOR_CASES, ids=lambda c: f"{c[0]}x{c[1]}x{c[2]}a{c[4]}")
+def test_matmul_tensorwise_small(case, modes):
+    x_mode, w_mode = modes
+    X, W, alpha = _small_inputs(case, seed=13)
+    s = X.shape[0]
+    pw = binding.llmint8_prepare_weight(to_dev(W), w_scale=w_mode)
+    Wq_ref, aw_ref = oracle.prepare_weight(W, tensor=(w_mode == TW))
+    ref, ci_ref = oracle.matmul(X, Wq_ref, aw_ref, alpha, want_ci=True,
+                                x_tensor=(x_mode == TW))
+    for path in ([1, 2] if s <= 16 else [1]):
+        ws = binding.Workspace(s, pw.h, pw.o)
+        ci = torch.full((s, pw.o), -7, dtype=torch.int32, device="cuda")
+        out = binding.llmint8_matmul(to_dev(X), pw, alpha, workspace=ws, ci=ci,
+                                     path=path, x_scale=x_mode)
+        torch.cuda.synchronize()
+        assert binding.llmint8_read_device_status(ws) == 0
+        assert np.array_equal(ci.cpu().numpy(), ci_ref), f"int32 accumulators, path {path}"
+        assert_close_fp16(out.cpu().numpy(), ref, f"out path {path}")
+
+
+@pytest.mark.parametrize("name", ["opt6.7b_attn_prefill", "opt175b_decode"])
+def test_workload_matmul_tensorwise(name):
+    """Both tensors tensor-wise at full size, on sampled rows and columns.
+    The oracle's weight constant is taken over the sampled columns plus the
+    column that holds W's largest magnitude, so it is W's own constant."""
+    wl, X, cols, W = workloads.make_inputs(name)
+    Wd = to_dev(W)
+    pw = binding.llmint8_prepare_weight(Wd, w_scale=TW)
+    del Wd
+    rows = sample_rows(wl.s, 48)
+    c = sample_cols(wl.o, 512)
+    jmax = int(np.abs(W.astype(np.float32)).max(axis=0).argmax())
+    cw = np.append(c, jmax)
+    Wq_ref, aw_ref = oracle.prepare_weight(np.ascontiguousarray(W[:, cw]), tensor=True)
+    ref, ci_ref = oracle.matmul(X, Wq_ref[:-1], aw_ref[:-1], wl.alpha, rows=rows,
+                                want_ci=True, x_tensor=True)
+    ws = binding.Workspace(wl.s, pw.h, pw.o)
+    ci = torch.empty((wl.s, pw.o), dtype=torch.int32, device="cuda")
+    out = binding.llmint8_matmul(to_dev(X), pw, wl.alpha, workspace=ws, ci=ci, x_scale=TW)
+    torch.cuda.synchronize()
+    assert binding.llmint8_read_device_status(ws) == 0
+    assert np.array_equal(pw.aw[c].cpu().numpy(), aw_ref[:-1])
+    assert np.array_equal(pw.wq[c].cpu().numpy(), Wq_ref[:-1])
+    assert np.array_equal(ci.cpu().numpy()[np.ix_(rows, c)], ci_ref)
+    assert_close_fp16(out.cpu().numpy()[np.ix_(rows, c)], ref)
+    del pw, ci, out, ws
+    torch.cuda.empty_cache()
+
+
 # rows too long for a shared-memory stage of the one-read pass (2h bytes plus
 # its bitmask above the per-CTA budget): the column-pass + row-pass kernels
 LONG_H = 108544
