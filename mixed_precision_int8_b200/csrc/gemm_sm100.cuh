@@ -16,13 +16,15 @@
 //               into a TMEM accumulator; tcgen05.commit frees ring slots
 //   warp 2      allocates / frees the 512 TMEM columns (2 accumulators)
 //   warps 4-11  epilogue: before the first tile, a share of the fp16 outlier
-//               rows of W; per tile, the column scales and outlier rows (as
-//               fp32) staged in shared memory while the MMA runs, then each
-//               warp tcgen05.lds its half of the columns of its 32 TMEM lanes
-//               (= 32 output rows), dequantises and adds the outlier product
-//               with packed f32x2 FMAs on CUDA cores, and writes fp16 through
-//               a 64B-swizzled 32x32 staging block with TMA stores; the other
-//               accumulator is being filled by the MMA meanwhile.
+//               rows of W; per tile, while the MMA runs, the column scales
+//               and outlier rows (as fp32) go to shared memory and each
+//               thread computes the outlier product of its row and its half
+//               of the tile's columns into registers (packed f32x2 FMAs).
+//               Once the accumulator is ready, each warp tcgen05.lds its half
+//               of the columns of its 32 TMEM lanes (= 32 output rows),
+//               dequantises, adds the outlier product and writes fp16
+//               through a 64B-swizzled 32x32 staging block with TMA stores;
+//               the other accumulator is being filled by the MMA meanwhile.
 // Every wait is bounded by the global timer; on a timeout the CTA records a
 // status bit, drains its in-flight copies and MMAs, frees TMEM and returns.
 #pragma once
@@ -52,7 +54,7 @@ constexpr int EPI_BARRIER = 1;       // named barrier of the epilogue warps
 constexpr int OUT_BOX_COLS = 32;     // fp16 columns per TMA store (64 bytes)
 constexpr uint32_t OUT_STAGE_BYTES = 32 * OUT_BOX_COLS * 2;  // per epilogue warp
 constexpr int REGS_LOW = 56;         // producer / MMA warpgroup after setmaxnreg
-constexpr int REGS_HIGH = 216;       // epilogue warpgroups after setmaxnreg
+constexpr int REGS_HIGH = 208;       // epilogue warpgroups after setmaxnreg
 constexpr int FAST_OUTLIERS = 16;    // outlier rows kept in shared memory
 constexpr uint32_t RING_BYTES = STAGES * (A_STAGE_BYTES + B_STAGE_BYTES);
 constexpr uint32_t OUT_OFF = RING_BYTES;
@@ -62,6 +64,12 @@ constexpr uint32_t BAR_OFF = AW_OFF + BN * 4;
 constexpr size_t SMEM_BYTES = 1024 + BAR_OFF + 256;
 
 static_assert(NUM_ACC * BN <= 512, "TMEM holds 512 columns");
+// registers a thread gets at launch (65536 / 384 rounded down to a multiple
+// of 8); setmaxnreg.inc can only hand out what .dec gave back
+constexpr int REGS_LAUNCH = 168;
+static_assert((NUM_THREADS - NUM_EPI_THREADS) * REGS_LOW + NUM_EPI_THREADS * REGS_HIGH <=
+                  NUM_THREADS * REGS_LAUNCH,
+              "register split exceeds the launch allocation");
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 static_assert(OUT_OFF % 1024 == 0, "swizzled staging must be 1024-byte aligned");
 static_assert(BAR_OFF % 8 == 0, "mbarrier alignment");
@@ -340,88 +348,96 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         xo[t] = (t < n_fast && row_ok)
                     ? __half2float(__ushort_as_half(p.XO[(int64_t)row * n_out + t]))
                     : 0.0f;
-      // (3) accumulator; a timeout in any epilogue thread stops all of them
+      // (3) the fp16 outlier product e = sum_t xo[t] * WO[t][j] of this
+      //     thread's BN/2 columns, while the MMA still fills the accumulator
+      //     (it does not depend on Ci); packed pairs of columns
+      uint64_t e2[BN / 64][16];
+#pragma unroll
+      for (int c = 0; c < BN / 64; ++c)
+#pragma unroll
+        for (int q = 0; q < 16; ++q) e2[c][q] = 0ull;
+#pragma unroll
+      for (int t = 0; t < FAST_OUTLIERS; ++t) {
+        if (t < n_fast) {
+          const uint64_t x2 = f32x2_pack(xo[t], xo[t]);
+          const float4 *wrow = reinterpret_cast<const float4 *>(sWO + t * BN + hc * (BN / 2));
+#pragma unroll
+          for (int q4 = 0; q4 < BN / 8; ++q4) {
+            const float4 w = wrow[q4];
+            uint64_t *e = e2[q4 / 8];
+            e[2 * (q4 % 8)] = f32x2_fma(x2, f32x2_pack(w.x, w.y), e[2 * (q4 % 8)]);
+            e[2 * (q4 % 8) + 1] = f32x2_fma(x2, f32x2_pack(w.z, w.w), e[2 * (q4 % 8) + 1]);
+          }
+        }
+      }
+      for (int32_t t = FAST_OUTLIERS; t < n_out; ++t) {
+        // outlier columns beyond the shared-memory fast path (|O| > 16):
+        // their fp16 rows of W straight from global memory (o % 16 == 0,
+        // so a group of 8 columns is either wholly inside or outside)
+        const float x =
+            row_ok ? __half2float(__ushort_as_half(p.XO[(int64_t)row * n_out + t])) : 0.0f;
+        const uint64_t x2 = f32x2_pack(x, x);
+        const uint16_t *wr = p.WO + (int64_t)t * p.o + n0 + hc * (BN / 2);
+#pragma unroll
+        for (int g = 0; g < BN / 16; ++g) {
+          uint4 w8 = make_uint4(0u, 0u, 0u, 0u);
+          if (n0 + hc * (BN / 2) + 8 * g < p.o)
+            w8 = __ldcg(reinterpret_cast<const uint4 *>(wr + 8 * g));
+          const uint32_t ww[4] = {w8.x, w8.y, w8.z, w8.w};
+          uint64_t *e = e2[g / 4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&ww[u]));
+            e[4 * (g % 4) + u] = f32x2_fma(x2, f32x2_pack(f.x, f.y), e[4 * (g % 4) + u]);
+          }
+        }
+      }
+      // (4) accumulator; a timeout in any epilogue thread stops all of them
       const bool ready = mbar_wait_bounded(tfull_bar(acc), acc_par, abort_flag, p.status,
                                            LLMINT8_DEV_TIMEOUT_EPILOGUE, p.timeout_ns);
       if (named_barrier_or(EPI_BARRIER, NUM_EPI_THREADS, !ready)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + ((uint32_t)(ew * 32) << 16) + acc * BN + hc * (BN / 2);
-#pragma unroll 1
+#pragma unroll
       for (int c = 0; c < BN / 64; ++c) {
         uint32_t v[32];
         __syncwarp();
         tmem_ld_32x32b_x32(t_row + c * 32, v);
+        // the staging block is free once the previous store has read it
+        if (lane == 0) bulk_wait_group_read0();
         tmem_ld_wait();
+        __syncwarp();
         if (c == BN / 64 - 1) {
           // the accumulator is fully read: hand it back to the MMA warp
           tc_fence_before();
           mbar_arrive(tempty_bar(acc));
         }
-        // outlier product e = sum_t xo[t] * WO[t][j], then
         // out = fp16(ci * (rs * aw[j]) + e), two columns per packed op
-        uint64_t e2[16];
-#pragma unroll
-        for (int q = 0; q < 16; ++q) e2[q] = 0ull;
-#pragma unroll
-        for (int t = 0; t < FAST_OUTLIERS; ++t) {
-          if (t < n_fast) {
-            const uint64_t x2 = f32x2_pack(xo[t], xo[t]);
-            const float4 *wrow =
-                reinterpret_cast<const float4 *>(sWO + t * BN + hc * (BN / 2) + c * 32);
-#pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4) {
-              const float4 w = wrow[q4];
-              e2[2 * q4] = f32x2_fma(x2, f32x2_pack(w.x, w.y), e2[2 * q4]);
-              e2[2 * q4 + 1] = f32x2_fma(x2, f32x2_pack(w.z, w.w), e2[2 * q4 + 1]);
-            }
-          }
-        }
         const int32_t j0 = n0 + hc * (BN / 2) + c * 32;
-        if (n_out > FAST_OUTLIERS) {
-          // outlier columns beyond the shared-memory fast path (|O| > 16)
-          float ef[32];
-#pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            ef[2 * q] = f32x2_lo(e2[q]);
-            ef[2 * q + 1] = f32x2_hi(e2[q]);
-          }
-          for (int32_t t = FAST_OUTLIERS; t < n_out; ++t) {
-            const float x =
-                row_ok ? __half2float(__ushort_as_half(p.XO[(int64_t)row * n_out + t])) : 0.0f;
-            const uint16_t *wr = p.WO + (int64_t)t * p.o;
-#pragma unroll
-            for (int q = 0; q < 32; ++q) {
-              const float w =
-                  (j0 + q < p.o) ? __half2float(__ushort_as_half(__ldcg(wr + j0 + q))) : 0.0f;
-              ef[q] = fmaf(x, w, ef[q]);
-            }
-          }
-#pragma unroll
-          for (int q = 0; q < 16; ++q) e2[q] = f32x2_pack(ef[2 * q], ef[2 * q + 1]);
-        }
+        // 8 outputs at a time into the 64B-swizzled 32x32 staging block;
+        // chunk k of row r lives at 16-byte slot k ^ ((r / 2) % 4)
         const uint64_t rs2 = f32x2_pack(rs, rs);
-        uint32_t h2[16];  // fp16 pairs of the 32 outputs
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          const float4 a4 = *reinterpret_cast<const float4 *>(sAW + hc * (BN / 2) + c * 32 + 4 * q4);
-          const uint64_t sv0 = f32x2_mul(rs2, f32x2_pack(a4.x, a4.y));
-          const uint64_t sv1 = f32x2_mul(rs2, f32x2_pack(a4.z, a4.w));
-          const uint64_t c0 = f32x2_pack((float)(int32_t)v[4 * q4], (float)(int32_t)v[4 * q4 + 1]);
-          const uint64_t c1 =
-              f32x2_pack((float)(int32_t)v[4 * q4 + 2], (float)(int32_t)v[4 * q4 + 3]);
-          const uint64_t r0 = f32x2_fma(c0, sv0, e2[2 * q4]);
-          const uint64_t r1 = f32x2_fma(c1, sv1, e2[2 * q4 + 1]);
-          h2[2 * q4] = f2h2(f32x2_lo(r0), f32x2_hi(r0));
-          h2[2 * q4 + 1] = f2h2(f32x2_lo(r1), f32x2_hi(r1));
-        }
-        // stage 32 fp16 (64 bytes) of this row into the 64B-swizzled 32x32
-        // block; chunk k of row r lives at 16-byte slot k ^ ((r / 2) % 4)
-        if (lane == 0) bulk_wait_group_read0();  // the previous store has read it
-        __syncwarp();
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8) {
-          const uint4 h8 = make_uint4(h2[4 * q8], h2[4 * q8 + 1], h2[4 * q8 + 2], h2[4 * q8 + 3]);
-          *reinterpret_cast<uint4 *>(sOut + lane * 64 + ((q8 ^ ((lane >> 1) & 3)) * 16)) = h8;
+          uint32_t h8[4];  // fp16 pairs
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int q4 = 2 * q8 + u;
+            const float4 a4 =
+                *reinterpret_cast<const float4 *>(sAW + hc * (BN / 2) + c * 32 + 4 * q4);
+            const uint64_t sv0 = f32x2_mul(rs2, f32x2_pack(a4.x, a4.y));
+            const uint64_t sv1 = f32x2_mul(rs2, f32x2_pack(a4.z, a4.w));
+            const uint64_t c0 =
+                f32x2_pack((float)(int32_t)v[4 * q4], (float)(int32_t)v[4 * q4 + 1]);
+            const uint64_t c1 =
+                f32x2_pack((float)(int32_t)v[4 * q4 + 2], (float)(int32_t)v[4 * q4 + 3]);
+            const uint64_t r0 = f32x2_fma(c0, sv0, e2[c][2 * q4]);
+            const uint64_t r1 = f32x2_fma(c1, sv1, e2[c][2 * q4 + 1]);
+            h8[2 * u] = f2h2(f32x2_lo(r0), f32x2_hi(r0));
+            h8[2 * u + 1] = f2h2(f32x2_lo(r1), f32x2_hi(r1));
+          }
+          *reinterpret_cast<uint4 *>(sOut + lane * 64 + ((q8 ^ ((lane >> 1) & 3)) * 16)) =
+              make_uint4(h8[0], h8[1], h8[2], h8[3]);
         }
         fence_proxy_async_smem();
         __syncwarp();
