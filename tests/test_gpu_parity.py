@@ -161,6 +161,29 @@ def test_workload_matmul_with_fp16_outlier_rows(name):
     torch.cuda.empty_cache()
 
 
+# More output tiles than SMs, with a ragged last wave, checked element by
+# element: ragged k (h = 1040) and o (60 full tiles + 16 columns), |O| = 17
+# (outlier rows beyond the shared-memory ones), an 8-row case forced onto
+# the prefill kernel, and two full waves plus two tiles.
+MANY_TILES = [
+    (300, 1040, 15376, tuple(range(3, 1040, 61)), 6.0),
+    (8, 512, 40960, (5, 300), 6.0),
+    (129, 4096, 38144, (11, 4000), 6.0),
+]
+
+
+@pytest.mark.parametrize("case", MANY_TILES, ids=lambda c: f"{c[0]}x{c[1]}x{c[2]}")
+def test_matmul_many_tiles_bit_exact_int32(case):
+    X, W, alpha = _small_inputs(case, seed=21)
+    pw, _ = gpu_prepare(W)
+    Wq_ref, aw_ref = oracle.prepare_weight(W)
+    ref, ci_ref = oracle.matmul(X, Wq_ref, aw_ref, alpha, want_ci=True)
+    for rep in range(2):  # the second call reuses the workspace
+        out, ci, _ = gpu_matmul(X, pw, alpha, path=1, want_ci=True)
+        assert np.array_equal(ci, ci_ref), f"int32 accumulators, call {rep}"
+        assert_close_fp16(out, ref, f"out, call {rep}")
+
+
 # Tensor-wise baselines ("Quantization Primitives"; Table 1 "Int8 absmax"):
 # one absmax for all of X and/or all of W, on the same kernels.
 TENSOR_CASES = [SMALL[i] for i in (0, 2, 4, 5, 6, 9, 11, 12)]
