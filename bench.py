@@ -23,6 +23,7 @@ on a bounded row sample of the same workload per step.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -153,6 +154,15 @@ class ClockSampler:
 
 # ------------------------------------------------------------ CPU oracle
 
+def with_alpha(wl, args):
+    """The workload with --alpha in place of its threshold, if given."""
+    return wl if args.alpha is None else dataclasses.replace(wl, alpha=args.alpha)
+
+
+def alpha_json(a: float):
+    return a if a != float("inf") else "inf"
+
+
 def cpu_oracle_run(wl, X, Wq, aw, budget_s: float, x_tensor: bool = False):
     """Time the oracle on a row sample sized to about budget_s seconds.
 
@@ -238,6 +248,7 @@ def run_ours(args, world, rank, local):
     build.build()
     binding.load_library()
     wl, X, cols, W = workloads.make_inputs(args.workload)
+    wl = with_alpha(wl, args)
     s, h, o = wl.s, wl.h, wl.o
     Xd = torch.from_numpy(X).to(dev)
     Wd = torch.from_numpy(W).to(dev)
@@ -352,7 +363,7 @@ def run_ours(args, world, rank, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "i8", "data": "synthetic (seeded, OPT-shaped outliers)",
         "config": {"workload": wl.name, "s": s, "h": h, "o": o,
-                   "alpha": wl.alpha, "outlier_cols": int(len(cols)),
+                   "alpha": alpha_json(wl.alpha), "outlier_cols": int(len(cols)),
                    "parallelism": f"replicas x{world}" if world > 1 else "single",
                    "scales": {"x": args.x_scale, "w": args.w_scale},
                    "l2": "flushed (512 MB write) before every timed step"},
@@ -381,6 +392,7 @@ def run_reference(args, world, rank, local):
         return None
     import oracle
     wl, X, cols, W = workloads.make_inputs(args.workload)
+    wl = with_alpha(wl, args)
     Wq, aw = oracle.prepare_weight(W, tensor=args.w_scale == "tensor")
     x_tensor = args.x_scale == "tensor"
     per_step = max(0.2, args.cpu_seconds / max(1, args.steps + args.warmup))
@@ -402,7 +414,7 @@ def run_reference(args, world, rank, local):
         "vs_baseline": None, "dtype": "i8 codes, fp64 accumulation",
         "data": "synthetic (seeded, OPT-shaped outliers)",
         "config": {"workload": wl.name, "s": wl.s, "h": wl.h, "o": wl.o,
-                   "alpha": wl.alpha, "parallelism": "single",
+                   "alpha": alpha_json(wl.alpha), "parallelism": "single",
                    "scales": {"x": args.x_scale, "w": args.w_scale}},
         "cpu_baseline": {"value": value, "unit": UNIT,
                          "cores": oracle.num_threads(), "kind": "oracle",
@@ -423,6 +435,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--alpha", type=float, default=None,
+                    help="outlier threshold instead of the workload's (inf: no "
+                         "decomposition, pure vector-wise int8)")
     ap.add_argument("--x-scale", default="row", choices=["row", "tensor"],
                     help="absmax per row of X (the method) or one per tensor")
     ap.add_argument("--w-scale", default="column", choices=["column", "tensor"],
