@@ -154,6 +154,36 @@ class ClockSampler:
 
 # ------------------------------------------------------------ CPU oracle
 
+def fp16_matmul_ms(X, W, dev, flush, K, Wm, world):
+    """The same product in plain fp16 through cuBLAS (fp32 accumulation),
+    timed like the step (L2 flushed before each): the reference the pages
+    quote their speedups against (Appendix D, Table 5)."""
+    import torch
+    torch.backends.cuda.matmul.allow_fp16_reduced_precision_reduction = False
+    Xd = torch.from_numpy(X).to(dev)
+    Wd = torch.from_numpy(W).to(dev)
+    out = torch.empty((X.shape[0], W.shape[1]), dtype=torch.float16, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(Wm):
+        flush.fill_(1)
+        torch.matmul(Xd, Wd, out=out)
+    ts = []
+    torch.cuda.synchronize()
+    for k in range(K):
+        flush.fill_(k & 0xFF)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        torch.matmul(Xd, Wd, out=out)
+        b.record(stream)
+        ts.append((a, b))
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in ts) / K
+    del Xd, Wd, out
+    torch.cuda.empty_cache()
+    return max_over_ranks(ms, world, dev)
+
+
 def with_alpha(wl, args):
     """The workload with --alpha in place of its threshold, if given."""
     return wl if args.alpha is None else dataclasses.replace(wl, alpha=args.alpha)
@@ -329,6 +359,7 @@ def run_ours(args, world, rank, local):
         e_ms.append(a.elapsed_time(b))
     barrier(world)
     e2e_ms = max_over_ranks(sum(e_ms) / K, world, dev)
+    fp16_ms = None if args.no_fp16_ref else fp16_matmul_ms(X, W, dev, flush, K, Wm, world)
 
     ops = 2.0 * s * h * o
     value = world * ops / (ms_per_step * 1e-3) / 1e12
@@ -373,6 +404,10 @@ def run_ours(args, world, rank, local):
         "gpu_launches": launches_per_step * K,
         "roofline": roof,
         "device_status": status_bits,
+        "fp16_matmul": None if fp16_ms is None else {
+            "ms_per_step": fp16_ms, "speedup": fp16_ms / ms_per_step,
+            "what": "torch.matmul of the fp16 X and W (cuBLAS, fp32 accumulation), "
+                    "timed like the step: the pages' Table 5 baseline"},
     }
     if clocks:
         line["clocks"] = clocks.summary(t_wall0, t_wall1)
@@ -435,6 +470,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-fp16-ref", action="store_true",
+                    help="skip timing the plain fp16 cuBLAS product for context")
     ap.add_argument("--alpha", type=float, default=None,
                     help="outlier threshold instead of the workload's (inf: no "
                          "decomposition, pure vector-wise int8)")

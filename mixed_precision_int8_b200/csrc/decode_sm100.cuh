@@ -356,7 +356,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int ew = warp - EPI_WARP0;
     const int et = threadIdx.x - EPI_WARP0 * 32;  // 0..127: one tile column
     const int32_t n_out = *p.n_out;
+    const int32_t nf = n_out < 16 ? n_out : 16;
     __shared__ int last_arrival;
+    // the row scales (over 16129) and the first 16 outlier activations of
+    // every row, shared by all columns of every tile this CTA finishes
+    __shared__ float s_rs[MAX_ROWS];
+    __shared__ float s_xo[MAX_ROWS][16];
+    for (int q = et; q < MAX_ROWS * 16; q += NUM_EPI_THREADS) {
+      const int i = q / 16, t = q % 16;
+      s_xo[i][t] = (i < p.s && t < nf)
+                       ? __half2float(__ushort_as_half(__ldg(p.XO + (int64_t)i * n_out + t)))
+                       : 0.0f;
+      if (t == 0) s_rs[i] = i < p.s ? __ldg(p.ax + i) * (1.0f / 16129.0f) : 0.0f;
+    }
+    named_barrier(EPI_BARRIER, NUM_EPI_THREADS);
     int32_t it = 0;
     for (int64_t u = u0; u < u1; ++it) {
       const int64_t m_blk = u / nk;
@@ -403,27 +416,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       named_barrier(EPI_BARRIER, NUM_EPI_THREADS);
       if (last_arrival && j < p.o) {
+        // every load of this column is issued before the first use: its
+        // scale, its outlier weights and the s int32 sums (one round trip)
         __threadfence();
         const float awj = __ldcg(p.aw + j);
         float wo[16];
-        const int32_t nf = n_out < 16 ? n_out : 16;
 #pragma unroll
         for (int t = 0; t < 16; ++t)
           wo[t] = (t < nf) ? __half2float(__ushort_as_half(__ldcg(p.WO + (int64_t)t * p.o + j)))
                            : 0.0f;
-        for (int32_t i = 0; i < p.s; ++i) {
-          const int32_t c = __ldcg(p.cacc + (int64_t)i * p.o + j);
-          float acc_f = (float)c * (__ldg(p.ax + i) * (1.0f / 16129.0f)) * awj;
-          const uint16_t *xo = p.XO + (int64_t)i * n_out;
+        int32_t cv[MAX_ROWS];
 #pragma unroll
-          for (int t = 0; t < 16; ++t)
-            if (t < nf) acc_f = fmaf(__half2float(__ushort_as_half(__ldcg(xo + t))), wo[t], acc_f);
-          for (int32_t t = 16; t < n_out; ++t)
-            acc_f = fmaf(__half2float(__ushort_as_half(__ldcg(xo + t))),
-                         __half2float(__ushort_as_half(__ldcg(p.WO + (int64_t)t * p.o + j))),
-                         acc_f);
-          p.out[(int64_t)i * p.o + j] = __half_as_ushort(__float2half_rn(acc_f));
-          if (p.ci) p.ci[(int64_t)i * p.o + j] = c;
+        for (int i = 0; i < MAX_ROWS; ++i)
+          cv[i] = i < p.s ? __ldcg(p.cacc + (int64_t)i * p.o + j) : 0;
+#pragma unroll
+        for (int i = 0; i < MAX_ROWS; ++i) {
+          if (i < p.s) {
+            float acc_f = (float)cv[i] * s_rs[i] * awj;
+#pragma unroll
+            for (int t = 0; t < 16; ++t) acc_f = fmaf(s_xo[i][t], wo[t], acc_f);
+            for (int32_t t = 16; t < n_out; ++t)
+              acc_f = fmaf(
+                  __half2float(__ushort_as_half(__ldcg(p.XO + (int64_t)i * n_out + t))),
+                  __half2float(__ushort_as_half(__ldcg(p.WO + (int64_t)t * p.o + j))), acc_f);
+            p.out[(int64_t)i * p.o + j] = __half_as_ushort(__float2half_rn(acc_f));
+            if (p.ci) p.ci[(int64_t)i * p.o + j] = cv[i];
+          }
         }
       }
       u = seg_end;
