@@ -64,3 +64,21 @@ def test_reference_arm_under_torchrun_prints_one_line_from_rank_zero():
     assert d["impl"] == "reference" and d["n_gpus"] == 2
     assert d["cpu_baseline"]["kind"] == "oracle" and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_threshold_and_scale_options_reach_the_workload_and_the_json_line():
+    """--alpha replaces the workload's threshold (inf: pure vector-wise), is
+    written as a JSON-safe value, and the scale flags map onto the library's
+    modes."""
+    sys.path.insert(0, ROOT)
+    import argparse
+    import bench
+    from mixed_precision_int8_b200 import workloads
+    wl = workloads.get_workload("tiny")
+    same = bench.with_alpha(wl, argparse.Namespace(alpha=None))
+    assert same.alpha == wl.alpha
+    off = bench.with_alpha(wl, argparse.Namespace(alpha=float("inf")))
+    assert off.alpha == float("inf") and off.s == wl.s and off.h == wl.h
+    assert json.loads(json.dumps({"alpha": bench.alpha_json(off.alpha)})) == {"alpha": "inf"}
+    assert bench.alpha_json(6.0) == 6.0
+    assert bench.SCALE_MODES == {"row": 0, "column": 0, "tensor": 1}
