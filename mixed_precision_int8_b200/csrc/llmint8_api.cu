@@ -765,6 +765,11 @@ llmint8_status llmint8_matmul_host_ex(const uint16_t *X_host, int64_t s, const l
   if (opts) opts->launches = 0;
   llmint8_status rc = validate_weight(w);
   if (rc) return rc;
+  // the options are checked here too, so that a bad one enqueues no copy
+  if (opts && (opts->path < 0 || opts->path > 2 || (opts->path == 2 && s > kDecodeMaxRows) ||
+               (opts->x_scale != LLMINT8_SCALE_VECTORWISE &&
+                opts->x_scale != LLMINT8_SCALE_TENSORWISE)))
+    return LLMINT8_ERR_ARG;
   if (s < 0 || s > (int64_t)INT32_MAX) return LLMINT8_ERR_SHAPE;
   if ((rc = check_alpha(alpha))) return rc;
   if (s == 0) return LLMINT8_OK;

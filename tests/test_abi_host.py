@@ -167,6 +167,30 @@ def test_prepare_and_quantize_rows_validation(lib):
     assert lib.llmint8_quantize_rows(*bad) == -1
 
 
+def test_scale_mode_constants_match_the_header():
+    text = open(HEADER).read()
+    got = dict(re.findall(r"#define\s+LLMINT8_SCALE_(\w+)\s+(\d+)", text))
+    assert int(got["VECTORWISE"]) == binding.SCALE_VECTORWISE
+    assert int(got["TENSORWISE"]) == binding.SCALE_TENSORWISE
+
+
+@needs_no_gpu
+def test_scale_modes_are_validated_on_the_host(lib):
+    w = _weight(256, 256)
+    assert lib.llmint8_prepare_weight_ex(FAKE, 256, 256, 2, ctypes.byref(w), None) == -7
+    nb = lib.llmint8_quantize_rows_scratch_size(256)
+    assert lib.llmint8_quantize_rows_ex(FAKE, 4, 256, 6.0, -1, FAKE, FAKE, FAKE, FAKE,
+                                        FAKE, FAKE, nb, None) == -7
+    big = 1 << 40
+    for bad in (2, -1):
+        opts = binding.llmint8_matmul_opts()
+        opts.x_scale = bad
+        assert lib.llmint8_matmul_ex(FAKE, 4, ctypes.byref(w), 6.0, FAKE, FAKE, big,
+                                     ctypes.byref(opts), None) == -7
+        assert lib.llmint8_matmul_host_ex(FAKE, 4, ctypes.byref(w), 6.0, FAKE, FAKE, big,
+                                          ctypes.byref(opts), None) == -7
+
+
 @needs_no_gpu
 def test_noalloc_size_limit_is_checked_on_the_host(lib):
     s, h, o = 16, 4096, 8192
