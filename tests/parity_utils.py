@@ -73,3 +73,13 @@ def oracle_prepared(W: np.ndarray, cols=None):
     if cols is None:
         return oracle.prepare_weight(W)
     return oracle.prepare_weight(np.ascontiguousarray(W[:, cols]))
+
+
+def oracle_prepared_by_blocks(W: np.ndarray, block: int = 4096):
+    """Oracle Wq [o,h] and aw [o] for every column, prepared one block of
+    columns at a time (each column's scale and codes depend on that column
+    alone, so this is the same result with a cache-friendly footprint)."""
+    parts = [oracle.prepare_weight(np.ascontiguousarray(W[:, j:j + block]))
+             for j in range(0, W.shape[1], block)]
+    return (np.concatenate([q for q, _ in parts]),
+            np.concatenate([a for _, a in parts]))

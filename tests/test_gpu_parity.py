@@ -18,7 +18,8 @@ import torch
 import oracle
 from mixed_precision_int8_b200 import binding, build, workloads
 from tests.parity_utils import (assert_close_fp16, gpu_matmul, gpu_prepare,
-                                oracle_prepared, sample_cols, sample_rows,
+                                oracle_prepared, oracle_prepared_by_blocks,
+                                sample_cols, sample_rows,
                                 to_dev)
 
 pytestmark = pytest.mark.gpu
@@ -434,10 +435,14 @@ def test_workload_prepare_weight_bit_exact(name):
 
 @pytest.mark.parametrize("name", workloads.WORKLOAD_ORDER)
 def test_workload_matmul(name):
+    """Every output of the small workloads (s * o <= 2048 * 4096: the tiny
+    case, the 6.7B attention projection and the 175B decode batch), and 256
+    rows x every column of the two large FFN shapes."""
     wl, X, cols, W, pw = _workload(name)
-    rows = sample_rows(wl.s, 48)
-    c = sample_cols(wl.o, 512)
-    Wq_ref, aw_ref = oracle_prepared(W, c)
+    full = wl.s * wl.o <= 2048 * 4096
+    rows = np.arange(wl.s) if full else sample_rows(wl.s, 256)
+    c = np.arange(wl.o)
+    Wq_ref, aw_ref = oracle_prepared_by_blocks(W)
     ref, ci_ref = oracle.matmul(X, Wq_ref, aw_ref, wl.alpha, rows=rows,
                                 want_ci=True)
     paths = [0, 1] if wl.s <= 16 else [0]
