@@ -4,18 +4,28 @@
 A step is one llmint8_matmul call: the whole hot path (outlier detection, row
 quantisation, outlier tiles, int8 tcgen05 GEMM with the fused dequantisation /
 outlier product / fp16 store) on one batch of seeded synthetic input already
-resident in HBM. The metric is effective TOPS = 2*s*h*o / step time.
+resident in HBM. The metric is effective TOPS = 2*s*h*o / step time, with the
+fraction of the layer's roofline max(2*s*h*o / P_int8, compulsory bytes / HBM)
+beside it.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                  [--impl ours|reference]
+                  [--per-shape A,B,..|none] [--impl ours|reference]
+
+The headline workload (default: the OPT-175B-like FFN up-projection, the
+largest single-GPU shape) gives the line's top-level keys; the other
+OPT-shaped workloads follow in ``per_shape`` with the same fields.
 
 Timing: W untimed warm-up steps; then exactly K steps between a barrier +
 synchronize on both sides, each step timed with CUDA events on the launching
-stream. The L2 cache (126 MB) is flushed by writing a 512 MB buffer before
-every timed step (outside the step's events), because the default workload's
-inputs fit in L2. Multi-GPU (torchrun): independent replicas on every rank
-(the layer has no exchange step), time = max over ranks, value = total work of
-all ranks / that time.
+stream. Where a workload's inputs (X and the int8 weight) fit twice in the
+126 MB L2, a 512 MB buffer is written before every timed step (outside the
+step's events); larger inputs stream from HBM by themselves and nothing is
+flushed. The line's ``config.l2`` says which. SM clocks and throttle reasons
+are sampled with NVML as fast as it answers during the K timed steps; a
+second, longer window of the same steps (``clocks_soak``) repeats them for at
+least half a second. Multi-GPU (torchrun, or --gpus N, which launches it):
+independent replicas on every rank (the layer has no exchange step), time =
+max over ranks, value = total work of all ranks / that time.
 
 --impl reference times the CPU oracle (plain C, OpenMP) on the host cores,
 on a bounded row sample of the same workload per step.
@@ -27,6 +37,7 @@ import dataclasses
 import hashlib
 import json
 import os
+import socket
 import statistics
 import subprocess
 import sys
@@ -43,8 +54,15 @@ from mixed_precision_int8_b200 import workloads  # noqa: E402
 
 METRIC = "LLM.int8() matmul effective TOPS"
 UNIT = "TOPS"
-DEFAULT_WORKLOAD = "opt6.7b_attn_prefill"
+DEFAULT_WORKLOAD = "opt175b_ffn_up_prefill"
+DEFAULT_PER_SHAPE = ("opt6.7b_attn_prefill", "opt13b_ffn_up_prefill",
+                     "opt175b_decode")
+L2_BYTES = 126 << 20
 FLUSH_BYTES = 512 << 20
+# per-shape entries time at least this many steps (short bursts, like the
+# headline's K steps, so no entry runs long enough to meet the power cap)
+PER_SHAPE_MIN_STEPS = 50
+SOAK_MIN_S = 0.5
 # scale granularity flags -> LLMINT8_SCALE_VECTORWISE (0) / TENSORWISE (1)
 SCALE_MODES = {"row": 0, "column": 0, "tensor": 1}
 KERNEL_SOURCES = ["mixed_precision_int8_b200/csrc/gemm_sm100.cuh",
@@ -88,17 +106,40 @@ def recorded_traffic(workload: str, kernel: str):
     return e.get("dram_bytes_per_launch")
 
 
+def l2_policy(wl) -> str:
+    """How the cache is kept out of the measurement for this workload."""
+    inputs = 2 * wl.s * wl.h + wl.h * wl.o
+    if inputs > 2 * L2_BYTES:
+        return (f"inputs larger than L2 (X + int8 W = {inputs / 1e6:.0f} MB > "
+                f"2 x 126 MB): no flush")
+    return "flushed (512 MB write) before every timed step"
+
+
+def needs_flush(wl) -> bool:
+    return 2 * wl.s * wl.h + wl.h * wl.o <= 2 * L2_BYTES
+
+
+def workload_config(wl, world: int, args) -> dict:
+    """The line's `config`: the same keys and values in both arms."""
+    return {"workload": wl.name, "s": wl.s, "h": wl.h, "o": wl.o,
+            "alpha": alpha_json(wl.alpha), "outlier_cols": wl.n_outlier_cols,
+            "parallelism": f"replicas x{world}" if world > 1 else "single",
+            "scales": {"x": args.x_scale, "w": args.w_scale},
+            "l2": l2_policy(wl)}
+
+
 # ----------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """Samples SM clock and throttle reasons with NVML in a thread."""
+    """Samples SM clock and throttle reasons with NVML in a thread, as fast
+    as NVML answers (a short sleep between reads)."""
 
     REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown",
                0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap",
                0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle",
                0x2: "applications_clocks_setting"}
 
-    def __init__(self, index: int, period_s: float = 0.002):
+    def __init__(self, index: int, period_s: float = 0.0002):
         self.samples = []
         self.ok = False
         self.period = period_s
@@ -135,6 +176,7 @@ class ClockSampler:
         if self._t is not None:
             self._stop.set()
             self._t.join()
+            self._t = None
 
     def summary(self, t0: float, t1: float):
         if not self.ok or not self.samples:
@@ -148,7 +190,7 @@ class ClockSampler:
         reasons = sorted(n for b, n in self.REASONS.items()
                          if bits & b and n != "gpu_idle")
         return {"sm_mhz": mhz, "sm_max_mhz": self.max_mhz, "reasons": reasons,
-                "samples": len(inside),
+                "samples": len(inside), "window_s": round(t1 - t0, 4),
                 "window": "timed region" if inside else "whole run"}
 
 
@@ -156,8 +198,8 @@ class ClockSampler:
 
 def fp16_matmul_ms(X, W, dev, flush, K, Wm, world):
     """The same product in plain fp16 through cuBLAS (fp32 accumulation),
-    timed like the step (L2 flushed before each): the reference the pages
-    quote their speedups against (Appendix D, Table 5)."""
+    timed like the step: the reference the pages quote their speedups
+    against (Appendix D, Table 5)."""
     import torch
     torch.backends.cuda.matmul.allow_fp16_reduced_precision_reduction = False
     Xd = torch.from_numpy(X).to(dev)
@@ -165,12 +207,14 @@ def fp16_matmul_ms(X, W, dev, flush, K, Wm, world):
     out = torch.empty((X.shape[0], W.shape[1]), dtype=torch.float16, device=dev)
     stream = torch.cuda.current_stream()
     for _ in range(Wm):
-        flush.fill_(1)
+        if flush is not None:
+            flush.fill_(1)
         torch.matmul(Xd, Wd, out=out)
     ts = []
     torch.cuda.synchronize()
     for k in range(K):
-        flush.fill_(k & 0xFF)
+        if flush is not None:
+            flush.fill_(k & 0xFF)
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record(stream)
@@ -193,15 +237,12 @@ def alpha_json(a: float):
     return a if a != float("inf") else "inf"
 
 
-def cpu_oracle_run(wl, X, Wq, aw, budget_s: float, x_tensor: bool = False):
-    """Time the oracle on a row sample sized to about budget_s seconds.
-
-    The sample is grown by 4x until a run takes a quarter of the budget (the
-    outlier set is always computed over all rows, a fixed cost), then scaled
-    to the budget and timed once more."""
+def oracle_rows_for(wl, X, Wq, aw, budget_s: float, x_tensor: bool = False):
+    """Number of rows of a sample that the oracle runs in about budget_s
+    (grown by 4x until a run takes a quarter of the budget; the outlier set
+    is always computed over all rows, a fixed cost)."""
     import oracle
-    rng = np.random.default_rng(123)
-    order = rng.permutation(wl.s)
+    order = np.random.default_rng(123).permutation(wl.s)
 
     def timed(n):
         rows = np.sort(order[:n])
@@ -214,9 +255,17 @@ def cpu_oracle_run(wl, X, Wq, aw, budget_s: float, x_tensor: bool = False):
     while el < budget_s / 4 and n < wl.s:
         n = min(wl.s, n * 4)
         el = timed(n)
-    n_final = int(max(1, min(wl.s, n * budget_s / max(el, 1e-6))))
-    if n_final != n:
-        n, el = n_final, timed(n_final)
+    return int(max(1, min(wl.s, n * budget_s / max(el, 1e-6)))), order
+
+
+def cpu_oracle_run(wl, X, Wq, aw, budget_s: float, x_tensor: bool = False):
+    """Time the oracle once on a row sample sized to about budget_s."""
+    import oracle
+    n, order = oracle_rows_for(wl, X, Wq, aw, budget_s, x_tensor)
+    rows = np.sort(order[:n])
+    t = time.perf_counter()
+    oracle.matmul(X, Wq, aw, wl.alpha, rows=rows, x_tensor=x_tensor)
+    el = time.perf_counter() - t
     tops = 2.0 * n * wl.h * wl.o / el / 1e12
     return {"value": tops, "unit": UNIT, "cores": oracle.num_threads(),
             "kind": "oracle",
@@ -267,17 +316,48 @@ def finish(world):
         dist.destroy_process_group()
 
 
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def launch_command(n: int, argv) -> list:
+    """torchrun command that runs this script on n local ranks."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            "--nproc-per-node", str(n), "--master-addr", "127.0.0.1",
+            "--master-port", str(_free_port()), os.path.abspath(__file__)] + list(argv)
+
+
+def check_world(n_gpus: int, env) -> str:
+    """'run' (this process is one of the n ranks), 'launch' (start n ranks
+    with torchrun) or an error message when --gpus and the launcher disagree."""
+    world = env.get("WORLD_SIZE")
+    if world is None:
+        return "run" if n_gpus == 1 else "launch"
+    if int(world) != n_gpus:
+        return (f"--gpus {n_gpus} but WORLD_SIZE={world}: launch one rank per "
+                f"GPU with torchrun --nproc-per-node {n_gpus}")
+    return "run"
+
+
 # ------------------------------------------------------------- our path
 
-def run_ours(args, world, rank, local):
-    import torch
-    from mixed_precision_int8_b200 import binding, build
+def layer_roofline_ms(wl, peaks) -> float:
+    """Roofline time of the whole layer: the slower of the int8 tensor peak
+    and the compulsory bytes at the measured HBM bandwidth."""
+    p_int8 = 2.0 * peaks["bf16_tflops"] * 1e12
+    return max(wl.int8_ops / p_int8, wl.compulsory_bytes / (peaks["hbm_gbs"] * 1e9)) * 1e3
 
-    torch.cuda.set_device(local)
+
+def bench_workload(name, args, world, rank, local, K, Wm, headline: bool):
+    """Time one workload; returns the per-shape entry (the headline's keys
+    are the line's top-level keys)."""
+    import torch
+    from mixed_precision_int8_b200 import binding
+
     dev = torch.device("cuda", local)
-    build.build()
-    binding.load_library()
-    wl, X, cols, W = workloads.make_inputs(args.workload)
+    wl, X, cols, W = workloads.make_inputs(name)
     wl = with_alpha(wl, args)
     s, h, o = wl.s, wl.h, wl.o
     Xd = torch.from_numpy(X).to(dev)
@@ -288,35 +368,40 @@ def run_ours(args, world, rank, local):
     del Wd
     out = torch.empty((s, o), dtype=torch.float16, device=dev)
     ws = binding.Workspace(s, h, o, device=dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = (torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+             if needs_flush(wl) else None)
     stream = torch.cuda.current_stream()
-    K, Wm = args.steps, args.warmup
 
     def step(ev=None):
         binding.llmint8_matmul(Xd, pw, wl.alpha, out=out, workspace=ws,
                                events=ev, x_scale=x_mode)
 
     for _ in range(Wm):
-        flush.fill_(1)
+        if flush is not None:
+            flush.fill_(1)
         step()
     torch.cuda.synchronize()
     launches_per_step = binding.llmint8_matmul.last_launches
+    gemm_launch = {-1: "decode kernel", 0: "ordinary", 1: "cooperative",
+                   2: "cooperative, programmatic dependent"}.get(
+        binding.llmint8_matmul.last_gemm_launch, "unknown")
 
-    def timed_steps(with_kernel_events: bool):
-        """K steps, each between CUDA events on the launching stream, with
-        an L2 flush before every step outside the events. With
-        with_kernel_events, the library also records events around its
-        GEMM/decode kernel (which turns off that launch's overlap with the
-        kernel before it, so the step time is taken without them)."""
-        starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-        stops = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-        g0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-        g1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    def timed_steps(n, with_kernel_events: bool):
+        """n steps, each between CUDA events on the launching stream (after
+        an L2 flush outside the events, where the workload needs one). With
+        with_kernel_events the library also records events around its
+        GEMM/decode kernel, which turns off that launch's overlap with the
+        kernel before it, so the step time is taken without them."""
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        stops = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        g0 = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        g1 = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
         barrier(world)
         torch.cuda.synchronize()
         t0 = time.perf_counter()
-        for k in range(K):
-            flush.fill_(k & 0xFF)
+        for k in range(n):
+            if flush is not None:
+                flush.fill_(k & 0xFF)
             starts[k].record(stream)
             step((g0[k], g1[k]) if with_kernel_events else None)
             stops[k].record(stream)
@@ -328,51 +413,73 @@ def run_ours(args, world, rank, local):
                    if with_kernel_events else None)
         return step_ms, kern_ms, t0, t1
 
+    # headline: exactly K steps; per-shape entries: at least
+    # PER_SHAPE_MIN_STEPS
+    n_steps = K if headline else max(K, PER_SHAPE_MIN_STEPS)
     clocks = ClockSampler(local) if rank == 0 else None
     if clocks:
         clocks.start()
-    step_ms, _, t_wall0, t_wall1 = timed_steps(False)
+    step_ms, _, t_wall0, t_wall1 = timed_steps(n_steps, False)
+    clock_sum = clocks.summary(t_wall0, t_wall1) if clocks else None
+    ms_per_step = max_over_ranks(sum(step_ms) / n_steps, world, dev)
+    # the dominant kernel's own time, right after (same conditions)
+    _, gemm_ms, g_t0, g_t1 = timed_steps(n_steps, True)
+    gemm_ms_avg = sum(gemm_ms) / n_steps
+    kernel_clocks = clocks.summary(g_t0, g_t1) if clocks else None
+    # then a longer window of the same steps (at least SOAK_MIN_S): how the
+    # layer holds up under sustained load, reported beside the K-step numbers
+    soak_ms, soak_t0, soak_t1 = [], None, None
+    if headline and not args.no_soak:
+        # the same number of repetitions on every rank (each has barriers)
+        reps = int(max_over_ranks(
+            float(int(SOAK_MIN_S / max(1e-4, t_wall1 - t_wall0)) + 1), world, dev))
+        soak_t0 = time.perf_counter()
+        for _ in range(reps):
+            ms, _, _, soak_t1 = timed_steps(n_steps, False)
+            soak_ms += ms
     if clocks:
         clocks.stop()
-    ms_per_step = max_over_ranks(sum(step_ms) / K, world, dev)
-    _, gemm_ms, _, _ = timed_steps(True)
-    gemm_ms_avg = sum(gemm_ms) / K
     status_bits = binding.llmint8_read_device_status(ws)
 
     # end to end through the host-buffer entry point
-    Xh = torch.from_numpy(X).pin_memory()
-    outh = torch.empty((s, o), dtype=torch.float16).pin_memory()
-    wsh = binding.Workspace(s, h, o, device=dev, host=True)
-    for _ in range(max(1, Wm)):
-        binding.llmint8_matmul_host(Xh, pw, wl.alpha, outh, wsh, x_scale=x_mode)
-    e_ms = []
-    barrier(world)
-    torch.cuda.synchronize()
-    for k in range(K):
-        flush.fill_(k & 0xFF)
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        binding.llmint8_matmul_host(Xh, pw, wl.alpha, outh, wsh, x_scale=x_mode)
-        b.record(stream)
-        b.synchronize()
-        e_ms.append(a.elapsed_time(b))
-    barrier(world)
-    e2e_ms = max_over_ranks(sum(e_ms) / K, world, dev)
-    fp16_ms = None if args.no_fp16_ref else fp16_matmul_ms(X, W, dev, flush, K, Wm, world)
+    e2e_ms = None
+    if not args.no_e2e:
+        Xh = torch.from_numpy(X).pin_memory()
+        outh = torch.empty((s, o), dtype=torch.float16).pin_memory()
+        wsh = binding.Workspace(s, h, o, device=dev, host=True)
+        for _ in range(max(1, Wm)):
+            binding.llmint8_matmul_host(Xh, pw, wl.alpha, outh, wsh, x_scale=x_mode)
+        e_ms = []
+        barrier(world)
+        torch.cuda.synchronize()
+        for k in range(n_steps):
+            if flush is not None:
+                flush.fill_(k & 0xFF)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            binding.llmint8_matmul_host(Xh, pw, wl.alpha, outh, wsh, x_scale=x_mode)
+            b.record(stream)
+            b.synchronize()
+            e_ms.append(a.elapsed_time(b))
+        barrier(world)
+        e2e_ms = max_over_ranks(sum(e_ms) / n_steps, world, dev)
+        del wsh, Xh, outh
+    fp16_ms = None if args.no_fp16_ref else fp16_matmul_ms(X, W, dev, flush, n_steps, Wm, world)
 
     ops = 2.0 * s * h * o
     value = world * ops / (ms_per_step * 1e-3) / 1e12
-    e2e_value = world * ops / (e2e_ms * 1e-3) / 1e12
+    e2e_value = None if e2e_ms is None else world * ops / (e2e_ms * 1e-3) / 1e12
     peaks = measured_peaks()
     decode = s <= binding.llmint8_decode_max_rows()
     if decode:
         kernel = "k_decode_i8"
-        algo_bytes = h * o + 16 * h  # int8 weight + padded int8 rows
+        # int8 weight + int8 rows + fp16 output + scales
+        algo_bytes = h * o + s * h + 2 * s * o + 4 * (s + o)
         achieved = algo_bytes / (gemm_ms_avg * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                "kernel": kernel,
+                "kernel": kernel, "algorithmic_bytes": algo_bytes,
                 "peak_source": f"hbm_gbs ({peaks['source']})"}
     else:
         kernel = "k_gemm_i8_fused"
@@ -385,93 +492,141 @@ def run_ours(args, world, rank, local):
     roof["traffic"] = recorded_traffic(wl.name, kernel)
     roof["kernel_ms"] = gemm_ms_avg
     roof["kernel_timing"] = ("CUDA events recorded by the library around "
-                             "this kernel, averaged over a second pass of K "
-                             "steps (same flushes)")
-
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-        "steps": K, "warmup": Wm, "ms_per_step": ms_per_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "i8", "data": "synthetic (seeded, OPT-shaped outliers)",
-        "config": {"workload": wl.name, "s": s, "h": h, "o": o,
-                   "alpha": alpha_json(wl.alpha), "outlier_cols": int(len(cols)),
-                   "parallelism": f"replicas x{world}" if world > 1 else "single",
-                   "scales": {"x": args.x_scale, "w": args.w_scale},
-                   "l2": "flushed (512 MB write) before every timed step"},
-        "e2e": {"value": e2e_value, "unit": UNIT,
-                "h2d_bytes_per_step": 2 * s * h,
-                "d2h_bytes_per_step": 2 * s * o},
-        "gpu_launches": launches_per_step * K,
+                             "this kernel, averaged over a second pass of the "
+                             "same steps right after the timed one")
+    roof["kernel_clocks"] = kernel_clocks
+    entry = {
+        "workload": wl.name, "value": value, "unit": UNIT,
+        "ms_per_step": ms_per_step, "steps": n_steps,
+        "step_roofline_frac": layer_roofline_ms(wl, peaks) / ms_per_step,
+        "config": workload_config(wl, world, args),
+        "e2e": None if e2e_value is None else {
+            "value": e2e_value, "unit": UNIT,
+            "h2d_bytes_per_step": 2 * s * h,
+            "d2h_bytes_per_step": 2 * s * o},
+        "gpu_launches": launches_per_step * n_steps,
+        "gemm_launch": gemm_launch,
         "roofline": roof,
         "device_status": status_bits,
         "fp16_matmul": None if fp16_ms is None else {
             "ms_per_step": fp16_ms, "speedup": fp16_ms / ms_per_step,
             "what": "torch.matmul of the fp16 X and W (cuBLAS, fp32 accumulation), "
                     "timed like the step: the pages' Table 5 baseline"},
+        "clocks": clock_sum,
     }
-    if clocks:
-        line["clocks"] = clocks.summary(t_wall0, t_wall1)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        import oracle
+    if headline and soak_t1 is not None:
+        soak = clocks.summary(soak_t0, soak_t1) if clocks else {}
+        soak = dict(soak or {})
+        soak["ms_per_step"] = sum(soak_ms) / len(soak_ms)
+        soak["value"] = world * ops / (soak["ms_per_step"] * 1e-3) / 1e12
+        soak["steps"] = len(soak_ms)
+        soak["what"] = ("the same steps back to back for at least "
+                        f"{SOAK_MIN_S} s after the timed ones (sustained load; "
+                        "the power cap may lower the clock)")
+        entry["clocks_soak"] = soak
+    if headline and rank == 0 and world == 1 and not args.no_cpu_baseline:
         Wq = pw.wq.cpu().numpy()
         aw = pw.aw.cpu().numpy()
-        line["cpu_baseline"] = cpu_oracle_run(wl, X, Wq, aw, args.cpu_seconds,
-                                              x_tensor=args.x_scale == "tensor")
+        entry["cpu_baseline"] = cpu_oracle_run(wl, X, Wq, aw, args.cpu_seconds,
+                                               x_tensor=args.x_scale == "tensor")
+    del pw, ws, out, Xd, flush
+    torch.cuda.empty_cache()
+    return entry
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    from mixed_precision_int8_b200 import binding, build
+
+    torch.cuda.set_device(local)
+    build.build()
+    binding.load_library()
+    K, Wm = args.steps, args.warmup
+    head = bench_workload(args.workload, args, world, rank, local, K, Wm, True)
+    shapes = [] if args.per_shape == "none" else [
+        n for n in (args.per_shape.split(",") if args.per_shape else DEFAULT_PER_SHAPE)
+        if n and n != args.workload]
+    per_shape = [bench_workload(n, args, world, rank, local, K, Wm, False) for n in shapes]
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": Wm, "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "i8", "data": "synthetic (seeded, OPT-shaped outliers)",
+        "config": head["config"], "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"], "gemm_launch": head["gemm_launch"],
+        "roofline": head["roofline"],
+        "step_roofline_frac": head["step_roofline_frac"],
+        "device_status": head["device_status"],
+        "fp16_matmul": head["fp16_matmul"], "clocks": head["clocks"],
+    }
+    for k in ("clocks_soak", "cpu_baseline"):
+        if k in head:
+            line[k] = head[k]
+    line["per_shape"] = per_shape
     return line
 
 
 # ------------------------------------------------------ reference (oracle)
 
-def run_reference(args, world, rank, local):
-    if rank != 0:
-        return None
+def run_reference(args, world):
+    """The CPU oracle on the host cores: each step one row sample of the
+    workload (the same sample every step), sized once during warm-up so that
+    warm-up plus K steps take about --cpu-seconds."""
     import oracle
     wl, X, cols, W = workloads.make_inputs(args.workload)
     wl = with_alpha(wl, args)
     Wq, aw = oracle.prepare_weight(W, tensor=args.w_scale == "tensor")
     x_tensor = args.x_scale == "tensor"
     per_step = max(0.2, args.cpu_seconds / max(1, args.steps + args.warmup))
+    n, order = oracle_rows_for(wl, X, Wq, aw, per_step, x_tensor)
+    rows = np.sort(order[:n])
+
+    def one():
+        t = time.perf_counter()
+        oracle.matmul(X, Wq, aw, wl.alpha, rows=rows, x_tensor=x_tensor)
+        return time.perf_counter() - t
+
     for _ in range(args.warmup):
-        cpu_oracle_run(wl, X, Wq, aw, per_step, x_tensor)
-    vals, samples = [], []
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        r = cpu_oracle_run(wl, X, Wq, aw, per_step, x_tensor)
-        vals.append(r["value"])
-        samples.append(r["sample"])
-    el = time.perf_counter() - t0
-    value = statistics.mean(vals)
-    ms = 2.0 * wl.s * wl.h * wl.o / (value * 1e12) * 1e3
+        one()
+    secs = [one() for _ in range(args.steps)]
+    ms = 1e3 * sum(secs) / len(secs)
+    value = 2.0 * n * wl.h * wl.o / (ms * 1e-3) / 1e12
+    sample = (f"{n} of {wl.s} rows x all {wl.o} columns of {wl.name} per step "
+              f"(outlier set over all rows); {args.steps} steps in {sum(secs):.1f} s")
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "i8 codes, fp64 accumulation",
         "data": "synthetic (seeded, OPT-shaped outliers)",
-        "config": {"workload": wl.name, "s": wl.s, "h": wl.h, "o": wl.o,
-                   "alpha": alpha_json(wl.alpha), "parallelism": "single",
-                   "scales": {"x": args.x_scale, "w": args.w_scale}},
+        "config": workload_config(wl, world, args),
         "cpu_baseline": {"value": value, "unit": UNIT,
                          "cores": oracle.num_threads(), "kind": "oracle",
-                         "sample": f"per step: {samples[-1]}; "
-                                   f"{args.steps} steps in {el:.1f} s"},
+                         "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
 
 
-def main():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     choices=list(workloads.WORKLOADS))
+    ap.add_argument("--per-shape", default=None,
+                    help="comma-separated workloads timed after the headline "
+                         "(default: the other OPT shapes; 'none' for none)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fp16-ref", action="store_true",
                     help="skip timing the plain fp16 cuBLAS product for context")
+    ap.add_argument("--no-soak", action="store_true",
+                    help="skip the sustained-load window (profiling runs)")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the host-buffer end-to-end timing (profiling runs)")
     ap.add_argument("--alpha", type=float, default=None,
                     help="outlier threshold instead of the workload's (inf: no "
                          "decomposition, pure vector-wise int8)")
@@ -479,16 +634,32 @@ def main():
                     help="absmax per row of X (the method) or one per tensor")
     ap.add_argument("--w-scale", default="column", choices=["column", "tensor"],
                     help="absmax per column of W (the method) or one per tensor")
-    args = ap.parse_args()
+    args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if args.per_shape not in (None, "none"):
+        bad = [n for n in args.per_shape.split(",") if n and n not in workloads.WORKLOADS]
+        if bad:
+            ap.error(f"unknown workloads in --per-shape: {bad}")
+    return args
+
+
+def main():
+    args = parse_args()
+    plan = check_world(args.gpus, os.environ)
+    if plan == "launch":
+        sys.exit(subprocess.call(launch_command(args.gpus, sys.argv[1:])))
+    if plan != "run":
+        print(plan, file=sys.stderr)
+        sys.exit(2)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     if args.impl == "reference":
         # rank 0 alone times the CPU oracle; other ranks exit without work
         if int(os.environ.get("RANK", "0")) != 0:
             return
-        line = run_reference(args, 1, 0, 0)
-        line["n_gpus"] = int(os.environ.get("WORLD_SIZE", "1"))
-        print(json.dumps(line), flush=True)
+        print(json.dumps(run_reference(args, world)), flush=True)
         return
     world, rank, local = dist_setup(args.gpus)
     try:

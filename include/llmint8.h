@@ -43,7 +43,11 @@
  *    with one IEEE fp32 division; a == 0 gives q == 0.
  *  - The kernels contain only bounded waits. If one runs out (it should not),
  *    the kernel records a bit in the workspace's status word and returns;
- *    llmint8_read_device_status() reports and clears it.
+ *    llmint8_read_device_status() reports and clears it. A caller that gives
+ *    llmint8_matmul_ex a mapped host status word (opts.status_host) has the
+ *    bits of each call copied there by the call's last kernel, and its next
+ *    call on that word returns LLMINT8_ERR_DEVICE_STATUS without enqueuing
+ *    anything, with no synchronisation.
  *  - Only sm_100 devices are supported; other devices give
  *    LLMINT8_ERR_UNSUPPORTED. There is no CPU fallback.
  */
@@ -70,7 +74,7 @@ typedef enum {
     LLMINT8_ERR_ALIGN = -3,         /* a pointer breaks the alignment rules */
     LLMINT8_ERR_WORKSPACE = -4,     /* workspace smaller than required */
     LLMINT8_ERR_CUDA = -5,          /* a CUDA runtime/driver call failed */
-    LLMINT8_ERR_DEVICE_STATUS = -6, /* a kernel flagged an anomaly */
+    LLMINT8_ERR_DEVICE_STATUS = -6, /* a kernel flagged an anomaly (see status_host) */
     LLMINT8_ERR_ARG = -7,           /* a scalar argument is invalid */
     LLMINT8_ERR_UNSUPPORTED = -8,   /* current device is not sm_100 */
     LLMINT8_ERR_TOO_LARGE = -9      /* problem exceeds the no-alloc scratch */
@@ -83,6 +87,9 @@ typedef enum {
 #define LLMINT8_DEV_TIMEOUT_DRAIN 0x8     /* drain after an abort timed out */
 #define LLMINT8_DEV_TIMEOUT_ROWS 0x10     /* activation row stream gave up waiting */
 #define LLMINT8_DEV_TIMEOUT_SELFTEST 0x20 /* llmint8_wait_selftest's waits ran out */
+#define LLMINT8_DEV_OUTLIER_CAP 0x40      /* |O| above the workspace's outlier
+                                             capacity: the call's output has no
+                                             fp16 outlier product */
 
 /* A prepared (offline-quantised) weight. Buffers are caller-owned device
  * memory: wq_dev is int8 [o][h] (the reduction index k contiguous, i.e. the
@@ -114,7 +121,32 @@ typedef struct {
  *  x_scale: LLMINT8_SCALE_VECTORWISE (0, the method: one absmax per row of
  *      X) or LLMINT8_SCALE_TENSORWISE (one absmax for all of X, the largest
  *      row scale, so every ax[i] is that constant); anything else is
- *      LLMINT8_ERR_ARG. Outlier columns are split off in both modes. */
+ *      LLMINT8_ERR_ARG. Outlier columns are split off in both modes.
+ *  max_outliers: outlier columns the workspace holds (0: h, the default and
+ *      the worst case). The workspace must then hold
+ *      llmint8_workspace_size_ex(s, h, o, max_outliers) bytes. A call whose
+ *      |O| exceeds it writes no outlier tile, skips the fp16 outlier product
+ *      (the output is the int8 part alone; the outlier columns are still
+ *      removed from it) and sets LLMINT8_DEV_OUTLIER_CAP. Negative or above
+ *      h: LLMINT8_ERR_ARG.
+ *  status_host: NULL, or a 4-byte word of pinned host memory that the device
+ *      can address (cudaHostAlloc / cudaMallocHost memory under unified
+ *      addressing; anything else is LLMINT8_ERR_ARG). When the word is
+ *      nonzero on entry the call returns LLMINT8_ERR_DEVICE_STATUS at once;
+ *      otherwise the call's last kernel ORs the workspace's status bits into
+ *      it as it finishes. The caller clears the word, and re-initialises the
+ *      workspace (llmint8_workspace_init), before going on.
+ *  gemm_plain: 0 (automatic): the prefill GEMM is launched cooperatively
+ *      where the device and driver accept it (all its CTAs resident at once);
+ *      its CTAs then build the fp16 outlier rows of W while their first
+ *      mainloops run and wait for each other's shares. Nonzero: an ordinary
+ *      launch, with those rows built by the activation kernels first and no
+ *      CTA of the GEMM waiting for another (for callers that cannot have a
+ *      cooperative launch, e.g. under SM partitioning). Results are the
+ *      same bit for bit.
+ *  gemm_launch (out): how this call launched its int8 GEMM: 0 ordinary,
+ *      1 cooperative, 2 cooperative with programmatic dependent launch
+ *      (overlapping the previous kernel's tail), -1 the decode kernel. */
 typedef struct {
     void *gemm_event_start;
     void *gemm_event_stop;
@@ -122,6 +154,10 @@ typedef struct {
     int32_t path;
     int32_t launches;
     int32_t x_scale;
+    int32_t max_outliers;
+    int32_t *status_host;
+    int32_t gemm_plain;
+    int32_t gemm_launch;
 } llmint8_matmul_opts;
 
 /* Scale granularity ("Quantization Primitives": absmax over a whole tensor;
@@ -140,6 +176,14 @@ LLMINT8_API const char *llmint8_status_string(llmint8_status st);
  * outlier rows of W) + 4*16*o (decode accumulators) + O(h + s). */
 LLMINT8_API size_t llmint8_workspace_size(int64_t s, int64_t h, int64_t o);
 
+/* Workspace for calls whose opts.max_outliers is max_outliers (0: h): the
+ * outlier tiles shrink to 2*s*max_outliers + 2*max_outliers*o bytes. For the
+ * OPT-175B shapes (h = 12288, o = 49152) and 64 outlier columns that is tens
+ * of MB instead of the 1.2 GB of the worst case. 0 if max_outliers is
+ * negative or above h. */
+LLMINT8_API size_t llmint8_workspace_size_ex(int64_t s, int64_t h, int64_t o,
+                                             int64_t max_outliers);
+
 /* Bytes at the front of a workspace that hold state kept between calls: the
  * status words (first 256 bytes), then the outlier bitmask that the one-read
  * activation pass accumulates into and leaves zero when it finishes. */
@@ -155,6 +199,8 @@ LLMINT8_API llmint8_status llmint8_workspace_init(void *ws_dev, size_t ws_bytes,
 /* Workspace for llmint8_matmul_host: llmint8_workspace_size plus staging
  * for the device copies of X (2*s*h bytes) and of C (2*s*o bytes). */
 LLMINT8_API size_t llmint8_workspace_size_host(int64_t s, int64_t h, int64_t o);
+LLMINT8_API size_t llmint8_workspace_size_host_ex(int64_t s, int64_t h, int64_t o,
+                                                  int64_t max_outliers);
 
 /* Offline weight preparation ("The Full LLM.int8() Algorithm", Step 1 remark
  * that W's part is fixed at model-load time, and section "Why vector-wise
@@ -254,6 +300,15 @@ LLMINT8_API llmint8_status llmint8_read_outlier_tiles(const void *ws_dev, size_t
                                           uint16_t *XO_host, uint16_t *WO_host,
                                           void *stream);
 
+/* llmint8_read_outlier_tiles for a call made with opts.max_outliers =
+ * max_outliers (the layout depends on it). When the call's |O| exceeded
+ * that capacity, *n_out_host is still |O| and nothing else is copied. */
+LLMINT8_API llmint8_status llmint8_read_outlier_tiles_ex(const void *ws_dev, size_t ws_bytes,
+                                             int64_t s, int64_t h, int64_t o,
+                                             int64_t max_outliers, int32_t *n_out_host,
+                                             uint16_t *XO_host, uint16_t *WO_host,
+                                             void *stream);
+
 /* Reads and clears the device status word kept in a matmul workspace;
  * synchronises `stream`. Returns LLMINT8_ERR_DEVICE_STATUS if any bit was
  * set (bits also stored in *bits_out when non-NULL), else LLMINT8_OK. */
@@ -299,6 +354,18 @@ LLMINT8_API llmint8_status llmint8_wait_selftest(void *ws_dev, size_t ws_bytes,
 LLMINT8_API llmint8_status llmint8_matmul_noalloc(const uint16_t *X_dev, int64_t s,
                                                   const llmint8_weight *w, float alpha,
                                                   uint16_t *out_dev, void *stream);
+
+/* Status of the allocation-free entry point on the current device (no
+ * counterpart on the pages either). Its kernels record anomalies (a bounded
+ * wait that ran out) in a status word inside the library's scratch array,
+ * where no caller buffer can see them; this reads that word into *bits_out
+ * (when non-NULL), clears it and clears the rest of the array's state block.
+ * Synchronises `stream`. Returns LLMINT8_ERR_DEVICE_STATUS if any bit was
+ * set, else LLMINT8_OK. Each llmint8_matmul_noalloc call starts from a clean
+ * activation state of its own, so a failed call does not spoil later ones,
+ * but its output is wrong and only this function reports it. Before the
+ * first no-alloc call on a device it returns LLMINT8_OK with no bits. */
+LLMINT8_API llmint8_status llmint8_noalloc_read_device_status(int32_t *bits_out, void *stream);
 
 /* Largest s the decode kernel accepts. */
 LLMINT8_API int64_t llmint8_decode_max_rows(void);

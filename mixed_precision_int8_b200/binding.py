@@ -23,6 +23,9 @@ STATUS_NAMES = {0: "OK", -1: "ERR_NULL", -2: "ERR_SHAPE", -3: "ERR_ALIGN",
                 -4: "ERR_WORKSPACE", -5: "ERR_CUDA", -6: "ERR_DEVICE_STATUS",
                 -7: "ERR_ARG", -8: "ERR_UNSUPPORTED", -9: "ERR_TOO_LARGE"}
 NOALLOC_MAX_SCRATCH_BYTES = 64 << 20  # LLMINT8_NOALLOC_MAX_SCRATCH_BYTES
+# device status bits (LLMINT8_DEV_*)
+DEV_TIMEOUT_SELFTEST = 0x20
+DEV_OUTLIER_CAP = 0x40
 SCALE_VECTORWISE = 0  # LLMINT8_SCALE_VECTORWISE: per row of X / column of W
 SCALE_TENSORWISE = 1  # LLMINT8_SCALE_TENSORWISE: one constant per tensor
 
@@ -38,7 +41,9 @@ class llmint8_weight(ctypes.Structure):
 class llmint8_matmul_opts(ctypes.Structure):
     _fields_ = [("gemm_event_start", _vp), ("gemm_event_stop", _vp),
                 ("ci_dev", _vp), ("path", _c_i32), ("launches", _c_i32),
-                ("x_scale", _c_i32)]
+                ("x_scale", _c_i32), ("max_outliers", _c_i32),
+                ("status_host", _vp), ("gemm_plain", _c_i32),
+                ("gemm_launch", _c_i32)]
 
 
 class Llmint8Error(RuntimeError):
@@ -64,7 +69,9 @@ def load_library():
     sig = {
         "llmint8_status_string": ([_c_i32], ctypes.c_char_p),
         "llmint8_workspace_size": ([_c_i64, _c_i64, _c_i64], _sz),
+        "llmint8_workspace_size_ex": ([_c_i64, _c_i64, _c_i64, _c_i64], _sz),
         "llmint8_workspace_size_host": ([_c_i64, _c_i64, _c_i64], _sz),
+        "llmint8_workspace_size_host_ex": ([_c_i64, _c_i64, _c_i64, _c_i64], _sz),
         "llmint8_workspace_init": ([_vp, _sz, _vp], _c_i32),
         "llmint8_prepare_weight": ([_vp, _c_i64, _c_i64,
                                     ctypes.POINTER(llmint8_weight), _vp], _c_i32),
@@ -87,11 +94,14 @@ def load_library():
                                     ctypes.POINTER(llmint8_matmul_opts), _vp], _c_i32),
         "llmint8_read_outlier_tiles": ([_vp, _sz, _c_i64, _c_i64, _c_i64, _vp,
                                         _vp, _vp, _vp], _c_i32),
+        "llmint8_read_outlier_tiles_ex": ([_vp, _sz, _c_i64, _c_i64, _c_i64,
+                                           _c_i64, _vp, _vp, _vp, _vp], _c_i32),
         "llmint8_read_device_status": ([_vp, _sz, _vp, _vp], _c_i32),
         "llmint8_decode_max_rows": ([], _c_i64),
         "llmint8_matmul_noalloc": ([_vp, _c_i64, ctypes.POINTER(llmint8_weight),
                                     _c_f32, _vp, _vp], _c_i32),
         "llmint8_wait_selftest": ([_vp, _sz, ctypes.c_uint64, _vp], _c_i32),
+        "llmint8_noalloc_read_device_status": ([_vp, _vp], _c_i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -109,7 +119,9 @@ EXPORTED = ("llmint8_status_string", "llmint8_workspace_size",
             "llmint8_read_device_status", "llmint8_decode_max_rows",
             "llmint8_matmul_noalloc", "llmint8_wait_selftest",
             "llmint8_prepare_weight_ex", "llmint8_quantize_rows_ex",
-            "llmint8_matmul_host_ex")
+            "llmint8_matmul_host_ex", "llmint8_workspace_size_ex",
+            "llmint8_workspace_size_host_ex", "llmint8_read_outlier_tiles_ex",
+            "llmint8_noalloc_read_device_status")
 
 
 def status_string(code: int) -> str:
@@ -153,22 +165,45 @@ class PreparedWeight:
 
 
 class Workspace:
-    """A caller-owned device workspace (torch uint8 buffer) for one stream."""
+    """A caller-owned device workspace (torch uint8 buffer) for one stream.
 
-    def __init__(self, s: int, h: int, o: int, device=None, host: bool = False):
+    max_outliers (0: h, any alpha) sizes its outlier tiles; calls on it pass
+    the same capacity to the library."""
+
+    def __init__(self, s: int, h: int, o: int, device=None, host: bool = False,
+                 max_outliers: int = 0):
         lib = load_library()
-        size_fn = (lib.llmint8_workspace_size_host if host
-                   else lib.llmint8_workspace_size)
-        self.nbytes = int(size_fn(s, h, o))
+        size_fn = (lib.llmint8_workspace_size_host_ex if host
+                   else lib.llmint8_workspace_size_ex)
+        self.nbytes = int(size_fn(s, h, o, int(max_outliers)))
+        if self.nbytes == 0:
+            raise ValueError(f"invalid workspace size arguments {(s, h, o, max_outliers)}")
         self.buf = torch.empty(self.nbytes, dtype=torch.uint8,
                                device=device or "cuda")
         self.s, self.h, self.o = s, h, o
+        self.max_outliers = int(max_outliers)
         _check("llmint8_workspace_init",
                lib.llmint8_workspace_init(_ptr(self.buf), self.nbytes, _stream()))
 
 
-def llmint8_workspace_size(s: int, h: int, o: int) -> int:
-    return int(load_library().llmint8_workspace_size(s, h, o))
+def llmint8_workspace_size(s: int, h: int, o: int, max_outliers: int = 0) -> int:
+    return int(load_library().llmint8_workspace_size_ex(s, h, o, int(max_outliers)))
+
+
+class HostStatusWord:
+    """A pinned host int32 that the device writes: passed as status_host, it
+    receives the status bits of each call's kernels, and the next call on it
+    raises ERR_DEVICE_STATUS (code -6) before enqueuing anything."""
+
+    def __init__(self):
+        self.t = torch.zeros((1,), dtype=torch.int32).pin_memory()
+
+    @property
+    def value(self) -> int:
+        return int(self.t[0].item())
+
+    def clear(self):
+        self.t[0] = 0
 
 
 def llmint8_decode_max_rows() -> int:
@@ -224,13 +259,18 @@ def llmint8_matmul(X: torch.Tensor, w: PreparedWeight, alpha: float = 6.0,
                    workspace: Optional[Workspace] = None,
                    ci: Optional[torch.Tensor] = None, path: int = 0,
                    events=None, stream=None,
-                   x_scale: int = SCALE_VECTORWISE) -> torch.Tensor:
+                   x_scale: int = SCALE_VECTORWISE,
+                   status_host: Optional[HostStatusWord] = None,
+                   gemm_plain: bool = False) -> torch.Tensor:
     """C = LLM.int8()(X, W): X fp16 [s,h] on the GPU -> fp16 [s,o].
 
     ci (optional, int32 [s,o]) receives the exact int32 accumulators; path
     forces the prefill (1) or decode (2) kernel; events = (start, stop)
     torch.cuda.Event pair recorded around the GEMM kernel; x_scale =
-    SCALE_TENSORWISE quantises X with one constant for the whole tensor.
+    SCALE_TENSORWISE quantises X with one constant for the whole tensor;
+    status_host (a HostStatusWord) reports device anomalies on the next call;
+    gemm_plain forces the ordinary (non-cooperative) prefill GEMM launch.
+    The workspace's max_outliers is passed along.
     """
     _f16_dev(X, "X")
     s, h = X.shape
@@ -243,6 +283,10 @@ def llmint8_matmul(X: torch.Tensor, w: PreparedWeight, alpha: float = 6.0,
     opts = llmint8_matmul_opts()
     opts.path = int(path)
     opts.x_scale = int(x_scale)
+    opts.max_outliers = workspace.max_outliers
+    opts.gemm_plain = int(bool(gemm_plain))
+    if status_host is not None:
+        opts.status_host = status_host.t.data_ptr()
     if ci is not None:
         if ci.dtype != torch.int32 or ci.shape != (s, w.o):
             raise ValueError("ci must be int32 [s,o]")
@@ -259,6 +303,7 @@ def llmint8_matmul(X: torch.Tensor, w: PreparedWeight, alpha: float = 6.0,
         _ptr(workspace.buf), workspace.nbytes, ctypes.byref(opts),
         _stream(stream)))
     llmint8_matmul.last_launches = int(opts.launches)
+    llmint8_matmul.last_gemm_launch = int(opts.gemm_launch)
     return out
 
 
@@ -291,6 +336,7 @@ def llmint8_matmul_host(X_host: torch.Tensor, w: PreparedWeight,
     s, h = X_host.shape
     opts = llmint8_matmul_opts()
     opts.x_scale = int(x_scale)
+    opts.max_outliers = workspace.max_outliers
     _check("llmint8_matmul_host_ex", load_library().llmint8_matmul_host_ex(
         _ptr(X_host), s, ctypes.byref(w.c), float(alpha), _ptr(out_host),
         _ptr(workspace.buf), workspace.nbytes, ctypes.byref(opts), _stream(stream)))
@@ -304,13 +350,16 @@ def llmint8_read_outlier_tiles(workspace: Workspace, s: Optional[int] = None,
     the workspace layout depends on it)."""
     h, o = workspace.h, workspace.o
     s = workspace.s if s is None else int(s)
+    cap = workspace.max_outliers or h
     n = ctypes.c_int32(0)
-    XO = torch.empty((s * h,), dtype=torch.float16)
-    WO = torch.empty((h * o,), dtype=torch.float16)
-    _check("llmint8_read_outlier_tiles", load_library().llmint8_read_outlier_tiles(
-        _ptr(workspace.buf), workspace.nbytes, s, h, o, ctypes.byref(n),
-        _ptr(XO), _ptr(WO), _stream(stream)))
+    XO = torch.empty((s * cap,), dtype=torch.float16)
+    WO = torch.empty((cap * o,), dtype=torch.float16)
+    _check("llmint8_read_outlier_tiles_ex", load_library().llmint8_read_outlier_tiles_ex(
+        _ptr(workspace.buf), workspace.nbytes, s, h, o, workspace.max_outliers,
+        ctypes.byref(n), _ptr(XO), _ptr(WO), _stream(stream)))
     k = n.value
+    if k > cap:  # the call kept no outlier tiles
+        return k, None, None
     return k, XO[: s * k].view(s, k), WO[: k * o].view(k, o)
 
 
@@ -319,6 +368,17 @@ def llmint8_wait_selftest(workspace: Workspace, limit_ns: int = 2_000_000,
     """Enqueue the bounded-wait self-test (its waits run out by design)."""
     _check("llmint8_wait_selftest", load_library().llmint8_wait_selftest(
         _ptr(workspace.buf), workspace.nbytes, int(limit_ns), _stream(stream)))
+
+
+def llmint8_noalloc_read_device_status(stream=None) -> int:
+    """Status bits of the allocation-free entry point on the current device
+    (read and cleared; its state block is cleared too)."""
+    bits = ctypes.c_int32(0)
+    rc = load_library().llmint8_noalloc_read_device_status(ctypes.byref(bits),
+                                                           _stream(stream))
+    if rc not in (OK, -6):
+        _check("llmint8_noalloc_read_device_status", rc)
+    return bits.value
 
 
 def llmint8_read_device_status(workspace: Workspace, stream=None) -> int:

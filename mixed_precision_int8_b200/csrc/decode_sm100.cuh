@@ -77,11 +77,15 @@ struct Params {
   uint16_t *WO;           // [n_out][o] fp16, written here
   const uint16_t *w16;    // optional fp16 W [h][o]: WO rows are its own rows
   const int32_t *n_out;
+  int32_t wo_cap;         // outlier rows the workspace holds; |O| above it:
+                          // no outlier product (the row pass flagged it)
   uint16_t *out;
   int32_t *ci;            // optional exact accumulators [s][o]
   int32_t *cacc;          // [s][o] int32 partial sums (zeroed before the launch)
   int32_t *tile_count;    // [num_m_blocks] arrivals (zeroed before the launch)
   int32_t *status;
+  int32_t *done_counter;  // CTAs finished (zero between calls), used only
+  int32_t *status_host;   // with a mapped host word (or null) for the status
   uint64_t timeout_ns;
 };
 
@@ -221,7 +225,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // compare. After each segment the rows are published (fence) by bumping
     // wo_segments.
     constexpr uint32_t idesc = idesc_i8_s32(BM, BN);
-    const int32_t n_out = *p.n_out;
+    const int32_t n_raw = *p.n_out;
+    const int32_t n_out = n_raw <= p.wo_cap ? n_raw : 0;
     const int32_t nwords = (p.h + 31) >> 5;
     const int32_t kb_words = (int32_t)((nk + 31) >> 5);
     for (int32_t w = lane; w < nwords; w += 32) {
@@ -355,7 +360,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ---------------------------------------------------------- epilogue
     const int ew = warp - EPI_WARP0;
     const int et = threadIdx.x - EPI_WARP0 * 32;  // 0..127: one tile column
-    const int32_t n_out = *p.n_out;
+    const int32_t n_raw = *p.n_out;
+    const int32_t n_out = n_raw <= p.wo_cap ? n_raw : 0;
     const int32_t nf = n_out < 16 ? n_out : 16;
     __shared__ int last_arrival;
     // the row scales (over 16129) and the first 16 outlier activations of
@@ -452,6 +458,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 2) tmem_dealloc(tmem_base, TMEM_COLS);
+  if (threadIdx.x == 0) mirror_status_to_host(p.status, p.done_counter, p.status_host);
 }
 
 }  // namespace decode

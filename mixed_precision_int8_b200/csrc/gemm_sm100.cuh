@@ -15,9 +15,13 @@
 //   warp 1      one thread issues tcgen05.mma.kind::i8 (M=128, N=256, K=32)
 //               into a TMEM accumulator; tcgen05.commit frees ring slots
 //   warp 2      allocates / frees the 512 TMEM columns (2 accumulators)
-//   warps 4-11  epilogue: before the first tile, a share of the fp16 outlier
-//               rows of W; per tile, while the MMA runs, the column scales
-//               and outlier rows (as fp32) go to shared memory and each
+//   warps 4-11  epilogue: before the first tile (launched cooperatively, so
+//               every CTA is resident), a share of the fp16 outlier rows
+//               of W, gathered while the first tiles' mainloops run, then
+//               announced on a counter; otherwise those rows come built by
+//               the activation fix-up. Per tile, while the MMA runs, the
+//               column scales and the tile's slice of the outlier rows go
+//               to shared memory as fp32, and each
 //               thread computes the outlier product of its row and its half
 //               of the tile's columns into registers (packed f32x2 FMAs).
 //               Once the accumulator is ready, each warp tcgen05.lds its half
@@ -25,6 +29,8 @@
 //               dequantises, adds the outlier product and writes fp16
 //               through a 64B-swizzled 32x32 staging block with TMA stores;
 //               the other accumulator is being filled by the MMA meanwhile.
+// The only wait on other CTAs is for their shares of the outlier rows of W,
+// and only in a cooperative launch, where all of them are resident.
 // Every wait is bounded by the global timer; on a timeout the CTA records a
 // status bit, drains its in-flight copies and MMAs, frees TMEM and returns.
 #pragma once
@@ -34,6 +40,7 @@
 #include <cuda_fp16.h>
 
 #include "ptx_sm100.cuh"
+#include "outlier_rows.cuh"
 
 namespace llmint8 {
 namespace gemm {
@@ -81,14 +88,21 @@ struct Params {
   const float *ax;        // [s]
   const float *aw;        // [o]
   const uint16_t *XO;     // [s][n_out] fp16
-  uint16_t *WO;           // [n_out][o] fp16, built here (Step 2, W side)
+  uint16_t *WO;           // [n_out][o] fp16: built here when build_wo, else
+                          // before this launch
   const int8_t *wq;       // [o][h] int8 codes of W
   const uint16_t *w16;    // optional fp16 W [h][o]: WO rows are its own rows
   const int32_t *idx;     // outlier columns, ascending
+  int32_t build_wo;       // 1 (cooperative launch only): the CTAs build WO
   int32_t *wo_counter;    // CTAs done with their share of WO; zero on entry
   const int32_t *n_out;   // device scalar |O|
+  int32_t wo_cap;         // outlier rows the workspace holds; |O| above it:
+                          // no outlier product (the fix-up flagged it)
   int32_t *ci;            // optional [s][o] int32
   int32_t *status;        // device status word
+  int32_t *done_counter;  // CTAs finished (zero between calls), used only
+  int32_t *status_host;   // with a mapped host word (or null) that receives
+                          // the status bits when the last CTA finishes
   uint64_t timeout_ns;
 };
 
@@ -237,49 +251,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // --------------------------------------------------------- epilogue
     const int ew = warp & 3;          // TMEM lane quarter of this warp
     const int hc = (warp - EPI_WARP0) >> 2;  // which half of the tile's columns
-    const int et = threadIdx.x - EPI_WARP0 * 32;  // 0..127
-    const int32_t n_out = *p.n_out;
+    const int et = threadIdx.x - EPI_WARP0 * 32;  // 0..255
+    const int32_t n_raw = *p.n_out;
+    const int32_t n_out = n_raw <= p.wo_cap ? n_raw : 0;
     const int32_t n_fast = n_out < FAST_OUTLIERS ? n_out : FAST_OUTLIERS;
-    bool wo_ready = n_out == 0;
-    if (n_out > 0) {
-      // Step 2, W side: WO[t][j] = fp16(fp32(fp32(wq[j][O_t]) * aw[j]) / 127)
-      // (or W[O_t][j] itself when the fp16 weight is given) for this CTA's
-      // share of the (t, j) pairs, while the first tile's mainloop runs; the
-      // one-byte gathers are spread over every CTA
-      const int64_t pairs = static_cast<int64_t>(n_out) * p.o;
-      const int64_t stride = static_cast<int64_t>(gridDim.x) * NUM_EPI_THREADS;
-      if (p.w16) {
-        for (int64_t q = static_cast<int64_t>(blockIdx.x) * NUM_EPI_THREADS + et; q < pairs;
-             q += stride) {
-          const int32_t t = static_cast<int32_t>(q / p.o);
-          const int32_t j = static_cast<int32_t>(q - static_cast<int64_t>(t) * p.o);
-          p.WO[q] = __ldg(p.w16 + static_cast<int64_t>(__ldg(p.idx + t)) * p.o + j);
-        }
-      }
-      for (int64_t q0 = static_cast<int64_t>(blockIdx.x) * NUM_EPI_THREADS + et;
-           !p.w16 && q0 < pairs; q0 += 4 * stride) {
-        int32_t b[4];
-        float aj[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int64_t q = q0 + u * stride;
-          b[u] = 0;
-          aj[u] = 0.0f;
-          if (q < pairs) {
-            const int32_t t = static_cast<int32_t>(q / p.o);
-            const int32_t j = static_cast<int32_t>(q - static_cast<int64_t>(t) * p.o);
-            b[u] = p.wq[static_cast<int64_t>(j) * p.h + __ldg(p.idx + t)];
-            aj[u] = __ldg(p.aw + j);
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int64_t q = q0 + u * stride;
-          if (q < pairs)
-            p.WO[q] = __half_as_ushort(
-                __float2half_rn(__fdiv_rn(static_cast<float>(b[u]) * aj[u], 127.0f)));
-        }
-      }
+    bool wo_ready = n_out == 0 || !p.build_wo;
+    if (!wo_ready) {
+      // Step 2, W side: this CTA's share of the (t, j) pairs of WO, while the
+      // first tile's mainloop runs; the one-byte gathers are spread over
+      // every CTA
+      build_wo_rows(n_out, p.idx, p.wq, p.aw, p.w16, p.h, p.o, p.WO,
+                    static_cast<int64_t>(blockIdx.x) * NUM_EPI_THREADS + et,
+                    static_cast<int64_t>(gridDim.x) * NUM_EPI_THREADS);
       __threadfence();
       named_barrier(EPI_BARRIER, NUM_EPI_THREADS);
       if (et == 0) atomicAdd(p.wo_counter, 1);
@@ -297,7 +280,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // (1) column scales and fp16 outlier rows of this tile into shared
       //     memory, while the MMA still works on the accumulator
       if (!wo_ready) {
-        // every CTA's share of WO is written (bounded wait)
+        // every CTA's share of WO is written (bounded wait; all CTAs are
+        // resident, so it ends unless a CTA has aborted)
         bool got = true;
         if (et == 0) {
           const uint64_t t0 = global_timer_ns();
@@ -318,9 +302,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         wo_ready = true;
       }
       named_barrier(EPI_BARRIER, NUM_EPI_THREADS);  // previous tile done reading
-      for (int i = et; i < BN; i += NUM_EPI_THREADS) {
-        const int32_t j = n0 + i;
-        sAW[i] = j < p.o ? __ldg(p.aw + j) : 0.0f;
+      static_assert(NUM_EPI_THREADS == BN, "one epilogue thread per tile column");
+      {
+        const int32_t j = n0 + et;
+        const bool jok = j < p.o;
+        const float awj = jok ? __ldg(p.aw + j) : 0.0f;
+        sAW[et] = awj;
       }
       for (int i = et; i < n_fast * (BN / 8); i += NUM_EPI_THREADS) {
         const int t = i / (BN / 8);
@@ -467,6 +454,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 2) tmem_dealloc(tmem_base, TMEM_COLS);
+  if (threadIdx.x == 0) mirror_status_to_host(p.status, p.done_counter, p.status_host);
 }
 
 }  // namespace gemm

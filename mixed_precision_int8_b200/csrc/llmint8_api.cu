@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -28,12 +29,20 @@ constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per individual wait
 constexpr uint32_t kActSmemOnePerSm = 220 * 1024;
 
 // ----------------------------------------------------------- device info
+// How the prefill GEMM is launched on a device. Cooperatively (all CTAs
+// resident at once, a launch the driver refuses otherwise), its CTAs build
+// the fp16 outlier rows of W themselves while their first mainloops run and
+// wait for each other's shares; otherwise the activation fix-up builds them
+// before the GEMM and no CTA waits for another. The first launch on a
+// device finds out which form the driver accepts (with programmatic
+// dependent launch, then without) and the answer is kept.
+enum GemmLaunch { kGemmUntested = -1, kGemmPlain = 0, kGemmCoop = 1, kGemmCoopPdl = 2 };
+
 struct DeviceInfo {
   bool init = false;
   bool supported = false;
   int sm_count = 0;
-  bool gemm_attr = false;
-  bool decode_attr = false;
+  std::atomic<int> gemm_launch{kGemmUntested};
 };
 constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
@@ -60,6 +69,16 @@ llmint8_status device_info(DeviceInfo **out) {
       if (cudaFuncSetAttribute(k_act_rows, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)kActSmemOnePerSm) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
+      // a cooperative GEMM needs one resident CTA per SM of its grid
+      int coop = 0, per_sm = 0;
+      if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess ||
+          cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemm::k_gemm_i8_fused,
+                                                        gemm::NUM_THREADS,
+                                                        gemm::SMEM_BYTES) != cudaSuccess) {
+        cudaGetLastError();
+        coop = 0;
+      }
+      d.gemm_launch.store((coop && per_sm >= 1) ? kGemmUntested : kGemmPlain);
     }
     d.init = true;
   }
@@ -136,7 +155,8 @@ int32_t mask_words(int64_t h) { return (int32_t)((h + 31) / 32); }
 constexpr size_t kStateBytes = 256 + ((4 * (size_t)((kMaxH + 31) / 32) + 255) & ~size_t(255));
 static_assert(kStateBytes == LLMINT8_WORKSPACE_STATE_BYTES, "state block size");
 
-Layout layout_for(int64_t s, int64_t h, int64_t o) {
+// `cap` = outlier columns the XO / WO tiles hold (h for any alpha).
+Layout layout_for(int64_t s, int64_t h, int64_t o, int64_t cap) {
   Layout L;
   size_t off = 0;
   L.status = off;  off = align256(off + 256);
@@ -146,10 +166,10 @@ Layout layout_for(int64_t s, int64_t h, int64_t o) {
   L.idx = off;     off = align256(off + 4 * (size_t)h);
   L.ax = off;      off = align256(off + 4 * (size_t)s);
   L.xq = off;      off = align256(off + (size_t)s * h);
-  L.xo = off;      off = align256(off + 2 * (size_t)s * h);
-  L.wo = off;      off = align256(off + 2 * (size_t)h * o);
   L.tiles = off;   off = align256(off + 4 * (size_t)((o + decode::BM - 1) / decode::BM));
   L.cacc = off;    off = align256(off + 4 * (size_t)kDecodeMaxRows * o);
+  L.xo = off;      off = align256(off + 2 * (size_t)s * cap);
+  L.wo = off;      off = align256(off + 2 * (size_t)cap * o);
   L.end = off;
   L.xstage = off;  off = align256(off + 2 * (size_t)s * h);
   L.ostage = off;  off = align256(off + 2 * (size_t)s * o);
@@ -159,12 +179,16 @@ Layout layout_for(int64_t s, int64_t h, int64_t o) {
 
 // status block: [0] device status bits, [1] |O|, [2] column-pass block
 // counter, [3] block counter of the one-read activation pass (zero between
-// calls), [4] CTAs of the GEMM done with their share of WO
+// calls), [4] CTAs of the call's last kernel that have finished (zero
+// between calls; counted only when the status bits go to a host word)
 int32_t *status_word(void *ws) { return reinterpret_cast<int32_t *>(ws); }
 int32_t *count_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 1; }
 int32_t *block_counter_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 2; }
 int32_t *act_counter_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 3; }
-int32_t *wo_counter_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 4; }
+int32_t *done_counter_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 4; }
+// [6] CTAs of a cooperative GEMM done with their share of the outlier rows
+// of W (zeroed by the call's activation kernels)
+int32_t *wo_counter_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 6; }
 float *tensor_scale_word(void *ws) { return reinterpret_cast<float *>(ws) + 5; }
 constexpr int kSelftestWord = 8;  // a status-block word no kernel sets
 
@@ -210,21 +234,38 @@ llmint8_status last_launch() {
 
 // Launch with programmatic stream serialization when `pdl`: the kernel may
 // be scheduled while its predecessor drains; it orders itself after the
-// predecessor with griddepcontrol.wait before touching memory.
+// predecessor with griddepcontrol.wait before touching memory. With `coop`
+// the launch is cooperative: every CTA of the grid is resident at once, or
+// the launch fails (and enqueues nothing).
 template <typename... KArgs, typename... Args>
-cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                   cudaStream_t st, bool pdl, Args &&...args) {
+cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t st, bool pdl, bool coop, Args &&...args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (coop) {
+    attr[n].id = cudaLaunchAttributeCooperative;
+    attr[n].val.cooperative = 1;
+    ++n;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = n;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                   cudaStream_t st, bool pdl, Args &&...args) {
+  return launch_ex(kernel, grid, block, smem, st, pdl, false, std::forward<Args>(args)...);
 }
 
 // Steps 1, 2 and 4 (activation side, plus the fp16 outlier rows of W when
@@ -239,18 +280,20 @@ struct ActivationArgs {
   uint32_t *acc_mask;     // one-read pass: accumulation bitmask (zero on entry
   int32_t *act_counter;   // and exit, with its block counter)
   bool act_reset;         // zero them first (their state is not known)
-  int32_t *gemm_counter;  // zeroed for the GEMM that follows (or null)
   uint8_t *flags;
   int8_t *Xq;
   float *ax;
   uint16_t *XO;
   const int8_t *wq;
   const float *aw;
+  const uint16_t *w16;
   int64_t o;
-  uint16_t *WO;
+  uint16_t *WO;  // fp16 outlier rows of W, built here for |O| > 16 (or null)
+  int32_t cap;   // outlier columns XO and WO hold
   int32_t *zero_buf;
   int64_t zero_n;
   int *status;  // device status bits
+  int32_t *gemm_counter;  // zeroed for a GEMM that builds WO itself (or null)
 };
 
 // Launch plan of k_act_rows (one CTA per SM): `groups` row groups of `wpr`
@@ -337,10 +380,32 @@ llmint8_status enqueue_activation_fused(const DeviceInfo &dev, const ActivationA
   *launches += 1;
   const int64_t fix_blocks = (a.s + kFixRowsPerBlock - 1) / kFixRowsPerBlock;
   if (fix_blocks > 0) {
-    e = launch(k_act_fixup, dim3((unsigned)fix_blocks), dim3(kFixThreads), 0, st, true, a.X,
-               a.s, (int32_t)a.h, p.thresh_bits, (const uint32_t *)a.mask,
-               (const int32_t *)a.wprefix, (const int32_t *)a.idx, (const int32_t *)a.count,
-               a.Xq, a.ax, a.XO, a.gemm_counter);
+    FixupParams f;
+    f.X = a.X;
+    f.s = a.s;
+    f.h = (int32_t)a.h;
+    f.thresh_bits = p.thresh_bits;
+    f.mask = a.mask;
+    f.word_prefix = a.wprefix;
+    f.idx = a.idx;
+    f.count = a.count;
+    f.Xq = a.Xq;
+    f.ax = a.ax;
+    f.XO = a.XO;
+    f.cap = a.cap;
+    f.row_blocks = fix_blocks;
+    f.wq = a.wq;
+    f.aw = a.aw;
+    f.w16 = a.w16;
+    f.o = (int32_t)a.o;
+    f.WO = a.WO;
+    f.status = a.status;
+    f.gemm_counter = a.gemm_counter;
+    // one extra block per SM builds the fp16 outlier rows of W while the
+    // row blocks run (|O| is known on the device only; with none they
+    // return at once)
+    const int64_t grid = fix_blocks + (a.WO ? (int64_t)dev.sm_count : 0);
+    e = launch(k_act_fixup, dim3((unsigned)grid), dim3(kFixThreads), 0, st, true, f);
     if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
     *launches += 1;
   }
@@ -375,8 +440,7 @@ llmint8_status enqueue_activation_pass(const DeviceInfo &dev, const ActivationAr
   int64_t reset_blocks = (reset_threads + 255) / 256;
   if (reset_blocks < 1) reset_blocks = 1;
   if (reset_blocks > 4 * (int64_t)dev.sm_count) reset_blocks = 4 * (int64_t)dev.sm_count;
-  // prefill: the one extra word zeroed is the GEMM's WO counter (the GEMM
-  // builds the fp16 outlier rows of W itself)
+  // the one extra word a prefill call may zero is the GEMM's WO counter
   int32_t *zb = a.zero_buf;
   int64_t zn = a.zero_n;
   if (!zb && a.gemm_counter) {
@@ -403,7 +467,15 @@ llmint8_status enqueue_activation_pass(const DeviceInfo &dev, const ActivationAr
   if (rb > 0) {
     e = launch(k_rows_any, dim3((unsigned)rb), dim3(kRowThreads), 0, st, true, a.X, a.s, hh,
                (const uint32_t *)a.mask, (const int32_t *)a.wprefix, (const int32_t *)a.count,
-               a.Xq, a.ax, a.XO);
+               a.Xq, a.ax, a.XO, a.cap, a.status);
+    if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+    *launches += 1;
+  }
+  if (a.WO) {
+    // fp16 outlier rows of W (returns at once without outlier columns)
+    e = launch(k_build_wo, dim3((unsigned)(2 * dev.sm_count)), dim3(256), 0, st, true,
+               (const int32_t *)a.count, (const int32_t *)a.idx, a.wq, a.aw, a.w16, hh,
+               (int32_t)a.o, a.WO, a.cap);
     if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
     *launches += 1;
   }
@@ -420,25 +492,64 @@ llmint8_status validate_weight(const llmint8_weight *w) {
   return LLMINT8_OK;
 }
 
+// opts->max_outliers as a capacity (h when 0); -1 when invalid.
+int64_t outlier_cap(const llmint8_matmul_opts *opts, int64_t h) {
+  const int64_t m = opts ? opts->max_outliers : 0;
+  if (m < 0 || m > h) return -1;
+  return m == 0 ? h : m;
+}
+
+// The options every matmul form checks before it enqueues anything.
+llmint8_status check_opts(const llmint8_matmul_opts *opts, int64_t s, int64_t h) {
+  if (!opts) return LLMINT8_OK;
+  if (opts->path < 0 || opts->path > 2 || (opts->path == 2 && s > kDecodeMaxRows))
+    return LLMINT8_ERR_ARG;
+  if (opts->x_scale != LLMINT8_SCALE_VECTORWISE && opts->x_scale != LLMINT8_SCALE_TENSORWISE)
+    return LLMINT8_ERR_ARG;
+  if (outlier_cap(opts, h) < 0) return LLMINT8_ERR_ARG;
+  if (opts->status_host) {
+    // pinned host memory the device reaches at the same address
+    cudaPointerAttributes pa;
+    if (cudaPointerGetAttributes(&pa, opts->status_host) != cudaSuccess) {
+      cudaGetLastError();
+      return LLMINT8_ERR_ARG;
+    }
+    if (pa.type != cudaMemoryTypeHost || pa.devicePointer != (void *)opts->status_host ||
+        !aligned(opts->status_host, 4))
+      return LLMINT8_ERR_ARG;
+  }
+  return LLMINT8_OK;
+}
+
+// A previous call left anomaly bits in the caller's host status word.
+bool host_status_set(const llmint8_matmul_opts *opts) {
+  return opts && opts->status_host &&
+         *reinterpret_cast<volatile int32_t *>(opts->status_host) != 0;
+}
+
 llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w, float alpha,
                            uint16_t *out, void *ws, size_t ws_bytes, llmint8_matmul_opts *opts,
-                           cudaStream_t st, bool host_layout) {
-  if (opts) opts->launches = 0;
+                           cudaStream_t st, bool host_layout, bool reset_state = false) {
+  if (opts) {
+    opts->launches = 0;
+    opts->gemm_launch = -1;
+  }
   llmint8_status rc = validate_weight(w);
   if (rc) return rc;
   if (s < 0 || s > (int64_t)INT32_MAX) return LLMINT8_ERR_SHAPE;
   if ((rc = check_alpha(alpha))) return rc;
+  if ((rc = check_opts(opts, s, w->h))) return rc;
   const int path = opts ? opts->path : 0;
-  if (path < 0 || path > 2 || (path == 2 && s > kDecodeMaxRows)) return LLMINT8_ERR_ARG;
   const int x_scale = opts ? opts->x_scale : LLMINT8_SCALE_VECTORWISE;
-  if (x_scale != LLMINT8_SCALE_VECTORWISE && x_scale != LLMINT8_SCALE_TENSORWISE)
-    return LLMINT8_ERR_ARG;
+  if (host_status_set(opts)) return LLMINT8_ERR_DEVICE_STATUS;
   if (s == 0) return LLMINT8_OK;
   if (!X || !out || !ws) return LLMINT8_ERR_NULL;
   if (!aligned(X, 16) || !aligned(out, 16) || !aligned(ws, 256)) return LLMINT8_ERR_ALIGN;
   if (opts && opts->ci_dev && !aligned(opts->ci_dev, 16)) return LLMINT8_ERR_ALIGN;
   const int64_t h = w->h, o = w->o;
-  const Layout L = layout_for(s, h, o);
+  const int64_t cap = outlier_cap(opts, h);
+  int32_t *status_host = opts ? opts->status_host : nullptr;
+  const Layout L = layout_for(s, h, o, cap);
   if (ws_bytes < (host_layout ? L.end_host : L.end)) return LLMINT8_ERR_WORKSPACE;
   DeviceInfo *dev = nullptr;
   if ((rc = device_info(&dev))) return rc;
@@ -484,8 +595,7 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
   act.block_counter = block_counter_word(ws);
   act.acc_mask = reinterpret_cast<uint32_t *>(wsb + L.acc);
   act.act_counter = act_counter_word(ws);
-  act.act_reset = false;  // the workspace keeps them zero between calls
-  act.gemm_counter = use_decode ? nullptr : wo_counter_word(ws);
+  act.act_reset = reset_state;  // otherwise the workspace keeps them zero
   act.flags = nullptr;
   act.status = status;
   act.Xq = xq;
@@ -493,11 +603,18 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
   act.XO = xo;
   act.wq = w->wq_dev;
   act.aw = w->aw_dev;
+  act.w16 = w->w16_dev;
   act.o = o;
+  act.cap = (int32_t)cap;
+  // prefill: the fp16 outlier rows of W come from the GEMM itself when it
+  // can be launched cooperatively, else from the activation kernels;
   // decode: the W^O gather and the finishing step run inside the decode
   // kernel; its tile counters and the s rows of int32 partial sums (one
   // contiguous region) start from zero
-  act.WO = use_decode ? nullptr : wo;
+  const bool gemm_builds_wo = !use_decode && dev->gemm_launch.load() != kGemmPlain &&
+                              !(opts && opts->gemm_plain);
+  act.WO = (use_decode || gemm_builds_wo) ? nullptr : wo;
+  act.gemm_counter = gemm_builds_wo ? wo_counter_word(ws) : nullptr;
   int32_t *tiles = reinterpret_cast<int32_t *>(wsb + L.tiles);
   act.zero_buf = use_decode ? tiles : nullptr;
   act.zero_n = use_decode ? (int64_t)((L.cacc - L.tiles) / 4) + s * o : 0;
@@ -520,7 +637,7 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
     e0 = launch(k_decode_rowpass, dim3((unsigned)col_blocks, (unsigned)s), dim3(kDecodeThreads), 0,
                 st, true,
                 X, (int32_t)s, (int32_t)h, (const uint32_t *)mask, (const uint32_t *)partial,
-                col_blocks, wprefix, count, ax, xq, xo);
+                col_blocks, wprefix, count, ax, xq, xo, (int32_t)cap, status);
     if (e0 != cudaSuccess) return LLMINT8_ERR_CUDA;
     launches += 2;
   } else if ((rc = enqueue_activation_pass(*dev, act, st, &launches))) {
@@ -548,11 +665,14 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
     p.WO = wo;
     p.w16 = w->w16_dev;
     p.n_out = count;
+    p.wo_cap = (int32_t)cap;
     p.out = out;
     p.ci = opts ? opts->ci_dev : nullptr;
     p.cacc = cacc;
     p.tile_count = tiles;
     p.status = status;
+    p.done_counter = done_counter_word(ws);
+    p.status_host = status_host;
     p.timeout_ns = kTimeoutNs;
     const int64_t total_units = (int64_t)p.num_m_blocks * p.num_k_blocks;
     int grid = dev->sm_count;
@@ -581,14 +701,52 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
     p.idx = idx;
     p.wo_counter = wo_counter_word(ws);
     p.n_out = count;
+    p.wo_cap = (int32_t)cap;
     p.ci = opts ? opts->ci_dev : nullptr;
     p.status = status;
+    p.done_counter = done_counter_word(ws);
+    p.status_host = status_host;
     p.timeout_ns = kTimeoutNs;
     const int64_t tiles = (int64_t)p.num_m_blocks * p.num_n_blocks;
     const int grid = (int)(tiles < dev->sm_count ? tiles : dev->sm_count);
-    e = launch(gemm::k_gemm_i8_fused, dim3(grid), dim3(gemm::NUM_THREADS), gemm::SMEM_BYTES, st,
-               !timed, tmA, tmB, tmOut, p);
+    e = cudaErrorNotSupported;
+    int used = kGemmPlain;
+    if (gemm_builds_wo) {
+      // cooperative, with programmatic dependent launch where accepted
+      p.build_wo = 1;
+      const int mode = dev->gemm_launch.load();
+      if (mode == kGemmUntested || mode == kGemmCoopPdl) {
+        e = launch_ex(gemm::k_gemm_i8_fused, dim3(grid), dim3(gemm::NUM_THREADS),
+                      gemm::SMEM_BYTES, st, !timed, true, tmA, tmB, tmOut, p);
+        if (e == cudaSuccess) used = timed ? kGemmCoop : kGemmCoopPdl;
+        if (e == cudaSuccess && !timed) dev->gemm_launch.store(kGemmCoopPdl);
+      }
+      if (e != cudaSuccess && (mode == kGemmUntested || mode == kGemmCoop || timed)) {
+        cudaGetLastError();
+        e = launch_ex(gemm::k_gemm_i8_fused, dim3(grid), dim3(gemm::NUM_THREADS),
+                      gemm::SMEM_BYTES, st, false, true, tmA, tmB, tmOut, p);
+        if (e == cudaSuccess) used = kGemmCoop;
+        if (e == cudaSuccess && mode == kGemmUntested) dev->gemm_launch.store(kGemmCoop);
+      }
+      if (e != cudaSuccess) {
+        // refused: from now on the activation kernels build the rows; this
+        // call builds them in a launch of its own
+        cudaGetLastError();
+        dev->gemm_launch.store(kGemmPlain);
+        e = launch(k_build_wo, dim3((unsigned)(2 * dev->sm_count)), dim3(256), 0, st, true,
+                   (const int32_t *)count, (const int32_t *)idx, w->wq_dev, w->aw_dev,
+                   w->w16_dev, (int32_t)h, (int32_t)o, wo, (int32_t)cap);
+        if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+        ++launches;
+      }
+    }
+    if (e != cudaSuccess) {
+      p.build_wo = 0;
+      e = launch(gemm::k_gemm_i8_fused, dim3(grid), dim3(gemm::NUM_THREADS), gemm::SMEM_BYTES,
+                 st, !timed, tmA, tmB, tmOut, p);
+    }
     if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
+    if (opts) opts->gemm_launch = used;
     if (opts && opts->gemm_event_stop)
       cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->gemm_event_stop), st);
     ++launches;
@@ -620,7 +778,12 @@ const char *llmint8_status_string(llmint8_status st) {
 
 size_t llmint8_workspace_size(int64_t s, int64_t h, int64_t o) {
   if (s < 0 || h < 0 || o < 0) return 0;
-  return layout_for(s, h, o).end;
+  return layout_for(s, h, o, h).end;
+}
+
+size_t llmint8_workspace_size_ex(int64_t s, int64_t h, int64_t o, int64_t max_outliers) {
+  if (s < 0 || h < 0 || o < 0 || max_outliers < 0 || max_outliers > h) return 0;
+  return layout_for(s, h, o, max_outliers == 0 ? h : max_outliers).end;
 }
 
 llmint8_status llmint8_workspace_init(void *ws_dev, size_t ws_bytes, void *stream) {
@@ -634,7 +797,12 @@ llmint8_status llmint8_workspace_init(void *ws_dev, size_t ws_bytes, void *strea
 
 size_t llmint8_workspace_size_host(int64_t s, int64_t h, int64_t o) {
   if (s < 0 || h < 0 || o < 0) return 0;
-  return layout_for(s, h, o).end_host;
+  return layout_for(s, h, o, h).end_host;
+}
+
+size_t llmint8_workspace_size_host_ex(int64_t s, int64_t h, int64_t o, int64_t max_outliers) {
+  if (s < 0 || h < 0 || o < 0 || max_outliers < 0 || max_outliers > h) return 0;
+  return layout_for(s, h, o, max_outliers == 0 ? h : max_outliers).end_host;
 }
 
 int64_t llmint8_decode_max_rows(void) { return kDecodeMaxRows; }
@@ -765,17 +933,15 @@ llmint8_status llmint8_matmul_host_ex(const uint16_t *X_host, int64_t s, const l
   if (opts) opts->launches = 0;
   llmint8_status rc = validate_weight(w);
   if (rc) return rc;
-  // the options are checked here too, so that a bad one enqueues no copy
-  if (opts && (opts->path < 0 || opts->path > 2 || (opts->path == 2 && s > kDecodeMaxRows) ||
-               (opts->x_scale != LLMINT8_SCALE_VECTORWISE &&
-                opts->x_scale != LLMINT8_SCALE_TENSORWISE)))
-    return LLMINT8_ERR_ARG;
   if (s < 0 || s > (int64_t)INT32_MAX) return LLMINT8_ERR_SHAPE;
+  // the options are checked here too, so that a bad one enqueues no copy
+  if ((rc = check_opts(opts, s, w->h))) return rc;
   if ((rc = check_alpha(alpha))) return rc;
+  if (host_status_set(opts)) return LLMINT8_ERR_DEVICE_STATUS;
   if (s == 0) return LLMINT8_OK;
   if (!X_host || !out_host || !ws_dev) return LLMINT8_ERR_NULL;
   if (!aligned(ws_dev, 256)) return LLMINT8_ERR_ALIGN;
-  const Layout L = layout_for(s, w->h, w->o);
+  const Layout L = layout_for(s, w->h, w->o, outlier_cap(opts, w->h));
   if (ws_bytes < L.end_host) return LLMINT8_ERR_WORKSPACE;
   cudaStream_t st = as_stream(stream);
   uint8_t *wsb = static_cast<uint8_t *>(ws_dev);
@@ -793,9 +959,19 @@ llmint8_status llmint8_matmul_host_ex(const uint16_t *X_host, int64_t s, const l
 llmint8_status llmint8_read_outlier_tiles(const void *ws_dev, size_t ws_bytes, int64_t s,
                                           int64_t h, int64_t o, int32_t *n_out_host,
                                           uint16_t *XO_host, uint16_t *WO_host, void *stream) {
+  return llmint8_read_outlier_tiles_ex(ws_dev, ws_bytes, s, h, o, 0, n_out_host, XO_host,
+                                       WO_host, stream);
+}
+
+llmint8_status llmint8_read_outlier_tiles_ex(const void *ws_dev, size_t ws_bytes, int64_t s,
+                                             int64_t h, int64_t o, int64_t max_outliers,
+                                             int32_t *n_out_host, uint16_t *XO_host,
+                                             uint16_t *WO_host, void *stream) {
   if (!ws_dev || !n_out_host) return LLMINT8_ERR_NULL;
   if (s < 0 || h < 0 || o < 0) return LLMINT8_ERR_SHAPE;
-  const Layout L = layout_for(s, h, o);
+  if (max_outliers < 0 || max_outliers > h) return LLMINT8_ERR_ARG;
+  const int64_t cap = max_outliers == 0 ? h : max_outliers;
+  const Layout L = layout_for(s, h, o, cap);
   if (ws_bytes < L.end) return LLMINT8_ERR_WORKSPACE;
   cudaStream_t st = as_stream(stream);
   const uint8_t *wsb = static_cast<const uint8_t *>(ws_dev);
@@ -805,6 +981,7 @@ llmint8_status llmint8_read_outlier_tiles(const void *ws_dev, size_t ws_bytes, i
     return LLMINT8_ERR_CUDA;
   if (n < 0 || n > h) return LLMINT8_ERR_DEVICE_STATUS;
   *n_out_host = n;
+  if (n > cap) return LLMINT8_OK;  // the call kept no outlier tiles
   if (XO_host && n > 0 &&
       cudaMemcpyAsync(XO_host, wsb + L.xo, 2 * (size_t)s * n, cudaMemcpyDeviceToHost, st) !=
           cudaSuccess)
@@ -857,31 +1034,31 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[LLMINT8_NOALLOC_MAX_S
 namespace {
 
 struct NoAllocSlot {
-  bool ready = false;
-  void *ptr = nullptr;  // device address of g_noalloc_scratch on that device
+  void *ptr = nullptr;  // device address of g_noalloc_scratch last seen on that device
 };
 NoAllocSlot g_noalloc[kMaxDevices];
 std::mutex g_noalloc_mutex;
 
 // Device address of the scratch array on the current device. In host code
 // the array's name is only a host-side stand-in, so the address is asked of
-// the runtime once per device (with that device current) and cached. The
-// first lookup also clears the state block, asynchronously on `st`.
+// the runtime (with that device current) on every call; the lookup
+// allocates nothing. When it differs from the one seen before (the first
+// call on the device, or a new context after a device reset), the array's
+// state block is cleared, asynchronously on `st`.
 llmint8_status noalloc_scratch(cudaStream_t st, void **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
     return LLMINT8_ERR_CUDA;
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+    return LLMINT8_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
   NoAllocSlot &slot = g_noalloc[dev];
-  if (!slot.ready) {
-    void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
-      return LLMINT8_ERR_CUDA;
+  if (slot.ptr != p) {
     if (cudaMemsetAsync(p, 0, kStateBytes, st) != cudaSuccess) return LLMINT8_ERR_CUDA;
     slot.ptr = p;
-    slot.ready = true;
   }
-  *out = slot.ptr;
+  *out = p;
   return LLMINT8_OK;
 }
 
@@ -893,7 +1070,7 @@ extern "C" llmint8_status llmint8_matmul_noalloc(const uint16_t *X_dev, int64_t 
   llmint8_status rc = validate_weight(w);
   if (rc) return rc;
   if (s < 0 || s > (int64_t)INT32_MAX) return LLMINT8_ERR_SHAPE;
-  if (layout_for(s, w->h, w->o).end > (size_t)LLMINT8_NOALLOC_MAX_SCRATCH_BYTES)
+  if (layout_for(s, w->h, w->o, w->h).end > (size_t)LLMINT8_NOALLOC_MAX_SCRATCH_BYTES)
     return LLMINT8_ERR_TOO_LARGE;
   if (s == 0) return llmint8_matmul(X_dev, s, w, alpha, out_dev, nullptr, 0, stream);
   DeviceInfo *dev = nullptr;
@@ -901,6 +1078,31 @@ extern "C" llmint8_status llmint8_matmul_noalloc(const uint16_t *X_dev, int64_t 
   cudaStream_t st = as_stream(stream);
   void *ws = nullptr;
   if ((rc = noalloc_scratch(st, &ws))) return rc;
+  // every call clears the activation pass's accumulation state first, so a
+  // call that gave up a wait (reported by llmint8_noalloc_read_device_status)
+  // leaves nothing behind for the next one
   return matmul_impl(X_dev, s, w, alpha, out_dev, ws, (size_t)LLMINT8_NOALLOC_MAX_SCRATCH_BYTES,
-                     nullptr, st, false);
+                     nullptr, st, false, /*reset_state=*/true);
+}
+
+extern "C" llmint8_status llmint8_noalloc_read_device_status(int32_t *bits_out, void *stream) {
+  if (bits_out) *bits_out = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return LLMINT8_ERR_CUDA;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc[dev].ptr == nullptr) return LLMINT8_OK;  // no call yet on this device
+  }
+  cudaStream_t st = as_stream(stream);
+  void *ws = nullptr;
+  llmint8_status rc = noalloc_scratch(st, &ws);
+  if (rc) return rc;
+  int32_t bits = 0;
+  if (cudaMemcpyAsync(&bits, ws, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemsetAsync(ws, 0, kStateBytes, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return LLMINT8_ERR_CUDA;
+  if (bits_out) *bits_out = bits;
+  return bits ? LLMINT8_ERR_DEVICE_STATUS : LLMINT8_OK;
 }

@@ -248,6 +248,25 @@ __device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
   return d;
 }
 
+// The last CTA of a launch copies the status word into the caller's mapped
+// host word (when given), so the next call sees this call's anomalies
+// without a synchronisation. One writer per launch; the counter is left
+// zero for the next call.
+__device__ __forceinline__ void mirror_status_to_host(int32_t *status, int32_t *done_counter,
+                                                      int32_t *status_host) {
+  if (status_host == nullptr) return;
+  __threadfence();
+  if (atomicAdd(done_counter, 1) != (int32_t)gridDim.x - 1) return;
+  __threadfence();
+  const int32_t bits = atomicOr(status, 0);
+  if (bits != 0) {
+    volatile int32_t *hw = status_host;
+    *hw = *hw | bits;
+  }
+  *done_counter = 0;
+  __threadfence();
+}
+
 // --------------------------------------------------------------- tcgen05
 
 // Whole warp: allocate `ncols` TMEM columns; the base address is written to

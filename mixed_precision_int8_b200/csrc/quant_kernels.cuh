@@ -2,8 +2,8 @@
 //   K0  offline weight preparation (column absmax + int8 codes, transposed)
 //   K1  activation pass: outlier-column bitmask, compaction of the outlier
 //       list, per-row absmax over regular columns and int8 row codes
-//   K2  fp16 outlier rows of W recovered from the int8 weight (same launch
-//       as the row quantisation)
+//   K2  fp16 outlier rows of W recovered from the int8 weight, before the
+//       GEMM (blocks of their own in the outlier fix-up's launch)
 //
 // Magnitude trick used throughout: for a non-NaN binary16 value, the bit
 // pattern with the sign cleared orders exactly like |x|, so maxima and the
@@ -16,6 +16,7 @@
 
 #include "llmint8.h"
 #include "ptx_sm100.cuh"
+#include "outlier_rows.cuh"
 
 namespace llmint8 {
 
@@ -543,36 +544,95 @@ __global__ void __launch_bounds__(kActMaxWarps * 32) k_act_rows(const ActRowsPar
   }
 }
 
+// The W side of Step 2 on its own (rows longer than a shared-memory stage,
+// where the fix-up kernel does not run), when |O| fits the workspace.
+__global__ void __launch_bounds__(256)
+    k_build_wo(const int32_t *__restrict__ count, const int32_t *__restrict__ idx,
+               const int8_t *__restrict__ wq, const float *__restrict__ aw,
+               const uint16_t *__restrict__ w16, int32_t h, int32_t o,
+               uint16_t *__restrict__ WO, int32_t cap) {
+  grid_dependency_wait();
+  grid_dependency_trigger();
+  const int32_t n = __ldcg(count);
+  if (n == 0 || n > cap) return;
+  build_wo_rows(n, idx, wq, aw, w16, h, o, WO,
+                static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x,
+                static_cast<int64_t>(gridDim.x) * blockDim.x);
+}
+
 // Completes k_act_rows once O is known. One warp per row:
 //   XO[i][t] = X[i][O_t]; Xq[i][O_t] = 0;
 //   m_i = max of |X[i][O_t]| below alpha; if m_i == a'_i > 0 the row's
 //   absmax over regular columns is recomputed and the row requantised by
 //   the whole block (every thread loads its chunks of the row at once).
-// Block 0 also zeroes *gemm_counter (used by the GEMM that follows).
+// Blocks beyond the row blocks (when WO is given) build the fp16 outlier
+// rows of W for the GEMM, side by side with the rows (when |O| fits the
+// workspace's `cap`). Block 0 also zeroes *gemm_counter for a GEMM that
+// builds those rows itself.
+// |O| above the cap: no outlier tile is written, block 0 sets
+// LLMINT8_DEV_OUTLIER_CAP and the layer goes without its outlier product.
 constexpr int kFixThreads = 256;
 constexpr int kFixRowsPerBlock = kFixThreads / 32;
 
-__global__ void __launch_bounds__(kFixThreads)
-    k_act_fixup(const uint16_t *__restrict__ X, int64_t s, int32_t h, uint32_t thresh_bits,
-                const uint32_t *__restrict__ mask, const int32_t *__restrict__ word_prefix,
-                const int32_t *__restrict__ idx, const int32_t *__restrict__ count,
-                int8_t *__restrict__ Xq, float *__restrict__ ax, uint16_t *__restrict__ XO,
-                int32_t *__restrict__ gemm_counter) {
+struct FixupParams {
+  const uint16_t *X;
+  int64_t s;
+  int32_t h;
+  uint32_t thresh_bits;
+  const uint32_t *mask;
+  const int32_t *word_prefix;
+  const int32_t *idx;
+  const int32_t *count;
+  int8_t *Xq;
+  float *ax;
+  uint16_t *XO;  // [s][|O|] or null
+  int32_t cap;   // outlier columns XO and WO hold
+  int64_t row_blocks;
+  // fp16 outlier rows of W (WO null: not built here)
+  const int8_t *wq;
+  const float *aw;
+  const uint16_t *w16;
+  int32_t o;
+  uint16_t *WO;
+  int *status;
+  int32_t *gemm_counter;  // zeroed for the GEMM that follows (or null)
+};
+
+__global__ void __launch_bounds__(kFixThreads) k_act_fixup(const FixupParams p) {
   __shared__ int redo[kFixRowsPerBlock];
   __shared__ uint32_t red[kFixThreads / 32];
   grid_dependency_wait();
   grid_dependency_trigger();
+  const uint16_t *__restrict__ X = p.X;
+  const int64_t s = p.s;
+  const int32_t h = p.h;
+  const int32_t *__restrict__ idx = p.idx;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (blockIdx.x == 0 && tid == 0 && gemm_counter) *gemm_counter = 0;
+  if (blockIdx.x == 0 && tid == 0 && p.gemm_counter) *p.gemm_counter = 0;
   // the first outlier columns, |O| and the row's scale are fetched together
   // (only |O| decides which of them are used), so a row costs two memory
   // round trips: these loads, then the gathers they address
   const int32_t j_pre = lane < h ? __ldcg(idx + lane) : 0;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * kFixRowsPerBlock + warp;
-  const bool row_ok = row < s;
-  const float a0 = row_ok ? __ldcg(ax + row) : 0.0f;
-  const int32_t n = __ldcg(count);
+  const bool row_ok = blockIdx.x < p.row_blocks && row < s;
+  const float a0 = row_ok ? __ldcg(p.ax + row) : 0.0f;
+  const int32_t n = __ldcg(p.count);
   if (n == 0) return;  // uniform over the grid
+  const bool fits = n <= p.cap;
+  if (!fits && blockIdx.x == 0 && tid == 0) atomicOr(p.status, LLMINT8_DEV_OUTLIER_CAP);
+  if (blockIdx.x >= p.row_blocks) {  // uniform over the block
+    if (fits && p.WO != nullptr)
+      build_wo_rows(n, idx, p.wq, p.aw, p.w16, h, p.o, p.WO,
+                    static_cast<int64_t>(blockIdx.x - p.row_blocks) * kFixThreads + tid,
+                    static_cast<int64_t>(gridDim.x - p.row_blocks) * kFixThreads);
+    return;
+  }
+  uint16_t *__restrict__ XO = fits ? p.XO : nullptr;
+  int8_t *__restrict__ Xq = p.Xq;
+  float *__restrict__ ax = p.ax;
+  const uint32_t thresh_bits = p.thresh_bits;
+  const uint32_t *__restrict__ mask = p.mask;
+  const int32_t *__restrict__ word_prefix = p.word_prefix;
   bool need = false;
   if (row_ok) {
     const uint16_t *xr = X + row * h;
@@ -656,11 +716,17 @@ __global__ void __launch_bounds__(kRowThreads)
     k_rows_any(const uint16_t *__restrict__ X, int64_t s, int32_t h,
                const uint32_t *__restrict__ mask, const int32_t *__restrict__ word_prefix,
                const int32_t *__restrict__ count, int8_t *__restrict__ Xq,
-               float *__restrict__ ax, uint16_t *__restrict__ XO) {
+               float *__restrict__ ax, uint16_t *__restrict__ XO, int32_t cap,
+               int *__restrict__ status) {
   grid_dependency_wait();
   grid_dependency_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerBlock + (threadIdx.x >> 5);
+  if (XO != nullptr && *count > cap) {
+    // more outlier columns than the workspace holds: no outlier tiles
+    if (row == 0 && lane == 0) atomicOr(status, LLMINT8_DEV_OUTLIER_CAP);
+    XO = nullptr;
+  }
   if (row >= s) return;
   const uint16_t *xr = X + row * h;
   uint32_t m2 = 0;
@@ -766,7 +832,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
                      const uint32_t *__restrict__ mask, const uint32_t *__restrict__ partial_max,
                      int32_t col_blocks, int32_t *__restrict__ word_prefix,
                      int32_t *__restrict__ count, float *__restrict__ ax,
-                     int8_t *__restrict__ Xq, uint16_t *__restrict__ XO) {
+                     int8_t *__restrict__ Xq, uint16_t *__restrict__ XO, int32_t cap,
+                     int *__restrict__ status) {
   __shared__ int32_t s_prefix[kDecodeColsPerBlock / 32];
   __shared__ int32_t red_before[kDecodeThreads / 32], red_total[kDecodeThreads / 32];
   __shared__ uint32_t red_max[kDecodeThreads / 32];
@@ -847,7 +914,10 @@ __global__ void __launch_bounds__(kDecodeThreads)
       if (pw == nwords - 1) word_prefix[nwords] = pre + pc;
     }
   }
-  if (row == 0 && blockIdx.x == 0 && tid == 0) *count = total;
+  if (row == 0 && blockIdx.x == 0 && tid == 0) {
+    *count = total;
+    if (total > cap) atomicOr(status, LLMINT8_DEV_OUTLIER_CAP);
+  }
   __syncthreads();
   if (c >= h) return;
   // codes of this chunk (outlier columns zeroed) and its fp16 outlier entries
@@ -861,6 +931,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
                              ((mk & 0x40u) ? 0u : 0x00FF0000u) | ((mk & 0x80u) ? 0u : 0xFF000000u);
     q.x &= keep_lo;
     q.y &= keep_hi;
+  }
+  if (mk && total <= cap) {  // fp16 outlier entries, when the workspace holds them
     const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
     const int32_t *pre_local = s_prefix - w_begin;  // indexed by global word
 #pragma unroll

@@ -211,3 +211,54 @@ def test_valid_call_without_a_gpu_reports_cuda_error_not_a_fallback(lib):
     rc = lib.llmint8_matmul(FAKE, 4, ctypes.byref(w), 6.0, FAKE, FAKE, need,
                             None)
     assert rc in (-5, -8)
+
+
+def test_workspace_with_an_outlier_cap_is_small_for_the_175b_shapes(lib):
+    """max_outliers shrinks the outlier tiles (2*s*cap + 2*cap*o bytes): at
+    cap 64 the OPT-175B FFN and decode workspaces are tens of MB, against
+    the worst case's 1.2 GB of W^O capacity alone."""
+    def a256(x):
+        return (x + 255) // 256 * 256
+
+    for s, h, o in [(2048, 12288, 49152), (8, 12288, 49152), (16, 256, 256)]:
+        full = lib.llmint8_workspace_size(s, h, o)
+        assert lib.llmint8_workspace_size_ex(s, h, o, 0) == full
+        assert lib.llmint8_workspace_size_ex(s, h, o, h) == full
+        for cap in (1, 16, 64):
+            got = lib.llmint8_workspace_size_ex(s, h, o, cap)
+            assert got == full - a256(2 * s * h) - a256(2 * h * o) \
+                + a256(2 * s * cap) + a256(2 * cap * o)
+            assert (lib.llmint8_workspace_size_host_ex(s, h, o, cap)
+                    == got + a256(2 * s * h) + a256(2 * s * o))
+    assert lib.llmint8_workspace_size(2048, 12288, 49152) > 1.2e9
+    assert lib.llmint8_workspace_size_ex(2048, 12288, 49152, 64) < 40e6
+    assert lib.llmint8_workspace_size_ex(8, 12288, 49152, 64) < 10e6
+    assert lib.llmint8_workspace_size_ex(16, 256, 256, -1) == 0
+    assert lib.llmint8_workspace_size_ex(16, 256, 256, 257) == 0
+
+
+@needs_no_gpu
+def test_outlier_cap_and_status_word_are_validated_on_the_host(lib):
+    w = _weight(256, 256)
+    big = 1 << 40
+    for bad in (-1, 257):
+        opts = binding.llmint8_matmul_opts()
+        opts.max_outliers = bad
+        assert lib.llmint8_matmul_ex(FAKE, 4, ctypes.byref(w), 6.0, FAKE, FAKE, big,
+                                     ctypes.byref(opts), None) == -7
+        assert lib.llmint8_matmul_host_ex(FAKE, 4, ctypes.byref(w), 6.0, FAKE, FAKE, big,
+                                          ctypes.byref(opts), None) == -7
+    # a workspace sized for cap 16 is enough for a call with cap 16 only
+    opts = binding.llmint8_matmul_opts()
+    opts.max_outliers = 16
+    need = lib.llmint8_workspace_size_ex(4, 256, 256, 16)
+    opts.status_host = None
+    assert lib.llmint8_matmul(FAKE, 4, ctypes.byref(w), 6.0, FAKE, FAKE, need, None) == -4
+    # a status word the device cannot address is refused before any work
+    word = ctypes.c_int32(0)
+    opts.status_host = ctypes.cast(ctypes.pointer(word), ctypes.c_void_p)
+    assert lib.llmint8_matmul_ex(FAKE, 4, ctypes.byref(w), 6.0, FAKE, FAKE, need,
+                                 ctypes.byref(opts), None) == -7
+    n = ctypes.c_int32(0)
+    assert lib.llmint8_read_outlier_tiles_ex(FAKE, big, 4, 256, 256, 300, ctypes.byref(n),
+                                             None, None, None) == -7

@@ -53,7 +53,7 @@ def test_reference_arm_under_torchrun_prints_one_line_from_rank_zero():
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
            "--nproc-per-node", "2", "--master-addr", "127.0.0.1",
            "--master-port", str(port), os.path.join(ROOT, "bench.py"),
-           "--impl", "reference", "--workload", "tiny", "--steps", "2",
+           "--impl", "reference", "--gpus", "2", "--workload", "tiny", "--steps", "2",
            "--warmup", "3", "--cpu-seconds", "0.5"]
     out = subprocess.run(cmd, capture_output=True, text=True, timeout=600,
                          cwd=ROOT)
@@ -64,6 +64,9 @@ def test_reference_arm_under_torchrun_prints_one_line_from_rank_zero():
     assert d["impl"] == "reference" and d["n_gpus"] == 2
     assert d["cpu_baseline"]["kind"] == "oracle" and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+    assert d["config"]["parallelism"] == "replicas x2"
+    # the time per step is that of the sample actually run each step
+    assert d["ms_per_step"] * d["steps"] / 1e3 < 600
 
 
 def test_threshold_and_scale_options_reach_the_workload_and_the_json_line():
@@ -82,3 +85,43 @@ def test_threshold_and_scale_options_reach_the_workload_and_the_json_line():
     assert json.loads(json.dumps({"alpha": bench.alpha_json(off.alpha)})) == {"alpha": "inf"}
     assert bench.alpha_json(6.0) == 6.0
     assert bench.SCALE_MODES == {"row": 0, "column": 0, "tensor": 1}
+
+
+def test_gpus_flag_and_launcher_must_agree():
+    """--gpus N without torchrun launches N ranks; under a launcher whose
+    WORLD_SIZE differs from N the run stops with an error instead of timing
+    the wrong number of replicas."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.check_world(1, {}) == "run"
+    assert bench.check_world(4, {}) == "launch"
+    assert bench.check_world(2, {"WORLD_SIZE": "2"}) == "run"
+    msg = bench.check_world(8, {"WORLD_SIZE": "1"})
+    assert msg not in ("run", "launch") and "WORLD_SIZE=1" in msg
+    cmd = bench.launch_command(2, ["--gpus", "2", "--steps", "3"])
+    assert cmd[1:3] == ["-m", "torch.distributed.run"]
+    assert "--nproc-per-node" in cmd and cmd[cmd.index("--nproc-per-node") + 1] == "2"
+    assert "127.0.0.1" in cmd and cmd[-3:] == ["--gpus", "2", "--steps", "3"][-3:]
+
+
+def test_both_arms_describe_the_workload_with_the_same_config():
+    """The reference arm's config has exactly our arm's keys and values, so
+    the two lines describe one workload; the L2 policy depends on the
+    workload's input size only."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from mixed_precision_int8_b200 import workloads
+    args = bench.parse_args(["--workload", "opt175b_ffn_up_prefill"])
+    for name in workloads.WORKLOAD_ORDER:
+        wl = workloads.get_workload(name)
+        c1 = bench.workload_config(wl, 1, args)
+        assert set(c1) == {"workload", "s", "h", "o", "alpha", "outlier_cols",
+                           "parallelism", "scales", "l2"}
+        assert c1 == bench.workload_config(wl, 1, args)
+    big = workloads.get_workload("opt175b_ffn_up_prefill")
+    small = workloads.get_workload("opt6.7b_attn_prefill")
+    assert not bench.needs_flush(big) and "no flush" in bench.l2_policy(big)
+    assert bench.needs_flush(small) and "flushed" in bench.l2_policy(small)
+    assert not bench.needs_flush(workloads.get_workload("opt175b_decode"))
+    assert args.workload == "opt175b_ffn_up_prefill"
+    assert bench.parse_args([]).workload == "opt175b_ffn_up_prefill"

@@ -127,6 +127,37 @@ def test_matmul_small_cases(case):
     assert np.array_equal(WO.numpy().view(np.uint16), WO_ref.view(np.uint16))
 
 
+PLAIN_CASES = [c for c in SMALL if c[0] > 16] + [
+    (300, 1040, 15376, tuple(range(3, 1040, 61)), 6.0),   # more tiles than SMs
+]
+
+
+@pytest.mark.parametrize("keep_fp16", [False, True], ids=["w_from_int8", "w_fp16"])
+@pytest.mark.parametrize("case", PLAIN_CASES, ids=lambda c: f"{c[0]}x{c[1]}x{c[2]}a{c[4]}")
+def test_plain_gemm_launch_matches_oracle_and_default_launch(case, keep_fp16):
+    """The ordinary GEMM launch (outlier rows of W built by the activation
+    fix-up, no CTA waiting for another) against the oracle, and bit for bit
+    against the default launch (cooperative where accepted)."""
+    X, W, alpha = _small_inputs(case, seed=17)
+    pw, _ = gpu_prepare(W, keep_fp16=keep_fp16)
+    Wq_ref, aw_ref = oracle.prepare_weight(W)
+    ref, ci_ref = oracle.matmul(X, Wq_ref, aw_ref, alpha, want_ci=True,
+                                W16=W if keep_fp16 else None)
+    f_ref, idx_ref, n_ref = oracle.detect_outliers(X, alpha)
+    WO_ref = (np.ascontiguousarray(W[idx_ref, :]) if keep_fp16
+              else oracle.outlier_weights(Wq_ref, aw_ref, idx_ref))
+    outs = []
+    for plain in (True, False):
+        out, ci, ws = gpu_matmul(X, pw, alpha, path=1, want_ci=True, gemm_plain=plain)
+        assert np.array_equal(ci, ci_ref), f"int32 accumulators, plain={plain}"
+        assert_close_fp16(out, ref, f"out plain={plain}")
+        n, _, WO = binding.llmint8_read_outlier_tiles(ws)
+        assert n == n_ref
+        assert np.array_equal(WO.numpy().view(np.uint16), WO_ref.view(np.uint16)), plain
+        outs.append(out)
+    assert np.array_equal(outs[0].view(np.uint16), outs[1].view(np.uint16))
+
+
 @pytest.mark.parametrize("case", SMALL, ids=lambda c: f"{c[0]}x{c[1]}x{c[2]}a{c[4]}")
 def test_matmul_small_cases_with_fp16_outlier_rows(case):
     """The caller's fp16 W supplies the outlier rows of W: output against the
