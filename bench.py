@@ -367,7 +367,7 @@ def bench_workload(name, args, world, rank, local, K, Wm, headline: bool):
     torch.cuda.synchronize()
     del Wd
     out = torch.empty((s, o), dtype=torch.float16, device=dev)
-    ws = binding.Workspace(s, h, o, device=dev)
+    ws = binding.Workspace(s, h, o, device=dev, max_outliers=args.max_outliers)
     flush = (torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
              if needs_flush(wl) else None)
     stream = torch.cuda.current_stream()
@@ -382,9 +382,6 @@ def bench_workload(name, args, world, rank, local, K, Wm, headline: bool):
         step()
     torch.cuda.synchronize()
     launches_per_step = binding.llmint8_matmul.last_launches
-    gemm_launch = {-1: "decode kernel", 0: "ordinary", 1: "cooperative",
-                   2: "cooperative, programmatic dependent"}.get(
-        binding.llmint8_matmul.last_gemm_launch, "unknown")
 
     def timed_steps(n, with_kernel_events: bool):
         """n steps, each between CUDA events on the launching stream (after
@@ -446,7 +443,8 @@ def bench_workload(name, args, world, rank, local, K, Wm, headline: bool):
     if not args.no_e2e:
         Xh = torch.from_numpy(X).pin_memory()
         outh = torch.empty((s, o), dtype=torch.float16).pin_memory()
-        wsh = binding.Workspace(s, h, o, device=dev, host=True)
+        wsh = binding.Workspace(s, h, o, device=dev, host=True,
+                                max_outliers=args.max_outliers)
         for _ in range(max(1, Wm)):
             binding.llmint8_matmul_host(Xh, pw, wl.alpha, outh, wsh, x_scale=x_mode)
         e_ms = []
@@ -505,7 +503,6 @@ def bench_workload(name, args, world, rank, local, K, Wm, headline: bool):
             "h2d_bytes_per_step": 2 * s * h,
             "d2h_bytes_per_step": 2 * s * o},
         "gpu_launches": launches_per_step * n_steps,
-        "gemm_launch": gemm_launch,
         "roofline": roof,
         "device_status": status_bits,
         "fp16_matmul": None if fp16_ms is None else {
@@ -553,8 +550,7 @@ def run_ours(args, world, rank, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "i8", "data": "synthetic (seeded, OPT-shaped outliers)",
         "config": head["config"], "e2e": head["e2e"],
-        "gpu_launches": head["gpu_launches"], "gemm_launch": head["gemm_launch"],
-        "roofline": head["roofline"],
+        "gpu_launches": head["gpu_launches"], "roofline": head["roofline"],
         "step_roofline_frac": head["step_roofline_frac"],
         "device_status": head["device_status"],
         "fp16_matmul": head["fp16_matmul"], "clocks": head["clocks"],
@@ -627,6 +623,8 @@ def parse_args(argv=None):
                     help="skip the sustained-load window (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer end-to-end timing (profiling runs)")
+    ap.add_argument("--max-outliers", type=int, default=0,
+                    help="outlier columns the workspace holds (0: h, any alpha)")
     ap.add_argument("--alpha", type=float, default=None,
                     help="outlier threshold instead of the workload's (inf: no "
                          "decomposition, pure vector-wise int8)")

@@ -136,17 +136,17 @@ typedef struct {
  *      otherwise the call's last kernel ORs the workspace's status bits into
  *      it as it finishes. The caller clears the word, and re-initialises the
  *      workspace (llmint8_workspace_init), before going on.
- *  gemm_plain: 0 (automatic): the prefill GEMM is launched cooperatively
- *      where the device and driver accept it (all its CTAs resident at once);
- *      its CTAs then build the fp16 outlier rows of W while their first
- *      mainloops run and wait for each other's shares. Nonzero: an ordinary
- *      launch, with those rows built by the activation kernels first and no
- *      CTA of the GEMM waiting for another (for callers that cannot have a
- *      cooperative launch, e.g. under SM partitioning). Results are the
- *      same bit for bit.
- *  gemm_launch (out): how this call launched its int8 GEMM: 0 ordinary,
- *      1 cooperative, 2 cooperative with programmatic dependent launch
- *      (overlapping the previous kernel's tail), -1 the decode kernel. */
+ *  wo_build: where the prefill path builds the fp16 outlier rows of W
+ *      (Step 2, W side); results are the same bit for bit in every form.
+ *      LLMINT8_WO_SHARED (0, default): the GEMM's CTAs, each a share, while
+ *      their first mainloops run; each then waits a short, bounded time for
+ *      the other shares, and a CTA that does not see them all in time (its
+ *      peers not resident, e.g. under SM partitioning) builds every row
+ *      itself, so the result never depends on how many CTAs run at once.
+ *      LLMINT8_WO_BEFORE_GEMM (1): the activation kernels, before the GEMM;
+ *      no CTA of the GEMM waits for another. LLMINT8_WO_EACH_CTA (2): every
+ *      GEMM CTA builds all rows itself at once (the fallback above, on
+ *      purpose; for testing). Anything else is LLMINT8_ERR_ARG. */
 typedef struct {
     void *gemm_event_start;
     void *gemm_event_stop;
@@ -156,9 +156,12 @@ typedef struct {
     int32_t x_scale;
     int32_t max_outliers;
     int32_t *status_host;
-    int32_t gemm_plain;
-    int32_t gemm_launch;
+    int32_t wo_build;
 } llmint8_matmul_opts;
+
+#define LLMINT8_WO_SHARED 0
+#define LLMINT8_WO_BEFORE_GEMM 1
+#define LLMINT8_WO_EACH_CTA 2
 
 /* Scale granularity ("Quantization Primitives": absmax over a whole tensor;
  * "Vector-wise Quantization": one constant per row of X and per column of

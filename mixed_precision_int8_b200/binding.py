@@ -27,6 +27,8 @@ NOALLOC_MAX_SCRATCH_BYTES = 64 << 20  # LLMINT8_NOALLOC_MAX_SCRATCH_BYTES
 DEV_TIMEOUT_SELFTEST = 0x20
 DEV_OUTLIER_CAP = 0x40
 SCALE_VECTORWISE = 0  # LLMINT8_SCALE_VECTORWISE: per row of X / column of W
+# where the prefill path builds the fp16 outlier rows of W (LLMINT8_WO_*)
+WO_SHARED, WO_BEFORE_GEMM, WO_EACH_CTA = 0, 1, 2
 SCALE_TENSORWISE = 1  # LLMINT8_SCALE_TENSORWISE: one constant per tensor
 
 _c_i64, _c_i32, _c_f32 = ctypes.c_int64, ctypes.c_int32, ctypes.c_float
@@ -42,8 +44,7 @@ class llmint8_matmul_opts(ctypes.Structure):
     _fields_ = [("gemm_event_start", _vp), ("gemm_event_stop", _vp),
                 ("ci_dev", _vp), ("path", _c_i32), ("launches", _c_i32),
                 ("x_scale", _c_i32), ("max_outliers", _c_i32),
-                ("status_host", _vp), ("gemm_plain", _c_i32),
-                ("gemm_launch", _c_i32)]
+                ("status_host", _vp), ("wo_build", _c_i32)]
 
 
 class Llmint8Error(RuntimeError):
@@ -261,7 +262,7 @@ def llmint8_matmul(X: torch.Tensor, w: PreparedWeight, alpha: float = 6.0,
                    events=None, stream=None,
                    x_scale: int = SCALE_VECTORWISE,
                    status_host: Optional[HostStatusWord] = None,
-                   gemm_plain: bool = False) -> torch.Tensor:
+                   wo_build: int = WO_SHARED) -> torch.Tensor:
     """C = LLM.int8()(X, W): X fp16 [s,h] on the GPU -> fp16 [s,o].
 
     ci (optional, int32 [s,o]) receives the exact int32 accumulators; path
@@ -269,7 +270,7 @@ def llmint8_matmul(X: torch.Tensor, w: PreparedWeight, alpha: float = 6.0,
     torch.cuda.Event pair recorded around the GEMM kernel; x_scale =
     SCALE_TENSORWISE quantises X with one constant for the whole tensor;
     status_host (a HostStatusWord) reports device anomalies on the next call;
-    gemm_plain forces the ordinary (non-cooperative) prefill GEMM launch.
+    wo_build picks where the fp16 outlier rows of W are built (WO_*).
     The workspace's max_outliers is passed along.
     """
     _f16_dev(X, "X")
@@ -284,7 +285,7 @@ def llmint8_matmul(X: torch.Tensor, w: PreparedWeight, alpha: float = 6.0,
     opts.path = int(path)
     opts.x_scale = int(x_scale)
     opts.max_outliers = workspace.max_outliers
-    opts.gemm_plain = int(bool(gemm_plain))
+    opts.wo_build = int(wo_build)
     if status_host is not None:
         opts.status_host = status_host.t.data_ptr()
     if ci is not None:
@@ -303,7 +304,6 @@ def llmint8_matmul(X: torch.Tensor, w: PreparedWeight, alpha: float = 6.0,
         _ptr(workspace.buf), workspace.nbytes, ctypes.byref(opts),
         _stream(stream)))
     llmint8_matmul.last_launches = int(opts.launches)
-    llmint8_matmul.last_gemm_launch = int(opts.gemm_launch)
     return out
 
 

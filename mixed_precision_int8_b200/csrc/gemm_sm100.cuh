@@ -15,13 +15,13 @@
 //   warp 1      one thread issues tcgen05.mma.kind::i8 (M=128, N=256, K=32)
 //               into a TMEM accumulator; tcgen05.commit frees ring slots
 //   warp 2      allocates / frees the 512 TMEM columns (2 accumulators)
-//   warps 4-11  epilogue: before the first tile (launched cooperatively, so
-//               every CTA is resident), a share of the fp16 outlier rows
-//               of W, gathered while the first tiles' mainloops run, then
-//               announced on a counter; otherwise those rows come built by
-//               the activation fix-up. Per tile, while the MMA runs, the
-//               column scales and the tile's slice of the outlier rows go
-//               to shared memory as fp32, and each
+//   warps 4-11  epilogue: before the first tile, a share of the fp16
+//               outlier rows of W, gathered while the first tiles'
+//               mainloops run and announced on a counter (or, with
+//               build_wo = 0, those rows come built by the activation
+//               fix-up). Per tile, while the MMA runs, the column scales
+//               and the tile's slice of the outlier rows go to shared
+//               memory as fp32, and each
 //               thread computes the outlier product of its row and its half
 //               of the tile's columns into registers (packed f32x2 FMAs).
 //               Once the accumulator is ready, each warp tcgen05.lds its half
@@ -29,8 +29,10 @@
 //               dequantises, adds the outlier product and writes fp16
 //               through a 64B-swizzled 32x32 staging block with TMA stores;
 //               the other accumulator is being filled by the MMA meanwhile.
-// The only wait on other CTAs is for their shares of the outlier rows of W,
-// and only in a cooperative launch, where all of them are resident.
+// The one wait on other CTAs, for their shares of the outlier rows of W, is
+// short and never needed for correctness: a CTA that has not seen every
+// share within wo_wait_ns (other CTAs not resident, e.g. under SM
+// partitioning) builds all the rows itself and goes on.
 // Every wait is bounded by the global timer; on a timeout the CTA records a
 // status bit, drains its in-flight copies and MMAs, frees TMEM and returns.
 #pragma once
@@ -93,8 +95,9 @@ struct Params {
   const int8_t *wq;       // [o][h] int8 codes of W
   const uint16_t *w16;    // optional fp16 W [h][o]: WO rows are its own rows
   const int32_t *idx;     // outlier columns, ascending
-  int32_t build_wo;       // 1 (cooperative launch only): the CTAs build WO
+  int32_t build_wo;       // 1: the CTAs build WO (shares, then the wait)
   int32_t *wo_counter;    // CTAs done with their share of WO; zero on entry
+  uint64_t wo_wait_ns;    // how long a CTA waits for the other shares
   const int32_t *n_out;   // device scalar |O|
   int32_t wo_cap;         // outlier rows the workspace holds; |O| above it:
                           // no outlier product (the fix-up flagged it)
@@ -280,25 +283,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // (1) column scales and fp16 outlier rows of this tile into shared
       //     memory, while the MMA still works on the accumulator
       if (!wo_ready) {
-        // every CTA's share of WO is written (bounded wait; all CTAs are
-        // resident, so it ends unless a CTA has aborted)
+        // every CTA's share of WO is written, or, if that takes longer than
+        // wo_wait_ns, this CTA writes all of WO itself (the same values)
         bool got = true;
         if (et == 0) {
           const uint64_t t0 = global_timer_ns();
           while (*reinterpret_cast<volatile int32_t *>(p.wo_counter) < (int32_t)gridDim.x) {
-            if (*abort_flag || global_timer_ns() - t0 > p.timeout_ns) {
+            if (*abort_flag || global_timer_ns() - t0 > p.wo_wait_ns) {
               got = false;
               break;
             }
             __nanosleep(128);
           }
-          if (!got && !*abort_flag) {
-            *abort_flag = 1;
-            atomicOr(p.status, LLMINT8_DEV_TIMEOUT_EPILOGUE);
-          }
           __threadfence();
         }
-        if (named_barrier_or(EPI_BARRIER, NUM_EPI_THREADS, !got)) break;
+        if (named_barrier_or(EPI_BARRIER, NUM_EPI_THREADS, !got)) {
+          // the same decision in every epilogue thread: stop on an abort,
+          // else build all of WO here
+          if (named_barrier_or(EPI_BARRIER, NUM_EPI_THREADS, *abort_flag != 0)) break;
+          build_wo_rows(n_out, p.idx, p.wq, p.aw, p.w16, p.h, p.o, p.WO, et, NUM_EPI_THREADS);
+          __threadfence();
+          named_barrier(EPI_BARRIER, NUM_EPI_THREADS);
+        }
         wo_ready = true;
       }
       named_barrier(EPI_BARRIER, NUM_EPI_THREADS);  // previous tile done reading

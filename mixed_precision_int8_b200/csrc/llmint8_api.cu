@@ -6,7 +6,6 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
-#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -25,24 +24,20 @@ using namespace llmint8;
 constexpr int64_t kMaxH = 133144;  // 127*127*h must fit int32
 constexpr int64_t kDecodeMaxRows = decode::MAX_ROWS;
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per individual wait
+// how long a GEMM CTA waits for the other CTAs' shares of the outlier rows of
+// W before it builds them all itself: far longer than the shares take when
+// every CTA is resident (a few microseconds), and shorter than building them
+// all alone takes on the large shapes, so it runs out only when peers are
+// not resident (SM partitioning, time slicing)
+constexpr uint64_t kWoWaitNs = 500000ull;
 // dynamic shared memory of k_act_rows (one CTA per SM)
 constexpr uint32_t kActSmemOnePerSm = 220 * 1024;
 
 // ----------------------------------------------------------- device info
-// How the prefill GEMM is launched on a device. Cooperatively (all CTAs
-// resident at once, a launch the driver refuses otherwise), its CTAs build
-// the fp16 outlier rows of W themselves while their first mainloops run and
-// wait for each other's shares; otherwise the activation fix-up builds them
-// before the GEMM and no CTA waits for another. The first launch on a
-// device finds out which form the driver accepts (with programmatic
-// dependent launch, then without) and the answer is kept.
-enum GemmLaunch { kGemmUntested = -1, kGemmPlain = 0, kGemmCoop = 1, kGemmCoopPdl = 2 };
-
 struct DeviceInfo {
   bool init = false;
   bool supported = false;
   int sm_count = 0;
-  std::atomic<int> gemm_launch{kGemmUntested};
 };
 constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
@@ -69,16 +64,6 @@ llmint8_status device_info(DeviceInfo **out) {
       if (cudaFuncSetAttribute(k_act_rows, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)kActSmemOnePerSm) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
-      // a cooperative GEMM needs one resident CTA per SM of its grid
-      int coop = 0, per_sm = 0;
-      if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess ||
-          cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemm::k_gemm_i8_fused,
-                                                        gemm::NUM_THREADS,
-                                                        gemm::SMEM_BYTES) != cudaSuccess) {
-        cudaGetLastError();
-        coop = 0;
-      }
-      d.gemm_launch.store((coop && per_sm >= 1) ? kGemmUntested : kGemmPlain);
     }
     d.init = true;
   }
@@ -186,8 +171,8 @@ int32_t *count_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 1; }
 int32_t *block_counter_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 2; }
 int32_t *act_counter_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 3; }
 int32_t *done_counter_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 4; }
-// [6] CTAs of a cooperative GEMM done with their share of the outlier rows
-// of W (zeroed by the call's activation kernels)
+// [6] CTAs of the GEMM done with their share of the outlier rows of W
+// (zeroed by the call's activation kernels)
 int32_t *wo_counter_word(void *ws) { return reinterpret_cast<int32_t *>(ws) + 6; }
 float *tensor_scale_word(void *ws) { return reinterpret_cast<float *>(ws) + 5; }
 constexpr int kSelftestWord = 8;  // a status-block word no kernel sets
@@ -234,38 +219,21 @@ llmint8_status last_launch() {
 
 // Launch with programmatic stream serialization when `pdl`: the kernel may
 // be scheduled while its predecessor drains; it orders itself after the
-// predecessor with griddepcontrol.wait before touching memory. With `coop`
-// the launch is cooperative: every CTA of the grid is resident at once, or
-// the launch fails (and enqueues nothing).
+// predecessor with griddepcontrol.wait before touching memory.
 template <typename... KArgs, typename... Args>
-cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                      cudaStream_t st, bool pdl, bool coop, Args &&...args) {
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                   cudaStream_t st, bool pdl, Args &&...args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[2];
-  unsigned n = 0;
-  if (pdl) {
-    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[n].val.programmaticStreamSerializationAllowed = 1;
-    ++n;
-  }
-  if (coop) {
-    attr[n].id = cudaLaunchAttributeCooperative;
-    attr[n].val.cooperative = 1;
-    ++n;
-  }
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = n;
+  cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
-}
-
-template <typename... KArgs, typename... Args>
-cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                   cudaStream_t st, bool pdl, Args &&...args) {
-  return launch_ex(kernel, grid, block, smem, st, pdl, false, std::forward<Args>(args)...);
 }
 
 // Steps 1, 2 and 4 (activation side, plus the fp16 outlier rows of W when
@@ -507,6 +475,8 @@ llmint8_status check_opts(const llmint8_matmul_opts *opts, int64_t s, int64_t h)
   if (opts->x_scale != LLMINT8_SCALE_VECTORWISE && opts->x_scale != LLMINT8_SCALE_TENSORWISE)
     return LLMINT8_ERR_ARG;
   if (outlier_cap(opts, h) < 0) return LLMINT8_ERR_ARG;
+  if (opts->wo_build < LLMINT8_WO_SHARED || opts->wo_build > LLMINT8_WO_EACH_CTA)
+    return LLMINT8_ERR_ARG;
   if (opts->status_host) {
     // pinned host memory the device reaches at the same address
     cudaPointerAttributes pa;
@@ -530,10 +500,7 @@ bool host_status_set(const llmint8_matmul_opts *opts) {
 llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w, float alpha,
                            uint16_t *out, void *ws, size_t ws_bytes, llmint8_matmul_opts *opts,
                            cudaStream_t st, bool host_layout, bool reset_state = false) {
-  if (opts) {
-    opts->launches = 0;
-    opts->gemm_launch = -1;
-  }
+  if (opts) opts->launches = 0;
   llmint8_status rc = validate_weight(w);
   if (rc) return rc;
   if (s < 0 || s > (int64_t)INT32_MAX) return LLMINT8_ERR_SHAPE;
@@ -606,13 +573,13 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
   act.w16 = w->w16_dev;
   act.o = o;
   act.cap = (int32_t)cap;
-  // prefill: the fp16 outlier rows of W come from the GEMM itself when it
-  // can be launched cooperatively, else from the activation kernels;
-  // decode: the W^O gather and the finishing step run inside the decode
-  // kernel; its tile counters and the s rows of int32 partial sums (one
-  // contiguous region) start from zero
-  const bool gemm_builds_wo = !use_decode && dev->gemm_launch.load() != kGemmPlain &&
-                              !(opts && opts->gemm_plain);
+  // prefill: the GEMM's CTAs build the fp16 outlier rows of W themselves
+  // while their first mainloops run (unless gemm_plain asks for them from
+  // the activation kernels); decode: the W^O gather and the finishing step
+  // run inside the decode kernel; its tile counters and the s rows of int32
+  // partial sums (one contiguous region) start from zero
+  const int wo_build = opts ? opts->wo_build : LLMINT8_WO_SHARED;
+  const bool gemm_builds_wo = !use_decode && wo_build != LLMINT8_WO_BEFORE_GEMM;
   act.WO = (use_decode || gemm_builds_wo) ? nullptr : wo;
   act.gemm_counter = gemm_builds_wo ? wo_counter_word(ws) : nullptr;
   int32_t *tiles = reinterpret_cast<int32_t *>(wsb + L.tiles);
@@ -709,44 +676,11 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
     p.timeout_ns = kTimeoutNs;
     const int64_t tiles = (int64_t)p.num_m_blocks * p.num_n_blocks;
     const int grid = (int)(tiles < dev->sm_count ? tiles : dev->sm_count);
-    e = cudaErrorNotSupported;
-    int used = kGemmPlain;
-    if (gemm_builds_wo) {
-      // cooperative, with programmatic dependent launch where accepted
-      p.build_wo = 1;
-      const int mode = dev->gemm_launch.load();
-      if (mode == kGemmUntested || mode == kGemmCoopPdl) {
-        e = launch_ex(gemm::k_gemm_i8_fused, dim3(grid), dim3(gemm::NUM_THREADS),
-                      gemm::SMEM_BYTES, st, !timed, true, tmA, tmB, tmOut, p);
-        if (e == cudaSuccess) used = timed ? kGemmCoop : kGemmCoopPdl;
-        if (e == cudaSuccess && !timed) dev->gemm_launch.store(kGemmCoopPdl);
-      }
-      if (e != cudaSuccess && (mode == kGemmUntested || mode == kGemmCoop || timed)) {
-        cudaGetLastError();
-        e = launch_ex(gemm::k_gemm_i8_fused, dim3(grid), dim3(gemm::NUM_THREADS),
-                      gemm::SMEM_BYTES, st, false, true, tmA, tmB, tmOut, p);
-        if (e == cudaSuccess) used = kGemmCoop;
-        if (e == cudaSuccess && mode == kGemmUntested) dev->gemm_launch.store(kGemmCoop);
-      }
-      if (e != cudaSuccess) {
-        // refused: from now on the activation kernels build the rows; this
-        // call builds them in a launch of its own
-        cudaGetLastError();
-        dev->gemm_launch.store(kGemmPlain);
-        e = launch(k_build_wo, dim3((unsigned)(2 * dev->sm_count)), dim3(256), 0, st, true,
-                   (const int32_t *)count, (const int32_t *)idx, w->wq_dev, w->aw_dev,
-                   w->w16_dev, (int32_t)h, (int32_t)o, wo, (int32_t)cap);
-        if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
-        ++launches;
-      }
-    }
-    if (e != cudaSuccess) {
-      p.build_wo = 0;
-      e = launch(gemm::k_gemm_i8_fused, dim3(grid), dim3(gemm::NUM_THREADS), gemm::SMEM_BYTES,
-                 st, !timed, tmA, tmB, tmOut, p);
-    }
+    p.build_wo = gemm_builds_wo ? 1 : 0;
+    p.wo_wait_ns = wo_build == LLMINT8_WO_EACH_CTA ? 0 : kWoWaitNs;
+    e = launch(gemm::k_gemm_i8_fused, dim3(grid), dim3(gemm::NUM_THREADS), gemm::SMEM_BYTES, st,
+               !timed, tmA, tmB, tmOut, p);
     if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
-    if (opts) opts->gemm_launch = used;
     if (opts && opts->gemm_event_stop)
       cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->gemm_event_stop), st);
     ++launches;

@@ -38,14 +38,14 @@ def gpu_prepare(W: np.ndarray, keep_fp16: bool = False):
 
 
 def gpu_matmul(X: np.ndarray, pw, alpha: float, path: int = 0,
-               want_ci: bool = False, gemm_plain: bool = False):
+               want_ci: bool = False, wo_build: int = 0):
     Xd = to_dev(X)
     s = X.shape[0]
     ws = binding.Workspace(s, pw.h, pw.o)
     ci = (torch.full((s, pw.o), -7, dtype=torch.int32, device="cuda")
           if want_ci else None)
     out = binding.llmint8_matmul(Xd, pw, alpha, workspace=ws, ci=ci, path=path,
-                                 gemm_plain=gemm_plain)
+                                 wo_build=wo_build)
     torch.cuda.synchronize()
     assert binding.llmint8_read_device_status(ws) == 0
     return out.cpu().numpy(), (ci.cpu().numpy() if want_ci else None), ws

@@ -172,6 +172,12 @@ def test_scale_mode_constants_match_the_header():
     got = dict(re.findall(r"#define\s+LLMINT8_SCALE_(\w+)\s+(\d+)", text))
     assert int(got["VECTORWISE"]) == binding.SCALE_VECTORWISE
     assert int(got["TENSORWISE"]) == binding.SCALE_TENSORWISE
+    wo = dict(re.findall(r"#define\s+LLMINT8_WO_(\w+)\s+(\d+)", text))
+    assert (int(wo["SHARED"]), int(wo["BEFORE_GEMM"]), int(wo["EACH_CTA"])) == (
+        binding.WO_SHARED, binding.WO_BEFORE_GEMM, binding.WO_EACH_CTA)
+    bits = dict(re.findall(r"#define\s+LLMINT8_DEV_(\w+)\s+(0x[0-9a-fA-F]+)", text))
+    assert int(bits["TIMEOUT_SELFTEST"], 16) == binding.DEV_TIMEOUT_SELFTEST
+    assert int(bits["OUTLIER_CAP"], 16) == binding.DEV_OUTLIER_CAP
 
 
 @needs_no_gpu
@@ -262,3 +268,8 @@ def test_outlier_cap_and_status_word_are_validated_on_the_host(lib):
     n = ctypes.c_int32(0)
     assert lib.llmint8_read_outlier_tiles_ex(FAKE, big, 4, 256, 256, 300, ctypes.byref(n),
                                              None, None, None) == -7
+    for bad in (-1, 3):
+        opts = binding.llmint8_matmul_opts()
+        opts.wo_build = bad
+        assert lib.llmint8_matmul_ex(FAKE, 4, ctypes.byref(w), 6.0, FAKE, FAKE, big,
+                                     ctypes.byref(opts), None) == -7

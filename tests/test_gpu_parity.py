@@ -134,10 +134,11 @@ PLAIN_CASES = [c for c in SMALL if c[0] > 16] + [
 
 @pytest.mark.parametrize("keep_fp16", [False, True], ids=["w_from_int8", "w_fp16"])
 @pytest.mark.parametrize("case", PLAIN_CASES, ids=lambda c: f"{c[0]}x{c[1]}x{c[2]}a{c[4]}")
-def test_plain_gemm_launch_matches_oracle_and_default_launch(case, keep_fp16):
-    """The ordinary GEMM launch (outlier rows of W built by the activation
-    fix-up, no CTA waiting for another) against the oracle, and bit for bit
-    against the default launch (cooperative where accepted)."""
+def test_every_place_of_the_outlier_row_build_matches_the_oracle(case, keep_fp16):
+    """The fp16 outlier rows of W built by the GEMM's CTAs in shares (the
+    default), by the activation fix-up before the GEMM, and by every GEMM
+    CTA on its own (what a CTA falls back to when its peers are not
+    resident): each against the oracle, and bit for bit against each other."""
     X, W, alpha = _small_inputs(case, seed=17)
     pw, _ = gpu_prepare(W, keep_fp16=keep_fp16)
     Wq_ref, aw_ref = oracle.prepare_weight(W)
@@ -147,15 +148,16 @@ def test_plain_gemm_launch_matches_oracle_and_default_launch(case, keep_fp16):
     WO_ref = (np.ascontiguousarray(W[idx_ref, :]) if keep_fp16
               else oracle.outlier_weights(Wq_ref, aw_ref, idx_ref))
     outs = []
-    for plain in (True, False):
-        out, ci, ws = gpu_matmul(X, pw, alpha, path=1, want_ci=True, gemm_plain=plain)
-        assert np.array_equal(ci, ci_ref), f"int32 accumulators, plain={plain}"
-        assert_close_fp16(out, ref, f"out plain={plain}")
+    for mode in (binding.WO_SHARED, binding.WO_BEFORE_GEMM, binding.WO_EACH_CTA):
+        out, ci, ws = gpu_matmul(X, pw, alpha, path=1, want_ci=True, wo_build=mode)
+        assert np.array_equal(ci, ci_ref), f"int32 accumulators, wo_build={mode}"
+        assert_close_fp16(out, ref, f"out wo_build={mode}")
         n, _, WO = binding.llmint8_read_outlier_tiles(ws)
         assert n == n_ref
-        assert np.array_equal(WO.numpy().view(np.uint16), WO_ref.view(np.uint16)), plain
+        assert np.array_equal(WO.numpy().view(np.uint16), WO_ref.view(np.uint16)), mode
         outs.append(out)
-    assert np.array_equal(outs[0].view(np.uint16), outs[1].view(np.uint16))
+    for o in outs[1:]:
+        assert np.array_equal(outs[0].view(np.uint16), o.view(np.uint16))
 
 
 @pytest.mark.parametrize("case", SMALL, ids=lambda c: f"{c[0]}x{c[1]}x{c[2]}a{c[4]}")
