@@ -306,66 +306,43 @@ __device__ __forceinline__ uint32_t hmax2_mag(uint32_t acc, uint32_t w) {
   return *reinterpret_cast<const uint32_t *>(&r);
 }
 
-// Eight codes (bytes, column order) of one 16-byte chunk whose magnitudes
-// are all <= a, with r = RN(127/a) (r = 0 when a == 0). With v = |x| r,
-// which is within 2^-17 of 127|x|/a, two fmas at 128.5 -+ 2^-15 give
-// y = 128 + (1/2 -+ 2^-15 + v) to 2^-17 (y lies in [128, 256), whose
-// spacing is 2^-16), and byte 2 of y's bits is floor(y - 128). When the two
-// bytes agree, z = 127|x|/a + 1/2 lies strictly between the two sums, so
-// that byte is floor(z): the magnitude rounded half away from zero, which
-// is absmax_code()'s result. Otherwise (z within about 2^-15 of an
-// integer) the chunk takes the exact two-residual correction. The sign is
-// applied bytewise: -n as a byte is (0x80 - n) ^ 0x80 for 0 <= n <= 127.
-__device__ __forceinline__ uint32_t gather_byte2(const uint64_t p01, const uint64_t p23) {
-  return prmt(prmt((uint32_t)p01, (uint32_t)(p01 >> 32), 0x0062u),
-              prmt((uint32_t)p23, (uint32_t)(p23 >> 32), 0x0062u), 0x5410u);
+// The per-row constant of the row codes: r2 = 2 RU(127 / a), twice the
+// reciprocal rounded up (0 when a == 0, so every code is 0).
+__device__ __forceinline__ float row_code_scale(float a) {
+  return a > 0.0f ? 2.0f * __fdiv_ru(127.0f, a) : 0.0f;
 }
 
-// Codes of one chunk (see above). Where the two candidates differ, the
-// result is the lower one or the next integer: it is the next one exactly
-// when 127|x| - (n + 1/2) a >= 0, a residual that one fma gives with its
-// sign exact ((n + 1/2) has at most 9 significant bits, a at most 11, so
-// the product is an exact fp32 value). Lanes whose |x| exceed a (values >=
-// alpha in outlier columns, zeroed later) get unspecified codes; nothing
-// else depends on them.
-__device__ __forceinline__ uint2 quant8_fma(const uint4 v, float a, float r) {
+// Eight codes (bytes, column order) of one 16-byte chunk whose magnitudes
+// are all <= a, with r2 = row_code_scale(a). Per element one fma rounded
+// toward minus infinity gives k = floor(2 |x| RU(127/a) + 1) as the low
+// byte of RM(|x| r2 + (2^23 + 1)) (in [2^23, 2^24) the fp32 spacing is 1),
+// and the code's magnitude is k >> 1 = floor(|x| RU(127/a) + 1/2). Since
+// RU(127/a) >= 127/a, that value is never below the exact 127|x|/a + 1/2
+// and exceeds it by less than q 2^-23, which is less than its distance to
+// the next integer whenever it is not an integer (binary16 mantissas have 11
+// bits): so k >> 1 is round-half-away-from-zero(127|x|/a), absmax_code()'s
+// result, ties included, with no division and no near-tie correction. The
+// sign is applied bytewise: -n as a byte is (0x80 - n) ^ 0x80 for
+// 0 <= n <= 127. Lanes whose |x| exceed a (values >= alpha in outlier
+// columns, zeroed later) get unspecified codes; nothing else depends on them.
+__device__ __forceinline__ uint2 quant8(const uint4 v, float r2) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  const uint64_t r2 = f32x2_pack(r, r);
-  const uint64_t clo = f32x2_pack(128.5f - 3.0517578125e-05f, 128.5f - 3.0517578125e-05f);
-  const uint64_t chi = f32x2_pack(128.5f + 3.0517578125e-05f, 128.5f + 3.0517578125e-05f);
-  uint64_t lo[4], hi[4], xm[4];
+  const uint64_t rr = f32x2_pack(r2, r2);
+  const uint64_t c = f32x2_pack(8388609.0f, 8388609.0f);  // 2^23 + 1
+  uint64_t y[4];
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
     const uint32_t m = w[e] & 0x7FFF7FFFu;
     const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&m));
-    xm[e] = f32x2_pack(f.x, f.y);
-    lo[e] = f32x2_fma(xm[e], r2, clo);
-    hi[e] = f32x2_fma(xm[e], r2, chi);
+    y[e] = f32x2_fma_rm(f32x2_pack(f.x, f.y), rr, c);
   }
-  // byte 2 of each sum; at most 0x7F for every |x| <= a, and masked so the
-  // unspecified ones cannot carry or borrow across bytes below
-  uint32_t n0 = gather_byte2(lo[0], lo[1]);
-  uint32_t n1 = gather_byte2(lo[2], lo[3]);
-  const bool near = (n0 != gather_byte2(hi[0], hi[1])) | (n1 != gather_byte2(hi[2], hi[3]));
-  n0 &= 0x7F7F7F7Fu;
-  n1 &= 0x7F7F7F7Fu;
-  if (near) {
-    const uint64_t c127 = f32x2_pack(127.0f, 127.0f);
-    const uint64_t cm = f32x2_pack(-127.5f, -127.5f);
-    const uint64_t one = f32x2_pack(1.0f, 1.0f);
-    const uint64_t na = f32x2_pack(-a, -a);
-    uint32_t up[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      // 128 + n (the sum with its fraction bits cleared), then n + 1/2
-      const uint64_t base = lo[e] & 0xFFFF0000FFFF0000ull;
-      const uint64_t half = f32x2_fma(base, one, cm);
-      const uint64_t res = f32x2_fma(half, na, f32x2_mul(xm[e], c127));
-      up[e] = (f32x2_lo(res) >= 0.0f ? 1u : 0u) | (f32x2_hi(res) >= 0.0f ? 0x100u : 0u);
-    }
-    n0 += up[0] | (up[1] << 16);
-    n1 += up[2] | (up[3] << 16);
-  }
+  // byte 0 of each result is k; the shift leaves k >> 1 in each byte
+  const uint32_t k0 = prmt(prmt((uint32_t)y[0], (uint32_t)(y[0] >> 32), 0x0040u),
+                           prmt((uint32_t)y[1], (uint32_t)(y[1] >> 32), 0x0040u), 0x5410u);
+  const uint32_t k1 = prmt(prmt((uint32_t)y[2], (uint32_t)(y[2] >> 32), 0x0040u),
+                           prmt((uint32_t)y[3], (uint32_t)(y[3] >> 32), 0x0040u), 0x5410u);
+  const uint32_t n0 = (k0 >> 1) & 0x7F7F7F7Fu;
+  const uint32_t n1 = (k1 >> 1) & 0x7F7F7F7Fu;
   const uint32_t s0 = prmt(w[0], w[1], 0xFDB9u);  // 0xFF where x < 0
   const uint32_t s1 = prmt(w[2], w[3], 0xFDB9u);
   const uint32_t g0 = (0x80808080u - n0) ^ 0x80808080u;
@@ -374,15 +351,15 @@ __device__ __forceinline__ uint2 quant8_fma(const uint4 v, float a, float r) {
 }
 
 // Codes for one 16-byte chunk (8 columns starting at c) of row `row`, with
-// r = RN(127/a): quant8_fma, outlier columns zeroed, and (if XO) the fp16
-// values of the chunk's outlier columns written to XO[row][rank].
-__device__ __forceinline__ void quantize_chunk(const uint4 v, uint32_t mw, int32_t c, float a,
-                                               float r, int64_t row, int32_t n_out,
+// r2 = row_code_scale(a): quant8, outlier columns zeroed, and (if XO) the
+// fp16 values of the chunk's outlier columns written to XO[row][rank].
+__device__ __forceinline__ void quantize_chunk(const uint4 v, uint32_t mw, int32_t c,
+                                               float r2, int64_t row, int32_t n_out,
                                                const int32_t *word_prefix,
                                                int8_t *__restrict__ qr,
                                                uint16_t *__restrict__ XO) {
   const uint32_t mk = (mw >> (c & 31)) & 0xFFu;
-  uint2 q = quant8_fma(v, a, r);
+  uint2 q = quant8(v, r2);
   if (mk != 0u) {
     uint32_t keep[2] = {0u, 0u};
 #pragma unroll
@@ -495,14 +472,14 @@ __global__ void __launch_bounds__(kActMaxWarps * 32) k_act_rows(const ActRowsPar
       break;
     }
     const float a = half_bits_to_float(run);
-    const float r = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
+    const float r2 = row_code_scale(a);
     if (leader) p.ax[row] = a;
     // Step 4 against the candidate scale (codes of values >= alpha are
     // overwritten by the fix-up, which zeroes every outlier column)
     int8_t *qr = p.Xq + row * h;
 #pragma unroll 2
     for (int32_t c = c0; c < nchunks; c += cstep)
-      *reinterpret_cast<uint2 *>(qr + 8 * c) = quant8_fma(rv[c], a, r);
+      *reinterpret_cast<uint2 *>(qr + 8 * c) = quant8(rv[c], r2);
     // every thread of the group is done with this stage (and with red[])
     if (wpr > 1) named_barrier(gbar, gthreads);
     else __syncwarp();
@@ -685,7 +662,7 @@ __global__ void __launch_bounds__(kFixThreads) k_act_fixup(const FixupParams p) 
 #pragma unroll
     for (int i = 1; i < kFixThreads / 32; ++i) mbits = max(mbits, red[i]);
     const float a = half_bits_to_float(mbits);
-    const float rr = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
+    const float rr = row_code_scale(a);
     if (tid == 0) ax[r] = a;
     int8_t *qr = Xq + r * h;
     for (int32_t c0 = tid; c0 < nchunks; c0 += 8 * kFixThreads) {
@@ -699,7 +676,7 @@ __global__ void __launch_bounds__(kFixThreads) k_act_fixup(const FixupParams p) 
       for (int u = 0; u < 8; ++u) {
         const int32_t c = c0 + u * kFixThreads;
         if (c < nchunks)
-          quantize_chunk(v[u], __ldcg(mask + (c >> 2)), 8 * c, a, rr, r, 0, word_prefix, qr,
+          quantize_chunk(v[u], __ldcg(mask + (c >> 2)), 8 * c, rr, r, 0, word_prefix, qr,
                          nullptr);
       }
     }
@@ -738,13 +715,13 @@ __global__ void __launch_bounds__(kRowThreads)
 #pragma unroll
   for (int d = 16; d > 0; d >>= 1) mbits = max(mbits, __shfl_xor_sync(0xFFFFFFFFu, mbits, d));
   const float a = half_bits_to_float(mbits);
-  const float r = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
+  const float r2 = row_code_scale(a);
   if (lane == 0) ax[row] = a;
   const int32_t n_out = (XO != nullptr) ? *count : 0;
   int8_t *qr = Xq + row * h;
   for (int32_t c = lane * 8; c < h; c += 256) {
     const uint4 v = __ldg(reinterpret_cast<const uint4 *>(xr + c));
-    quantize_chunk(v, __ldg(mask + (c >> 5)), c, a, r, row, n_out, word_prefix, qr, XO);
+    quantize_chunk(v, __ldg(mask + (c >> 5)), c, r2, row, n_out, word_prefix, qr, XO);
   }
 }
 
@@ -921,8 +898,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
   __syncthreads();
   if (c >= h) return;
   // codes of this chunk (outlier columns zeroed) and its fp16 outlier entries
-  const float r = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
-  uint2 q = quant8_fma(v, a, r);
+  uint2 q = quant8(v, row_code_scale(a));
   const uint32_t mk = (mw >> (c & 31)) & 0xFFu;
   if (mk) {
     const uint32_t keep_lo = ((mk & 0x1u) ? 0u : 0x000000FFu) | ((mk & 0x2u) ? 0u : 0x0000FF00u) |
@@ -999,13 +975,13 @@ __global__ void __launch_bounds__(kRowThreads)
   const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowsPerBlock + (threadIdx.x >> 5);
   if (row >= s) return;
   const float a = *scale;
-  const float r = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
+  const float r2 = row_code_scale(a);
   if (lane == 0) ax[row] = a;
   const uint16_t *xr = X + row * h;
   int8_t *qr = Xq + row * h;
   for (int32_t c = lane * 8; c < h; c += 256) {
     const uint4 v = __ldg(reinterpret_cast<const uint4 *>(xr + c));
-    quantize_chunk(v, __ldcg(mask + (c >> 5)), c, a, r, row, 0, word_prefix, qr, nullptr);
+    quantize_chunk(v, __ldcg(mask + (c >> 5)), c, r2, row, 0, word_prefix, qr, nullptr);
   }
 }
 
