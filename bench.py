@@ -25,7 +25,10 @@ are sampled with NVML as fast as it answers during the K timed steps; a
 second, longer window of the same steps (``clocks_soak``) repeats them for at
 least half a second. Multi-GPU (torchrun, or --gpus N, which launches it):
 independent replicas on every rank (the layer has no exchange step), time =
-max over ranks, value = total work of all ranks / that time.
+max over ranks, value = total work of all ranks / that time. With
+--parallel columns each rank instead owns a block of W's output columns
+(strong scaling: the layer's work is split, value = the whole layer's work /
+the slowest rank's time; the blocks need no exchange).
 
 --impl reference times the CPU oracle (plain C, OpenMP) on the host cores,
 on a bounded row sample of the same workload per step.
@@ -119,11 +122,17 @@ def needs_flush(wl) -> bool:
     return 2 * wl.s * wl.h + wl.h * wl.o <= 2 * L2_BYTES
 
 
+def parallelism(world: int, args) -> str:
+    if world <= 1:
+        return "single"
+    return f"{'column blocks' if args.parallel == 'columns' else 'replicas'} x{world}"
+
+
 def workload_config(wl, world: int, args) -> dict:
     """The line's `config`: the same keys and values in both arms."""
     return {"workload": wl.name, "s": wl.s, "h": wl.h, "o": wl.o,
             "alpha": alpha_json(wl.alpha), "outlier_cols": wl.n_outlier_cols,
-            "parallelism": f"replicas x{world}" if world > 1 else "single",
+            "parallelism": parallelism(world, args),
             "scales": {"x": args.x_scale, "w": args.w_scale},
             "l2": l2_policy(wl)}
 
@@ -355,15 +364,20 @@ def bench_workload(name, args, world, rank, local, K, Wm, headline: bool):
     are the line's top-level keys)."""
     import torch
     from mixed_precision_int8_b200 import binding
+    from mixed_precision_int8_b200.column_parallel import shard_columns
 
     dev = torch.device("cuda", local)
     wl, X, cols, W = workloads.make_inputs(name)
     wl = with_alpha(wl, args)
-    s, h, o = wl.s, wl.h, wl.o
+    s, h, o_layer = wl.s, wl.h, wl.o
+    columns = args.parallel == "columns" and world > 1
+    col0, o = shard_columns(o_layer, world, rank) if columns else (0, o_layer)
+    if o == 0:
+        raise SystemExit(f"rank {rank} has no columns of {o_layer} at world {world}")
     Xd = torch.from_numpy(X).to(dev)
     Wd = torch.from_numpy(W).to(dev)
     x_mode = SCALE_MODES[args.x_scale]
-    pw = binding.llmint8_prepare_weight(Wd, w_scale=SCALE_MODES[args.w_scale])
+    pw = binding.llmint8_prepare_weight_cols(Wd, col0, o, w_scale=SCALE_MODES[args.w_scale])
     torch.cuda.synchronize()
     del Wd
     out = torch.empty((s, o), dtype=torch.float16, device=dev)
@@ -463,11 +477,14 @@ def bench_workload(name, args, world, rank, local, K, Wm, headline: bool):
         barrier(world)
         e2e_ms = max_over_ranks(sum(e_ms) / n_steps, world, dev)
         del wsh, Xh, outh
-    fp16_ms = None if args.no_fp16_ref else fp16_matmul_ms(X, W, dev, flush, n_steps, Wm, world)
+    fp16_ms = None if args.no_fp16_ref else fp16_matmul_ms(
+        X, np.ascontiguousarray(W[:, col0:col0 + o]), dev, flush, n_steps, Wm, world)
 
-    ops = 2.0 * s * h * o
-    value = world * ops / (ms_per_step * 1e-3) / 1e12
-    e2e_value = None if e2e_ms is None else world * ops / (e2e_ms * 1e-3) / 1e12
+    ops = 2.0 * s * h * o  # this rank's
+    # whole-job work: every replica's layer, or the one layer split in blocks
+    job_ops = 2.0 * s * h * o_layer * (1 if columns else world)
+    value = job_ops / (ms_per_step * 1e-3) / 1e12
+    e2e_value = None if e2e_ms is None else job_ops / (e2e_ms * 1e-3) / 1e12
     peaks = measured_peaks()
     decode = s <= binding.llmint8_decode_max_rows()
     if decode:
@@ -495,8 +512,10 @@ def bench_workload(name, args, world, rank, local, K, Wm, headline: bool):
     roof["kernel_clocks"] = kernel_clocks
     entry = {
         "workload": wl.name, "value": value, "unit": UNIT,
+        "scaling": "strong" if columns else "weak",
         "ms_per_step": ms_per_step, "steps": n_steps,
-        "step_roofline_frac": layer_roofline_ms(wl, peaks) / ms_per_step,
+        # the roofline of this rank's share of the layer
+        "step_roofline_frac": layer_roofline_ms(dataclasses.replace(wl, o=o), peaks) / ms_per_step,
         "config": workload_config(wl, world, args),
         "e2e": None if e2e_value is None else {
             "value": e2e_value, "unit": UNIT,
@@ -515,7 +534,7 @@ def bench_workload(name, args, world, rank, local, K, Wm, headline: bool):
         soak = clocks.summary(soak_t0, soak_t1) if clocks else {}
         soak = dict(soak or {})
         soak["ms_per_step"] = sum(soak_ms) / len(soak_ms)
-        soak["value"] = world * ops / (soak["ms_per_step"] * 1e-3) / 1e12
+        soak["value"] = job_ops / (soak["ms_per_step"] * 1e-3) / 1e12
         soak["steps"] = len(soak_ms)
         soak["what"] = ("the same steps back to back for at least "
                         f"{SOAK_MIN_S} s after the timed ones (sustained load; "
@@ -547,7 +566,7 @@ def run_ours(args, world, rank, local):
     line = {
         "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world,
         "steps": K, "warmup": Wm, "ms_per_step": head["ms_per_step"],
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "higher_is_better": True, "scaling": head["scaling"], "vs_baseline": None,
         "dtype": "i8", "data": "synthetic (seeded, OPT-shaped outliers)",
         "config": head["config"], "e2e": head["e2e"],
         "gpu_launches": head["gpu_launches"], "roofline": head["roofline"],
@@ -625,6 +644,9 @@ def parse_args(argv=None):
                     help="skip the host-buffer end-to-end timing (profiling runs)")
     ap.add_argument("--max-outliers", type=int, default=0,
                     help="outlier columns the workspace holds (0: h, any alpha)")
+    ap.add_argument("--parallel", default="replicas", choices=["replicas", "columns"],
+                    help="N > 1: independent replicas (weak scaling) or one layer "
+                         "split into blocks of output columns (strong scaling)")
     ap.add_argument("--alpha", type=float, default=None,
                     help="outlier threshold instead of the workload's (inf: no "
                          "decomposition, pure vector-wise int8)")

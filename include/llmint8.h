@@ -224,6 +224,22 @@ LLMINT8_API llmint8_status llmint8_prepare_weight_ex(const uint16_t *W_dev, int6
                                          int64_t o, int32_t w_scale,
                                          llmint8_weight *out, void *stream);
 
+/* Column-parallel preparation ("LLM.int8(): 8-bit Matrix Multiplication for
+ * Transformers at Scale", Appendix D: a 175B-size layer spread over several
+ * GPUs): prepares columns [col0, col0 + o) of a weight W_dev [h][ldw] (row
+ * stride ldw elements) exactly as llmint8_prepare_weight prepares a weight
+ * made of those columns alone. Every column's scale and codes depend on
+ * that column only, so the shards of a layer, each on its own GPU, together
+ * hold the whole prepared weight, and each shard's llmint8_matmul output is
+ * that block of the layer's output columns, bit for bit. Rules: o as for
+ * llmint8_prepare_weight; ldw >= col0 + o; ldw and col0 multiples of 8 (so
+ * that W_dev + col0 is 16-byte aligned); out->o == o, out->h == h; w_scale
+ * as in llmint8_prepare_weight_ex. */
+LLMINT8_API llmint8_status llmint8_prepare_weight_cols(const uint16_t *W_dev, int64_t h,
+                                           int64_t ldw, int64_t col0, int64_t o,
+                                           int32_t w_scale, llmint8_weight *out,
+                                           void *stream);
+
 /* Steps 1 and 4 (activation side) on their own, for testing:
  *   flags_dev[j]  = 1 if column j is an outlier column, else 0   (u8 [h])
  *   idx_dev[0..n) = outlier columns in ascending order           (i32 [h])

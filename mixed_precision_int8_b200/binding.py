@@ -78,6 +78,8 @@ def load_library():
                                     ctypes.POINTER(llmint8_weight), _vp], _c_i32),
         "llmint8_prepare_weight_ex": ([_vp, _c_i64, _c_i64, _c_i32,
                                        ctypes.POINTER(llmint8_weight), _vp], _c_i32),
+        "llmint8_prepare_weight_cols": ([_vp, _c_i64, _c_i64, _c_i64, _c_i64, _c_i32,
+                                         ctypes.POINTER(llmint8_weight), _vp], _c_i32),
         "llmint8_quantize_rows_scratch_size": ([_c_i64], _sz),
         "llmint8_quantize_rows_ex": ([_vp, _c_i64, _c_i64, _c_f32, _c_i32, _vp,
                                       _vp, _vp, _vp, _vp, _vp, _sz, _vp], _c_i32),
@@ -122,7 +124,7 @@ EXPORTED = ("llmint8_status_string", "llmint8_workspace_size",
             "llmint8_prepare_weight_ex", "llmint8_quantize_rows_ex",
             "llmint8_matmul_host_ex", "llmint8_workspace_size_ex",
             "llmint8_workspace_size_host_ex", "llmint8_read_outlier_tiles_ex",
-            "llmint8_noalloc_read_device_status")
+            "llmint8_noalloc_read_device_status", "llmint8_prepare_weight_cols")
 
 
 def status_string(code: int) -> str:
@@ -226,6 +228,21 @@ def llmint8_prepare_weight(W: torch.Tensor, stream=None,
     pw = PreparedWeight(wq, aw, W if keep_fp16 else None)
     _check("llmint8_prepare_weight_ex", load_library().llmint8_prepare_weight_ex(
         _ptr(W), h, o, int(w_scale), ctypes.byref(pw.c), _stream(stream)))
+    return pw
+
+
+def llmint8_prepare_weight_cols(W: torch.Tensor, col0: int, o: int, stream=None,
+                                w_scale: int = SCALE_VECTORWISE) -> PreparedWeight:
+    """Columns [col0, col0 + o) of W fp16 [h, o_total] (on the GPU) prepared
+    as a weight of their own: one column-parallel shard."""
+    _f16_dev(W, "W")
+    h, ldw = W.shape
+    wq = torch.empty((o, h), dtype=torch.int8, device=W.device)
+    aw = torch.empty((o,), dtype=torch.float32, device=W.device)
+    pw = PreparedWeight(wq, aw, None)
+    _check("llmint8_prepare_weight_cols", load_library().llmint8_prepare_weight_cols(
+        _ptr(W), h, ldw, int(col0), int(o), int(w_scale), ctypes.byref(pw.c),
+        _stream(stream)))
     return pw
 
 

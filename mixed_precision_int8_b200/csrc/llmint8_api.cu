@@ -748,13 +748,22 @@ llmint8_status llmint8_prepare_weight(const uint16_t *W_dev, int64_t h, int64_t 
 
 llmint8_status llmint8_prepare_weight_ex(const uint16_t *W_dev, int64_t h, int64_t o,
                                          int32_t w_scale, llmint8_weight *out, void *stream) {
+  return llmint8_prepare_weight_cols(W_dev, h, o, 0, o, w_scale, out, stream);
+}
+
+llmint8_status llmint8_prepare_weight_cols(const uint16_t *W_dev, int64_t h, int64_t ldw,
+                                           int64_t col0, int64_t o, int32_t w_scale,
+                                           llmint8_weight *out, void *stream) {
   if (w_scale != LLMINT8_SCALE_VECTORWISE && w_scale != LLMINT8_SCALE_TENSORWISE)
     return LLMINT8_ERR_ARG;
   if (!W_dev || !out || !out->wq_dev || !out->aw_dev) return LLMINT8_ERR_NULL;
   llmint8_status rc = check_hw(h, o);
   if (rc) return rc;
+  if (col0 < 0 || ldw < o || col0 > ldw - o || (ldw % 8) != 0 || (col0 % 8) != 0)
+    return LLMINT8_ERR_SHAPE;
   if (out->h != h || out->o != o) return LLMINT8_ERR_SHAPE;
-  if (!aligned(W_dev, 16) || !aligned(out->wq_dev, 16) || !aligned(out->aw_dev, 16))
+  const uint16_t *W0 = W_dev + col0;
+  if (!aligned(W0, 16) || !aligned(out->wq_dev, 16) || !aligned(out->aw_dev, 16))
     return LLMINT8_ERR_ALIGN;
   DeviceInfo *dev = nullptr;
   if ((rc = device_info(&dev))) return rc;
@@ -767,11 +776,11 @@ llmint8_status llmint8_prepare_weight_ex(const uint16_t *W_dev, int64_t h, int64
   int64_t rpb = (h + gy_target - 1) / gy_target;
   if (rpb < 8) rpb = 8;
   const int gy = (int)((h + rpb - 1) / rpb);
-  k_weight_colmax<<<dim3(gx, gy), 256, 0, st>>>(W_dev, hh, oo, (int32_t)rpb, awb);
+  k_weight_colmax<<<dim3(gx, gy), 256, 0, st>>>(W0, hh, oo, ldw, (int32_t)rpb, awb);
   if (w_scale == LLMINT8_SCALE_TENSORWISE) k_bits_to_tensor_max<<<1, 1024, 0, st>>>(awb, o);
   k_weight_codes<<<dim3((unsigned)((o + kWqTile - 1) / kWqTile),
                         (unsigned)((h + kWqTile - 1) / kWqTile)),
-                   256, 0, st>>>(W_dev, hh, oo, awb, out->wq_dev);
+                   256, 0, st>>>(W0, hh, oo, ldw, awb, out->wq_dev);
   k_widen_scales<<<(unsigned)((o + 255) / 256), 256, 0, st>>>(awb, oo);
   return last_launch();
 }

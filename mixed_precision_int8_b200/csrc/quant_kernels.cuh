@@ -1011,7 +1011,9 @@ __global__ void k_wait_selftest(int *__restrict__ status, const int *never_set,
 // ------------------------------------------------------------------- K0
 // Offline weight preparation. Column absmax as binary16 magnitude bits
 // (atomicMax over row blocks), then codes written transposed ([o][h]) through
-// a shared-memory tile, then the absmax bits widened to fp32 in place.
+// a shared-memory tile, then the absmax bits widened to fp32 in place. W is
+// read as [h][o] with row stride ldw >= o (a block of columns of a wider
+// weight, for column-parallel sharding).
 __global__ void k_zero_u32(uint32_t *__restrict__ p, int64_t n) {
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x)
@@ -1019,7 +1021,7 @@ __global__ void k_zero_u32(uint32_t *__restrict__ p, int64_t n) {
 }
 
 __global__ void __launch_bounds__(256)
-    k_weight_colmax(const uint16_t *__restrict__ W, int32_t h, int32_t o,
+    k_weight_colmax(const uint16_t *__restrict__ W, int32_t h, int32_t o, int64_t ldw,
                     int32_t rows_per_block, uint32_t *__restrict__ aw_bits) {
   const int32_t c = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
   if (c >= o) return;
@@ -1027,7 +1029,7 @@ __global__ void __launch_bounds__(256)
   const int32_t r1 = min(h, r0 + rows_per_block);
   uint32_t m[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   for (int32_t r = r0; r < r1; ++r) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(W + (int64_t)r * o + c));
+    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(W + (int64_t)r * ldw + c));
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -1043,7 +1045,7 @@ __global__ void __launch_bounds__(256)
 constexpr int kWqTile = 64;
 
 __global__ void __launch_bounds__(256)
-    k_weight_codes(const uint16_t *__restrict__ W, int32_t h, int32_t o,
+    k_weight_codes(const uint16_t *__restrict__ W, int32_t h, int32_t o, int64_t ldw,
                    const uint32_t *__restrict__ aw_bits, int8_t *__restrict__ wq) {
   __shared__ int8_t tile[kWqTile][kWqTile + 4];
   const int32_t k0 = blockIdx.y * kWqTile;
@@ -1055,7 +1057,7 @@ __global__ void __launch_bounds__(256)
     const int32_t k = k0 + kk, j = j0 + jj;
     int32_t q[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (k < h && j < o) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4 *>(W + (int64_t)k * o + j));
+      const uint4 v = __ldg(reinterpret_cast<const uint4 *>(W + (int64_t)k * ldw + j));
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
