@@ -27,6 +27,7 @@
 #include <cuda_fp16.h>
 
 #include "ptx_sm100.cuh"
+#include "outlier_rows.cuh"
 
 namespace llmint8 {
 namespace decode {
@@ -73,8 +74,9 @@ struct Params {
   const float *aw;
   const uint32_t *mask;   // outlier-column bitmask [ceil(h/32)]
   const int32_t *word_prefix;  // outlier columns before each mask word
-  const uint16_t *XO;     // [s][n_out] fp16
-  uint16_t *WO;           // [n_out][o] fp16, written here
+  const uint16_t *XO;     // outlier columns of X (layout: outlier_rows.cuh)
+  uint16_t *WO;           // outlier rows of W, written here (same layout rules)
+  int32_t ldk;            // row stride of the wide layout
   const uint16_t *w16;    // optional fp16 W [h][o]: WO rows are its own rows
   const int32_t *n_out;
   int32_t wo_cap;         // outlier rows the workspace holds; |O| above it:
@@ -320,15 +322,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const int r = lane + 32 * q;
                 const int64_t j = m_blk * BM + r;
                 if (j < p.o) {
+                  const int64_t dst = wo_index(rank, j, n_out, p.o, p.ldk);
                   if (p.w16) {  // the caller's fp16 row of W
-                    p.WO[(int64_t)rank * p.o + j] =
-                        __ldg(p.w16 + (int64_t)(k0 + cc) * p.o + j);
+                    p.WO[dst] = __ldg(p.w16 + (int64_t)(k0 + cc) * p.o + j);
                   } else {
                     const int8_t code = static_cast<int8_t>(
                         box[r * BOX_K + ((((cb >> 4) ^ (r & 7)) << 4) | (cb & 15))]);
                     const float prod = static_cast<float>(code) * aw_rows[q];
-                    p.WO[(int64_t)rank * p.o + j] =
-                        __half_as_ushort(__float2half_rn(__fdiv_rn(prod, 127.0f)));
+                    p.WO[dst] = __half_as_ushort(__float2half_rn(__fdiv_rn(prod, 127.0f)));
                   }
                 }
               }
@@ -371,7 +372,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int q = et; q < MAX_ROWS * 16; q += NUM_EPI_THREADS) {
       const int i = q / 16, t = q % 16;
       s_xo[i][t] = (i < p.s && t < nf)
-                       ? __half2float(__ushort_as_half(__ldg(p.XO + (int64_t)i * n_out + t)))
+                       ? __half2float(__ushort_as_half(__ldg(p.XO + xo_index(i, t, n_out, p.ldk))))
                        : 0.0f;
       if (t == 0) s_rs[i] = i < p.s ? __ldg(p.ax + i) * (1.0f / 16129.0f) : 0.0f;
     }
@@ -429,7 +430,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         float wo[16];
 #pragma unroll
         for (int t = 0; t < 16; ++t)
-          wo[t] = (t < nf) ? __half2float(__ushort_as_half(__ldcg(p.WO + (int64_t)t * p.o + j)))
+          wo[t] = (t < nf) ? __half2float(__ushort_as_half(
+                                 __ldcg(p.WO + wo_index(t, j, n_out, p.o, p.ldk))))
                            : 0.0f;
         int32_t cv[MAX_ROWS];
 #pragma unroll
@@ -443,8 +445,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int t = 0; t < 16; ++t) acc_f = fmaf(s_xo[i][t], wo[t], acc_f);
             for (int32_t t = 16; t < n_out; ++t)
               acc_f = fmaf(
-                  __half2float(__ushort_as_half(__ldcg(p.XO + (int64_t)i * n_out + t))),
-                  __half2float(__ushort_as_half(__ldcg(p.WO + (int64_t)t * p.o + j))), acc_f);
+                  __half2float(__ushort_as_half(__ldcg(p.XO + xo_index(i, t, n_out, p.ldk)))),
+                  __half2float(__ushort_as_half(__ldcg(p.WO + wo_index(t, j, n_out, p.o, p.ldk)))),
+                  acc_f);
             p.out[(int64_t)i * p.o + j] = __half_as_ushort(__float2half_rn(acc_f));
             if (p.ci) p.ci[(int64_t)i * p.o + j] = cv[i];
           }

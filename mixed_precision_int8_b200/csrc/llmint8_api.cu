@@ -11,6 +11,7 @@
 #include <cstring>
 #include <mutex>
 #include <utility>
+#include <vector>
 
 #include "llmint8.h"
 #include "quant_kernels.cuh"
@@ -140,8 +141,14 @@ int32_t mask_words(int64_t h) { return (int32_t)((h + 31) / 32); }
 constexpr size_t kStateBytes = 256 + ((4 * (size_t)((kMaxH + 31) / 32) + 255) & ~size_t(255));
 static_assert(kStateBytes == LLMINT8_WORKSPACE_STATE_BYTES, "state block size");
 
+// Row stride of the wide outlier layout (more than 16 outlier columns, K-major
+// for the tensor cores, outlier_rows.cuh): the capacity rounded up to 64, or
+// 0 when the capacity admits only the narrow layout.
+int64_t wide_ld(int64_t cap) { return cap > kNarrowOutliers ? (cap + 63) / 64 * 64 : 0; }
+
 // `cap` = outlier columns the XO / WO tiles hold (h for any alpha).
 Layout layout_for(int64_t s, int64_t h, int64_t o, int64_t cap) {
+  const int64_t kcap = std::max(cap, wide_ld(cap));
   Layout L;
   size_t off = 0;
   L.status = off;  off = align256(off + 256);
@@ -153,8 +160,8 @@ Layout layout_for(int64_t s, int64_t h, int64_t o, int64_t cap) {
   L.xq = off;      off = align256(off + (size_t)s * h);
   L.tiles = off;   off = align256(off + 4 * (size_t)((o + decode::BM - 1) / decode::BM));
   L.cacc = off;    off = align256(off + 4 * (size_t)kDecodeMaxRows * o);
-  L.xo = off;      off = align256(off + 2 * (size_t)s * cap);
-  L.wo = off;      off = align256(off + 2 * (size_t)cap * o);
+  L.xo = off;      off = align256(off + 2 * (size_t)s * kcap);
+  L.wo = off;      off = align256(off + 2 * (size_t)kcap * o);
   L.end = off;
   L.xstage = off;  off = align256(off + 2 * (size_t)s * h);
   L.ostage = off;  off = align256(off + 2 * (size_t)s * o);
@@ -258,6 +265,7 @@ struct ActivationArgs {
   int64_t o;
   uint16_t *WO;  // fp16 outlier rows of W, built here for |O| > 16 (or null)
   int32_t cap;   // outlier columns XO and WO hold
+  int32_t ldk;   // row stride of the wide outlier layout
   int32_t *zero_buf;
   int64_t zero_n;
   int *status;  // device status bits
@@ -361,6 +369,7 @@ llmint8_status enqueue_activation_fused(const DeviceInfo &dev, const ActivationA
     f.ax = a.ax;
     f.XO = a.XO;
     f.cap = a.cap;
+    f.ldk = a.ldk;
     f.row_blocks = fix_blocks;
     f.wq = a.wq;
     f.aw = a.aw;
@@ -435,7 +444,7 @@ llmint8_status enqueue_activation_pass(const DeviceInfo &dev, const ActivationAr
   if (rb > 0) {
     e = launch(k_rows_any, dim3((unsigned)rb), dim3(kRowThreads), 0, st, true, a.X, a.s, hh,
                (const uint32_t *)a.mask, (const int32_t *)a.wprefix, (const int32_t *)a.count,
-               a.Xq, a.ax, a.XO, a.cap, a.status);
+               a.Xq, a.ax, a.XO, a.cap, a.ldk, a.status);
     if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
     *launches += 1;
   }
@@ -443,7 +452,7 @@ llmint8_status enqueue_activation_pass(const DeviceInfo &dev, const ActivationAr
     // fp16 outlier rows of W (returns at once without outlier columns)
     e = launch(k_build_wo, dim3((unsigned)(2 * dev.sm_count)), dim3(256), 0, st, true,
                (const int32_t *)a.count, (const int32_t *)a.idx, a.wq, a.aw, a.w16, hh,
-               (int32_t)a.o, a.WO, a.cap);
+               (int32_t)a.o, a.ldk, a.WO, a.cap);
     if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
     *launches += 1;
   }
@@ -515,6 +524,7 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
   if (opts && opts->ci_dev && !aligned(opts->ci_dev, 16)) return LLMINT8_ERR_ALIGN;
   const int64_t h = w->h, o = w->o;
   const int64_t cap = outlier_cap(opts, h);
+  const int64_t ldk = wide_ld(cap);
   int32_t *status_host = opts ? opts->status_host : nullptr;
   const Layout L = layout_for(s, h, o, cap);
   if (ws_bytes < (host_layout ? L.end_host : L.end)) return LLMINT8_ERR_WORKSPACE;
@@ -536,7 +546,7 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
   const bool use_decode = (path == 2) || (path == 0 && s <= kDecodeMaxRows);
 
   // Tensor maps first: a failure here must leave nothing enqueued.
-  CUtensorMap tmA, tmB, tmOut;
+  CUtensorMap tmA, tmB, tmOut, tmXO, tmWO;
   if (use_decode) {
     // A = Wq tiles (rows of o), B = Xq rows (s <= 16, zero-filled to 16)
     if (!make_tmap_i8(&tmA, w->wq_dev, (uint64_t)h, (uint64_t)o, decode::BOX_K, decode::BM) ||
@@ -547,6 +557,15 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
         !make_tmap_i8(&tmB, w->wq_dev, (uint64_t)h, (uint64_t)o, gemm::BK, gemm::BN) ||
         !make_tmap_f16(&tmOut, out, (uint64_t)o, (uint64_t)s, gemm::OUT_BOX_COLS, 32))
       return LLMINT8_ERR_CUDA;
+    // the wide outlier tiles for the tensor cores (used only when |O| > 16)
+    if (ldk > 0) {
+      if (!make_tmap_f16(&tmXO, xo, (uint64_t)ldk, (uint64_t)s, gemm::OK, gemm::BM) ||
+          !make_tmap_f16(&tmWO, wo, (uint64_t)ldk, (uint64_t)o, gemm::OK, gemm::BN))
+        return LLMINT8_ERR_CUDA;
+    } else {
+      tmXO = tmA;
+      tmWO = tmB;
+    }
   }
 
   int32_t launches = 0;
@@ -573,6 +592,7 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
   act.w16 = w->w16_dev;
   act.o = o;
   act.cap = (int32_t)cap;
+  act.ldk = (int32_t)ldk;
   // prefill: the GEMM's CTAs build the fp16 outlier rows of W themselves
   // while their first mainloops run (unless gemm_plain asks for them from
   // the activation kernels); decode: the W^O gather and the finishing step
@@ -604,7 +624,7 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
     e0 = launch(k_decode_rowpass, dim3((unsigned)col_blocks, (unsigned)s), dim3(kDecodeThreads), 0,
                 st, true,
                 X, (int32_t)s, (int32_t)h, (const uint32_t *)mask, (const uint32_t *)partial,
-                col_blocks, wprefix, count, ax, xq, xo, (int32_t)cap, status);
+                col_blocks, wprefix, count, ax, xq, xo, (int32_t)cap, (int32_t)ldk, status);
     if (e0 != cudaSuccess) return LLMINT8_ERR_CUDA;
     launches += 2;
   } else if ((rc = enqueue_activation_pass(*dev, act, st, &launches))) {
@@ -630,6 +650,7 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
     p.word_prefix = wprefix;
     p.XO = xo;
     p.WO = wo;
+    p.ldk = (int32_t)ldk;
     p.w16 = w->w16_dev;
     p.n_out = count;
     p.wo_cap = (int32_t)cap;
@@ -663,6 +684,7 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
     p.aw = w->aw_dev;
     p.XO = xo;
     p.WO = wo;
+    p.ldk = (int32_t)ldk;
     p.wq = w->wq_dev;
     p.w16 = w->w16_dev;
     p.idx = idx;
@@ -679,7 +701,7 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
     p.build_wo = gemm_builds_wo ? 1 : 0;
     p.wo_wait_ns = wo_build == LLMINT8_WO_EACH_CTA ? 0 : kWoWaitNs;
     e = launch(gemm::k_gemm_i8_fused, dim3(grid), dim3(gemm::NUM_THREADS), gemm::SMEM_BYTES, st,
-               !timed, tmA, tmB, tmOut, p);
+               !timed, tmA, tmB, tmOut, tmXO, tmWO, p);
     if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
     if (opts && opts->gemm_event_stop)
       cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->gemm_event_stop), st);
@@ -924,16 +946,36 @@ llmint8_status llmint8_read_outlier_tiles_ex(const void *ws_dev, size_t ws_bytes
     return LLMINT8_ERR_CUDA;
   if (n < 0 || n > h) return LLMINT8_ERR_DEVICE_STATUS;
   *n_out_host = n;
-  if (n > cap) return LLMINT8_OK;  // the call kept no outlier tiles
-  if (XO_host && n > 0 &&
-      cudaMemcpyAsync(XO_host, wsb + L.xo, 2 * (size_t)s * n, cudaMemcpyDeviceToHost, st) !=
-          cudaSuccess)
+  if (n > cap || n == 0) return LLMINT8_OK;  // no outlier tiles kept
+  if (!outliers_wide(n)) {  // narrow: XO [s][n], WO [n][o]
+    if (XO_host &&
+        cudaMemcpyAsync(XO_host, wsb + L.xo, 2 * (size_t)s * n, cudaMemcpyDeviceToHost, st) !=
+            cudaSuccess)
+      return LLMINT8_ERR_CUDA;
+    if (WO_host &&
+        cudaMemcpyAsync(WO_host, wsb + L.wo, 2 * (size_t)n * o, cudaMemcpyDeviceToHost, st) !=
+            cudaSuccess)
+      return LLMINT8_ERR_CUDA;
+    return cudaStreamSynchronize(st) == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA;
+  }
+  // wide: XO [s][ldk] and WO [o][ldk], copied to [s][n] and (transposed) [n][o]
+  const int64_t ldk = wide_ld(cap);
+  if (XO_host && s > 0 &&
+      cudaMemcpy2DAsync(XO_host, 2 * (size_t)n, wsb + L.xo, 2 * (size_t)ldk, 2 * (size_t)n,
+                        (size_t)s, cudaMemcpyDeviceToHost, st) != cudaSuccess)
     return LLMINT8_ERR_CUDA;
-  if (WO_host && n > 0 &&
-      cudaMemcpyAsync(WO_host, wsb + L.wo, 2 * (size_t)n * o, cudaMemcpyDeviceToHost, st) !=
-          cudaSuccess)
-    return LLMINT8_ERR_CUDA;
-  return cudaStreamSynchronize(st) == cudaSuccess ? LLMINT8_OK : LLMINT8_ERR_CUDA;
+  std::vector<uint16_t> wot;
+  if (WO_host) {
+    wot.resize((size_t)o * n);
+    if (cudaMemcpy2DAsync(wot.data(), 2 * (size_t)n, wsb + L.wo, 2 * (size_t)ldk,
+                          2 * (size_t)n, (size_t)o, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+      return LLMINT8_ERR_CUDA;
+  }
+  if (cudaStreamSynchronize(st) != cudaSuccess) return LLMINT8_ERR_CUDA;
+  if (WO_host)
+    for (int64_t j = 0; j < o; ++j)
+      for (int64_t t = 0; t < n; ++t) WO_host[t * o + j] = wot[(size_t)j * n + t];
+  return LLMINT8_OK;
 }
 
 llmint8_status llmint8_read_device_status(void *ws_dev, size_t ws_bytes, int32_t *bits_out,

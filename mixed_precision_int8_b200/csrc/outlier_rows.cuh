@@ -1,8 +1,17 @@
-// The fp16 outlier rows of W (Step 2 of "The Full LLM.int8() Algorithm",
-// W side), shared by the kernels that build them: the int8 GEMM's epilogue
-// (while its first tiles' mainloops run) and, where the GEMM cannot be
-// launched so that all its CTAs are resident together, blocks of the
-// activation fix-up.
+// The fp16 outlier tiles of Step 2 of "The Full LLM.int8() Algorithm": the
+// outlier columns of X (XO) and the matching rows of W (WO), their layout in
+// the workspace, and the builder of WO shared by the kernels that make it.
+//
+// The layout is decided by |O| alone, so every kernel of a call, and the
+// read-back, agree on it without the host knowing |O|:
+//   narrow, |O| <= kNarrowOutliers: XO [s][|O|] and WO [|O|][o] (a row of WO
+//     per outlier column; the GEMM stages them in shared memory and sums
+//     the products on CUDA cores);
+//   wide, |O| > kNarrowOutliers: XO [s][ldk] and WO [o][ldk], both with the
+//     outlier index contiguous (K-major) and zero from |O| up to the next
+//     multiple of 64, so that the GEMM streams them through TMA into the
+//     tensor cores as a second product (fp16 x fp16 -> fp32).
+// ldk is the workspace's outlier capacity rounded up to a multiple of 64.
 #pragma once
 
 #include <cstdint>
@@ -10,32 +19,99 @@
 
 namespace llmint8 {
 
+constexpr int kNarrowOutliers = 16;
+
+__host__ __device__ __forceinline__ bool outliers_wide(int32_t n) { return n > kNarrowOutliers; }
+__host__ __device__ __forceinline__ int32_t pad64(int32_t n) { return (n + 63) & ~63; }
+
+// Element (row, t) of XO and (t, j) of WO.
+__device__ __forceinline__ int64_t xo_index(int64_t row, int32_t t, int32_t n, int32_t ldk) {
+  return row * (outliers_wide(n) ? ldk : n) + t;
+}
+__device__ __forceinline__ int64_t wo_index(int32_t t, int64_t j, int32_t n, int32_t o,
+                                            int32_t ldk) {
+  return outliers_wide(n) ? j * ldk + t : static_cast<int64_t>(t) * o + j;
+}
+
 // Step 2, W side, for every outlier column: WO[t][j] = fp16(fp32(fp32(
 // wq[j][O_t]) * aw[j]) / 127), or W[O_t][j] itself when the caller's fp16
-// weight w16 is given. Pairs (t, j) (j fastest, so the stores coalesce) from
-// `first` in steps of `stride`, eight independent gathers in flight per
-// thread.
-__device__ __forceinline__ void build_wo_rows(int32_t n, const int32_t *__restrict__ idx,
+// weight w16 is given, in the layout above (wide: also the zero padding).
+// Work items q from `first` in steps of `stride`, eight independent gathers
+// in flight per thread; narrow: q = t*o + j (j fastest, stores coalesce),
+// wide: q = j*pad64(n) + t (t fastest, stores coalesce). Out of line: it
+// runs once per thread and block, and inlined it would be compiled into the
+// GEMM epilogue's hot loop.
+__device__ __noinline__ void build_wo_rows(int32_t n, const int32_t *__restrict__ idx,
                                               const int8_t *__restrict__ wq,
                                               const float *__restrict__ aw,
                                               const uint16_t *__restrict__ w16, int32_t h,
-                                              int32_t o, uint16_t *__restrict__ WO,
-                                              int64_t first, int64_t stride) {
+                                              int32_t o, int32_t ldk,
+                                              uint16_t *__restrict__ WO, int64_t first,
+                                              int64_t stride) {
   constexpr int U = 8;
-  const int64_t pairs = static_cast<int64_t>(n) * o;
-  for (int64_t q0 = first; q0 < pairs; q0 += U * stride) {
-    int32_t code[U];
+  const bool wide = outliers_wide(n);
+  if (!wide) {
+    // narrow: q = t*o + j, at most 16 rows of o, one division per item
+    const int64_t pairs = static_cast<int64_t>(n) * o;
+    for (int64_t q0 = first; q0 < pairs; q0 += U * stride) {
+      int32_t code[U];
+      float scale[U];
+      uint16_t w[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int64_t q = q0 + u * stride;
+        code[u] = 0;
+        scale[u] = 0.0f;
+        w[u] = 0;
+        if (q < pairs) {
+          const int32_t t = static_cast<int32_t>(q / o);
+          const int32_t j = static_cast<int32_t>(q - static_cast<int64_t>(t) * o);
+          const int32_t c = __ldcg(idx + t);
+          if (w16 != nullptr) {
+            w[u] = __ldg(w16 + static_cast<int64_t>(c) * o + j);
+          } else {
+            code[u] = __ldg(wq + static_cast<int64_t>(j) * h + c);
+            scale[u] = __ldg(aw + j);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int64_t q = q0 + u * stride;
+        if (q < pairs)
+          WO[q] = w16 != nullptr
+                      ? w[u]
+                      : __half_as_ushort(__float2half_rn(
+                            __fdiv_rn(static_cast<float>(code[u]) * scale[u], 127.0f)));
+      }
+    }
+    return;
+  }
+  // wide: many items per thread; (group, offset) stepped without a division
+  const int32_t per = pad64(n);  // items per group (row of the q order)
+  const int64_t groups = o;
+  // each item's group and offset, stepped without a division per item
+  int64_t g0 = first / per;
+  int32_t r0 = static_cast<int32_t>(first - g0 * per);
+  const int64_t sg = stride / per;
+  const int32_t sr = static_cast<int32_t>(stride - sg * per);
+  while (g0 < groups) {
+    int32_t code[U], rr[U];
+    int64_t gg[U];
     float scale[U];
     uint16_t w[U];
+    bool live[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int64_t q = q0 + u * stride;
+      gg[u] = g0;
+      rr[u] = r0;
+      const int32_t t = r0;
+      const int32_t j = static_cast<int32_t>(g0);
       code[u] = 0;
       scale[u] = 0.0f;
       w[u] = 0;
-      if (q < pairs) {
-        const int32_t t = static_cast<int32_t>(q / o);
-        const int32_t j = static_cast<int32_t>(q - static_cast<int64_t>(t) * o);
+      live[u] = g0 < groups && t < n;
+      if (live[u]) {
         const int32_t c = __ldcg(idx + t);
         if (w16 != nullptr) {
           w[u] = __ldg(w16 + static_cast<int64_t>(c) * o + j);
@@ -44,14 +120,23 @@ __device__ __forceinline__ void build_wo_rows(int32_t n, const int32_t *__restri
           scale[u] = __ldg(aw + j);
         }
       }
+      g0 += sg;
+      r0 += sr;
+      if (r0 >= per) {
+        r0 -= per;
+        ++g0;
+      }
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int64_t q = q0 + u * stride;
-      if (q < pairs)
-        WO[q] = w16 != nullptr ? w[u]
-                               : __half_as_ushort(__float2half_rn(
-                                     __fdiv_rn(static_cast<float>(code[u]) * scale[u], 127.0f)));
+      if (gg[u] < groups) {
+        const int64_t dst = gg[u] * ldk + rr[u];
+        WO[dst] = !live[u] ? static_cast<uint16_t>(0)
+                  : w16 != nullptr
+                      ? w[u]
+                      : __half_as_ushort(__float2half_rn(
+                            __fdiv_rn(static_cast<float>(code[u]) * scale[u], 127.0f)));
+      }
     }
   }
 }

@@ -355,7 +355,7 @@ __device__ __forceinline__ uint2 quant8(const uint4 v, float r2) {
 // fp16 values of the chunk's outlier columns written to XO[row][rank].
 __device__ __forceinline__ void quantize_chunk(const uint4 v, uint32_t mw, int32_t c,
                                                float r2, int64_t row, int32_t n_out,
-                                               const int32_t *word_prefix,
+                                               int32_t ldk, const int32_t *word_prefix,
                                                int8_t *__restrict__ qr,
                                                uint16_t *__restrict__ XO) {
   const uint32_t mk = (mw >> (c & 31)) & 0xFFu;
@@ -373,7 +373,8 @@ __device__ __forceinline__ void quantize_chunk(const uint4 v, uint32_t mw, int32
       for (int e = 0; e < 8; ++e) {
         if ((mk >> e) & 1u) {
           const uint32_t hv = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
-          XO[row * n_out + outlier_rank(word_prefix, mw, c, e)] = static_cast<uint16_t>(hv);
+          XO[xo_index(row, outlier_rank(word_prefix, mw, c, e), n_out, ldk)] =
+              static_cast<uint16_t>(hv);
         }
       }
     }
@@ -526,13 +527,13 @@ __global__ void __launch_bounds__(kActMaxWarps * 32) k_act_rows(const ActRowsPar
 __global__ void __launch_bounds__(256)
     k_build_wo(const int32_t *__restrict__ count, const int32_t *__restrict__ idx,
                const int8_t *__restrict__ wq, const float *__restrict__ aw,
-               const uint16_t *__restrict__ w16, int32_t h, int32_t o,
+               const uint16_t *__restrict__ w16, int32_t h, int32_t o, int32_t ldk,
                uint16_t *__restrict__ WO, int32_t cap) {
   grid_dependency_wait();
   grid_dependency_trigger();
   const int32_t n = __ldcg(count);
   if (n == 0 || n > cap) return;
-  build_wo_rows(n, idx, wq, aw, w16, h, o, WO,
+  build_wo_rows(n, idx, wq, aw, w16, h, o, ldk, WO,
                 static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x,
                 static_cast<int64_t>(gridDim.x) * blockDim.x);
 }
@@ -562,8 +563,9 @@ struct FixupParams {
   const int32_t *count;
   int8_t *Xq;
   float *ax;
-  uint16_t *XO;  // [s][|O|] or null
+  uint16_t *XO;  // the outlier columns of X (layout: outlier_rows.cuh) or null
   int32_t cap;   // outlier columns XO and WO hold
+  int32_t ldk;   // row stride of the wide layout
   int64_t row_blocks;
   // fp16 outlier rows of W (WO null: not built here)
   const int8_t *wq;
@@ -599,7 +601,7 @@ __global__ void __launch_bounds__(kFixThreads) k_act_fixup(const FixupParams p) 
   if (!fits && blockIdx.x == 0 && tid == 0) atomicOr(p.status, LLMINT8_DEV_OUTLIER_CAP);
   if (blockIdx.x >= p.row_blocks) {  // uniform over the block
     if (fits && p.WO != nullptr)
-      build_wo_rows(n, idx, p.wq, p.aw, p.w16, h, p.o, p.WO,
+      build_wo_rows(n, idx, p.wq, p.aw, p.w16, h, p.o, p.ldk, p.WO,
                     static_cast<int64_t>(blockIdx.x - p.row_blocks) * kFixThreads + tid,
                     static_cast<int64_t>(gridDim.x - p.row_blocks) * kFixThreads);
     return;
@@ -614,19 +616,49 @@ __global__ void __launch_bounds__(kFixThreads) k_act_fixup(const FixupParams p) 
   if (row_ok) {
     const uint16_t *xr = X + row * h;
     uint32_t mo = 0;
-    for (int32_t t = lane; t < n; t += 32) {
-      const int32_t j = t < 32 ? j_pre : __ldcg(idx + t);
-      const uint32_t hv = xr[j];
-      if (XO) XO[row * n + t] = static_cast<uint16_t>(hv);
-      const uint32_t mag = hv & 0x7FFFu;
-      if (mag < thresh_bits) mo = max(mo, mag);
+    if (n <= 32) {  // at most one outlier column per lane
+      if (lane < n) {
+        const uint32_t hv = xr[j_pre];
+        if (XO) XO[xo_index(row, lane, n, p.ldk)] = static_cast<uint16_t>(hv);
+        const uint32_t mag = hv & 0x7FFFu;
+        if (mag < thresh_bits) mo = mag;
+      }
+    } else {
+    // four gathers in flight per lane (many outlier columns: up to h)
+    for (int32_t t0 = lane; t0 < n; t0 += 4 * 32) {
+      int32_t jj[4];
+      uint32_t hv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int32_t t = t0 + 32 * u;
+        jj[u] = t < 32 ? j_pre : (t < n ? __ldcg(idx + t) : 0);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) hv[u] = t0 + 32 * u < n ? xr[jj[u]] : 0u;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int32_t t = t0 + 32 * u;
+        if (t < n) {
+          if (XO) XO[xo_index(row, t, n, p.ldk)] = static_cast<uint16_t>(hv[u]);
+          const uint32_t mag = hv[u] & 0x7FFFu;
+          if (mag < thresh_bits) mo = max(mo, mag);
+        }
+      }
     }
+    }
+    if (XO && outliers_wide(n))  // zero padding of the wide layout
+      for (int32_t t = n + lane; t < pad64(n); t += 32) XO[row * p.ldk + t] = 0;
 #pragma unroll
     for (int d = 16; d > 0; d >>= 1) mo = max(mo, __shfl_xor_sync(0xFFFFFFFFu, mo, d));
     need = a0 > 0.0f && half_bits_to_float(mo) == a0;
     if (!need) {
       int8_t *qr = Xq + row * h;
-      for (int32_t t = lane; t < n; t += 32) qr[t < 32 ? j_pre : __ldcg(idx + t)] = 0;
+      if (n <= 32) {
+        if (lane < n) qr[j_pre] = 0;
+      } else {
+#pragma unroll 4
+        for (int32_t t = lane; t < n; t += 32) qr[t < 32 ? j_pre : __ldcg(idx + t)] = 0;
+      }
     }
   }
   if (lane == 0) redo[warp] = need ? 1 : 0;
@@ -676,7 +708,7 @@ __global__ void __launch_bounds__(kFixThreads) k_act_fixup(const FixupParams p) 
       for (int u = 0; u < 8; ++u) {
         const int32_t c = c0 + u * kFixThreads;
         if (c < nchunks)
-          quantize_chunk(v[u], __ldcg(mask + (c >> 2)), 8 * c, rr, r, 0, word_prefix, qr,
+          quantize_chunk(v[u], __ldcg(mask + (c >> 2)), 8 * c, rr, r, 0, 0, word_prefix, qr,
                          nullptr);
       }
     }
@@ -694,7 +726,7 @@ __global__ void __launch_bounds__(kRowThreads)
                const uint32_t *__restrict__ mask, const int32_t *__restrict__ word_prefix,
                const int32_t *__restrict__ count, int8_t *__restrict__ Xq,
                float *__restrict__ ax, uint16_t *__restrict__ XO, int32_t cap,
-               int *__restrict__ status) {
+               int32_t ldk, int *__restrict__ status) {
   grid_dependency_wait();
   grid_dependency_trigger();
   const int lane = threadIdx.x & 31;
@@ -721,8 +753,10 @@ __global__ void __launch_bounds__(kRowThreads)
   int8_t *qr = Xq + row * h;
   for (int32_t c = lane * 8; c < h; c += 256) {
     const uint4 v = __ldg(reinterpret_cast<const uint4 *>(xr + c));
-    quantize_chunk(v, __ldg(mask + (c >> 5)), c, r2, row, n_out, word_prefix, qr, XO);
+    quantize_chunk(v, __ldg(mask + (c >> 5)), c, r2, row, n_out, ldk, word_prefix, qr, XO);
   }
+  if (XO != nullptr && outliers_wide(n_out))  // zero padding of the wide layout
+    for (int32_t t = n_out + lane; t < pad64(n_out); t += 32) XO[row * ldk + t] = 0;
 }
 
 // ----------------------------------------------------- K1 for s <= 16
@@ -810,7 +844,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
                      int32_t col_blocks, int32_t *__restrict__ word_prefix,
                      int32_t *__restrict__ count, float *__restrict__ ax,
                      int8_t *__restrict__ Xq, uint16_t *__restrict__ XO, int32_t cap,
-                     int *__restrict__ status) {
+                     int32_t ldk, int *__restrict__ status) {
   __shared__ int32_t s_prefix[kDecodeColsPerBlock / 32];
   __shared__ int32_t red_before[kDecodeThreads / 32], red_total[kDecodeThreads / 32];
   __shared__ uint32_t red_max[kDecodeThreads / 32];
@@ -915,7 +949,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
     for (int e = 0; e < 8; ++e) {
       if ((mk >> e) & 1u) {
         const uint32_t hv = (e & 1) ? (w4[e >> 1] >> 16) : (w4[e >> 1] & 0xFFFFu);
-        XO[(int64_t)row * total + outlier_rank(pre_local, mw, c, e)] = static_cast<uint16_t>(hv);
+        XO[xo_index(row, outlier_rank(pre_local, mw, c, e), total, ldk)] =
+            static_cast<uint16_t>(hv);
       }
     }
   }
@@ -981,7 +1016,7 @@ __global__ void __launch_bounds__(kRowThreads)
   int8_t *qr = Xq + row * h;
   for (int32_t c = lane * 8; c < h; c += 256) {
     const uint4 v = __ldg(reinterpret_cast<const uint4 *>(xr + c));
-    quantize_chunk(v, __ldcg(mask + (c >> 5)), c, r2, row, 0, word_prefix, qr, nullptr);
+    quantize_chunk(v, __ldcg(mask + (c >> 5)), c, r2, row, 0, 0, word_prefix, qr, nullptr);
   }
 }
 

@@ -68,8 +68,9 @@ def test_workspace_size_formula(lib):
                     (3, 272, 784)]:
         nw = (h + 31) // 32
         state = 256 + a256(4 * ((133144 + 31) // 32))  # status + accumulation bitmask
+        kcap = max(h, (h + 63) // 64 * 64)  # outlier tiles: the wide layout's stride
         exp = (state + a256(4 * nw) + a256(4 * (nw + 1)) + a256(4 * h)
-               + a256(4 * s) + a256(s * h) + a256(2 * s * h) + a256(2 * h * o)
+               + a256(4 * s) + a256(s * h) + a256(2 * s * kcap) + a256(2 * kcap * o)
                + a256(4 * ((o + 127) // 128)) + a256(4 * 16 * o))
         assert lib.llmint8_workspace_size(s, h, o) == exp
         assert (lib.llmint8_workspace_size_host(s, h, o)
@@ -226,14 +227,19 @@ def test_workspace_with_an_outlier_cap_is_small_for_the_175b_shapes(lib):
     def a256(x):
         return (x + 255) // 256 * 256
 
-    for s, h, o in [(2048, 12288, 49152), (8, 12288, 49152), (16, 256, 256)]:
+    def kcap(cap):  # more than 16: the wide layout, stride rounded up to 64
+        return cap if cap <= 16 else (cap + 63) // 64 * 64
+
+    for s, h, o in [(2048, 12288, 49152), (8, 12288, 49152), (16, 256, 256), (40, 272, 784)]:
         full = lib.llmint8_workspace_size(s, h, o)
         assert lib.llmint8_workspace_size_ex(s, h, o, 0) == full
         assert lib.llmint8_workspace_size_ex(s, h, o, h) == full
-        for cap in (1, 16, 64):
+        for cap in (1, 16, 17, 64, 100):
+            if cap > h:
+                continue
             got = lib.llmint8_workspace_size_ex(s, h, o, cap)
-            assert got == full - a256(2 * s * h) - a256(2 * h * o) \
-                + a256(2 * s * cap) + a256(2 * cap * o)
+            assert got == full - a256(2 * s * kcap(h)) - a256(2 * kcap(h) * o) \
+                + a256(2 * s * kcap(cap)) + a256(2 * kcap(cap) * o)
             assert (lib.llmint8_workspace_size_host_ex(s, h, o, cap)
                     == got + a256(2 * s * h) + a256(2 * s * o))
     assert lib.llmint8_workspace_size(2048, 12288, 49152) > 1.2e9

@@ -486,3 +486,60 @@ def test_workload_matmul(name):
         # properties that hold for every output: finite, and rows with no
         # outlier entry and zero codes are exactly zero
         assert np.isfinite(out.astype(np.float32)).all()
+
+
+# More than 16 outlier columns: the outlier tiles take the wide (K-major,
+# zero-padded) layout and the prefill GEMM sums the fp16 outlier product on
+# the tensor cores (kind::f16 into a second TMEM accumulator); the decode
+# kernel reads the same layout on CUDA cores.
+WIDE_CASES = [
+    (300, 1024, 1024, tuple(range(5, 1024, 16)), 6.0),   # |O| = 64: one fp16 k-block
+    (129, 1040, 784, tuple(range(3, 1040, 13)), 6.0),    # |O| = 80: a partial k-block
+    (256, 512, 2048, (), 0.0),                           # every column out: |O| = 512
+    (8, 1024, 512, tuple(range(5, 1024, 16)), 6.0),      # |O| = 64, decode and prefill
+]
+
+
+@pytest.mark.parametrize("keep_fp16", [False, True], ids=["w_from_int8", "w_fp16"])
+@pytest.mark.parametrize("case", WIDE_CASES, ids=lambda c: f"{c[0]}x{c[1]}x{c[2]}a{c[4]}")
+def test_wide_outlier_sets_on_the_tensor_cores(case, keep_fp16):
+    X, W, alpha = _small_inputs(case, seed=23)
+    s = X.shape[0]
+    pw, _ = gpu_prepare(W, keep_fp16=keep_fp16)
+    Wq_ref, aw_ref = oracle.prepare_weight(W)
+    ref, ci_ref = oracle.matmul(X, Wq_ref, aw_ref, alpha, want_ci=True,
+                                W16=W if keep_fp16 else None)
+    f_ref, idx_ref, n_ref = oracle.detect_outliers(X, alpha)
+    assert n_ref > 16
+    WO_ref = (np.ascontiguousarray(W[idx_ref, :]) if keep_fp16
+              else oracle.outlier_weights(Wq_ref, aw_ref, idx_ref))
+    XO_ref = np.ascontiguousarray(X[:, idx_ref])
+    runs = [(1, m) for m in (binding.WO_SHARED, binding.WO_BEFORE_GEMM, binding.WO_EACH_CTA)]
+    if s <= 16:
+        runs.append((2, binding.WO_SHARED))
+    for path, mode in runs:
+        out, ci, ws = gpu_matmul(X, pw, alpha, path=path, want_ci=True, wo_build=mode)
+        assert np.array_equal(ci, ci_ref), f"int32 accumulators, path {path} mode {mode}"
+        assert_close_fp16(out, ref, f"out path {path} mode {mode}")
+        n, XO, WO = binding.llmint8_read_outlier_tiles(ws)
+        assert n == n_ref
+        assert np.array_equal(XO.numpy().view(np.uint16), XO_ref.view(np.uint16))
+        assert np.array_equal(WO.numpy().view(np.uint16), WO_ref.view(np.uint16))
+
+
+def test_every_column_an_outlier_at_the_6p7b_shape():
+    """alpha = 0 on the OPT-6.7B attention shape: |O| = h = 4096, so the
+    layer is the fp16 product X.W^O on the tensor cores (64 fp16 k-blocks
+    per tile) plus an all-zero int8 part; 64 sampled rows x every column."""
+    wl, X, cols, W = workloads.make_inputs("opt6.7b_attn_prefill")
+    pw, _ = gpu_prepare(W)
+    rows = sample_rows(wl.s, 64)
+    Wq_ref, aw_ref = oracle_prepared_by_blocks(W)
+    ref, ci_ref = oracle.matmul(X, Wq_ref, aw_ref, 0.0, rows=rows, want_ci=True)
+    assert not ci_ref.any()
+    out, ci, ws = gpu_matmul(X, pw, 0.0, want_ci=True)
+    assert not ci.any()
+    assert_close_fp16(out[rows], ref)
+    assert np.isfinite(out.astype(np.float32)).all()
+    del pw, ws
+    torch.cuda.empty_cache()
