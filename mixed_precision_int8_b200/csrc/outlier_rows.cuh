@@ -87,57 +87,54 @@ __device__ __noinline__ void build_wo_rows(int32_t n, const int32_t *__restrict_
     }
     return;
   }
-  // wide: many items per thread; (group, offset) stepped without a division
-  const int32_t per = pad64(n);  // items per group (row of the q order)
-  const int64_t groups = o;
-  // each item's group and offset, stepped without a division per item
-  int64_t g0 = first / per;
-  int32_t r0 = static_cast<int32_t>(first - g0 * per);
-  const int64_t sg = stride / per;
-  const int32_t sr = static_cast<int32_t>(stride - sg * per);
-  while (g0 < groups) {
-    int32_t code[U], rr[U];
-    int64_t gg[U];
-    float scale[U];
-    uint16_t w[U];
-    bool live[U];
+  // wide: the items are (t, j) with t < pad64(n) and j < o, stored at
+  // WO[j*ldk + t]. Each thread keeps one t (its index loaded once) and walks
+  // j; a warp covers 32 consecutive t of one row j, so the gathers from wq
+  // and the stores coalesce. With fewer threads than t values (a CTA
+  // building every row alone) each thread takes several t in turn.
+  const int32_t T = pad64(n);
+  constexpr int UW = 8;  // gathers in flight per thread
+  auto column = [&](int32_t t, int64_t jbeg, int64_t jstep) {
+    const bool tl = t < n;
+    const int32_t c = tl ? __ldcg(idx + t) : 0;
+    for (int64_t j0 = jbeg; j0 < o; j0 += UW * jstep) {
+      int32_t code[UW];
+      float scale[UW];
+      uint16_t w[UW];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      gg[u] = g0;
-      rr[u] = r0;
-      const int32_t t = r0;
-      const int32_t j = static_cast<int32_t>(g0);
-      code[u] = 0;
-      scale[u] = 0.0f;
-      w[u] = 0;
-      live[u] = g0 < groups && t < n;
-      if (live[u]) {
-        const int32_t c = __ldcg(idx + t);
-        if (w16 != nullptr) {
-          w[u] = __ldg(w16 + static_cast<int64_t>(c) * o + j);
-        } else {
-          code[u] = __ldg(wq + static_cast<int64_t>(j) * h + c);
-          scale[u] = __ldg(aw + j);
+      for (int u = 0; u < UW; ++u) {
+        const int64_t j = j0 + u * jstep;
+        code[u] = 0;
+        scale[u] = 0.0f;
+        w[u] = 0;
+        if (tl && j < o) {
+          if (w16 != nullptr) {
+            w[u] = __ldg(w16 + static_cast<int64_t>(c) * o + j);
+          } else {
+            code[u] = __ldg(wq + j * h + c);
+            scale[u] = __ldg(aw + j);
+          }
         }
       }
-      g0 += sg;
-      r0 += sr;
-      if (r0 >= per) {
-        r0 -= per;
-        ++g0;
-      }
-    }
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      if (gg[u] < groups) {
-        const int64_t dst = gg[u] * ldk + rr[u];
-        WO[dst] = !live[u] ? static_cast<uint16_t>(0)
-                  : w16 != nullptr
-                      ? w[u]
-                      : __half_as_ushort(__float2half_rn(
-                            __fdiv_rn(static_cast<float>(code[u]) * scale[u], 127.0f)));
+      for (int u = 0; u < UW; ++u) {
+        const int64_t j = j0 + u * jstep;
+        if (j < o)
+          WO[j * ldk + t] = !tl ? static_cast<uint16_t>(0)
+                            : w16 != nullptr
+                                ? w[u]
+                                : __half_as_ushort(__float2half_rn(
+                                      __fdiv_rn(static_cast<float>(code[u]) * scale[u], 127.0f)));
       }
     }
+  };
+  if (stride >= T) {
+    // thread `first` takes t = first % T and every jstep-th column j from
+    // first / T: each (t, j) exactly once over the first jstep*T threads
+    const int64_t jstep = stride / T;
+    if (first < jstep * T) column(static_cast<int32_t>(first % T), first / T, jstep);
+  } else {
+    for (int64_t t = first; t < T; t += stride) column(static_cast<int32_t>(t), 0, 1);
   }
 }
 

@@ -642,6 +642,9 @@ __global__ void __launch_bounds__(kFixThreads) k_act_fixup(const FixupParams p) 
           if (XO) XO[xo_index(row, t, n, p.ldk)] = static_cast<uint16_t>(hv[u]);
           const uint32_t mag = hv[u] & 0x7FFFu;
           if (mag < thresh_bits) mo = max(mo, mag);
+          // the outlier column's code (a row sent to recomputation below is
+          // requantised whole, outlier columns zero again)
+          Xq[row * h + jj[u]] = 0;
         }
       }
     }
@@ -653,12 +656,7 @@ __global__ void __launch_bounds__(kFixThreads) k_act_fixup(const FixupParams p) 
     need = a0 > 0.0f && half_bits_to_float(mo) == a0;
     if (!need) {
       int8_t *qr = Xq + row * h;
-      if (n <= 32) {
-        if (lane < n) qr[j_pre] = 0;
-      } else {
-#pragma unroll 4
-        for (int32_t t = lane; t < n; t += 32) qr[t < 32 ? j_pre : __ldcg(idx + t)] = 0;
-      }
+      if (n <= 32 && lane < n) qr[j_pre] = 0;  // more: zeroed in the gather loop
     }
   }
   if (lane == 0) redo[warp] = need ? 1 : 0;
