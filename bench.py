@@ -58,8 +58,11 @@ from mixed_precision_int8_b200 import workloads  # noqa: E402
 METRIC = "LLM.int8() matmul effective TOPS"
 UNIT = "TOPS"
 DEFAULT_WORKLOAD = "opt175b_ffn_up_prefill"
+# name@alpha: the workload with another outlier threshold (4.5: about 63
+# outlier columns on the 6.7B shape; 0: every column, the fp16 extreme)
 DEFAULT_PER_SHAPE = ("opt6.7b_attn_prefill", "opt13b_ffn_up_prefill",
-                     "opt175b_decode")
+                     "opt175b_decode", "opt6.7b_attn_prefill@4.5",
+                     "opt6.7b_attn_prefill@0")
 L2_BYTES = 126 << 20
 FLUSH_BYTES = 512 << 20
 # per-shape entries time at least this many steps (short bursts, like the
@@ -237,9 +240,16 @@ def fp16_matmul_ms(X, W, dev, flush, K, Wm, world):
     return max_over_ranks(ms, world, dev)
 
 
-def with_alpha(wl, args):
-    """The workload with --alpha in place of its threshold, if given."""
-    return wl if args.alpha is None else dataclasses.replace(wl, alpha=args.alpha)
+def with_alpha(wl, args, alpha=None):
+    """The workload with `alpha` (else --alpha) in place of its threshold."""
+    a = alpha if alpha is not None else args.alpha
+    return wl if a is None else dataclasses.replace(wl, alpha=a)
+
+
+def split_spec(spec: str):
+    """'name' or 'name@alpha' -> (name, alpha or None)."""
+    name, _, a = spec.partition("@")
+    return name, (float(a) if a else None)
 
 
 def alpha_json(a: float):
@@ -367,8 +377,9 @@ def bench_workload(name, args, world, rank, local, K, Wm, headline: bool):
     from mixed_precision_int8_b200.column_parallel import shard_columns
 
     dev = torch.device("cuda", local)
+    name, alpha_override = split_spec(name)
     wl, X, cols, W = workloads.make_inputs(name)
-    wl = with_alpha(wl, args)
+    wl = with_alpha(wl, args, alpha_override)
     s, h, o_layer = wl.s, wl.h, wl.o
     columns = args.parallel == "columns" and world > 1
     col0, o = shard_columns(o_layer, world, rank) if columns else (0, o_layer)
@@ -396,6 +407,7 @@ def bench_workload(name, args, world, rank, local, K, Wm, headline: bool):
         step()
     torch.cuda.synchronize()
     launches_per_step = binding.llmint8_matmul.last_launches
+    n_outliers, _, _ = binding.llmint8_read_outlier_tiles(ws, tiles=False)  # |O|
 
     def timed_steps(n, with_kernel_events: bool):
         """n steps, each between CUDA events on the launching stream (after
@@ -511,7 +523,8 @@ def bench_workload(name, args, world, rank, local, K, Wm, headline: bool):
                              "same steps right after the timed one")
     roof["kernel_clocks"] = kernel_clocks
     entry = {
-        "workload": wl.name, "value": value, "unit": UNIT,
+        "workload": wl.name if alpha_override is None else f"{wl.name}@alpha={alpha_override:g}",
+        "outliers": n_outliers, "value": value, "unit": UNIT,
         "scaling": "strong" if columns else "weak",
         "ms_per_step": ms_per_step, "steps": n_steps,
         # the roofline of this rank's share of the layer
@@ -660,7 +673,8 @@ def parse_args(argv=None):
     if args.gpus < 1:
         ap.error("--gpus must be >= 1")
     if args.per_shape not in (None, "none"):
-        bad = [n for n in args.per_shape.split(",") if n and n not in workloads.WORKLOADS]
+        bad = [n for n in args.per_shape.split(",")
+               if n and split_spec(n)[0] not in workloads.WORKLOADS]
         if bad:
             ap.error(f"unknown workloads in --per-shape: {bad}")
     return args

@@ -361,14 +361,19 @@ def llmint8_matmul_host(X_host: torch.Tensor, w: PreparedWeight,
 
 
 def llmint8_read_outlier_tiles(workspace: Workspace, s: Optional[int] = None,
-                               stream=None):
+                               stream=None, tiles: bool = True):
     """(n, XO [s,n] fp16, WO [n,o] fp16) of the last matmul on `workspace`,
     which had `s` rows (default: the row count the workspace was sized for;
-    the workspace layout depends on it)."""
+    the workspace layout depends on it). tiles=False reads |O| alone."""
     h, o = workspace.h, workspace.o
     s = workspace.s if s is None else int(s)
     cap = workspace.max_outliers or h
     n = ctypes.c_int32(0)
+    if not tiles:
+        _check("llmint8_read_outlier_tiles_ex", load_library().llmint8_read_outlier_tiles_ex(
+            _ptr(workspace.buf), workspace.nbytes, s, h, o, workspace.max_outliers,
+            ctypes.byref(n), None, None, _stream(stream)))
+        return n.value, None, None
     XO = torch.empty((s * cap,), dtype=torch.float16)
     WO = torch.empty((cap * o,), dtype=torch.float16)
     _check("llmint8_read_outlier_tiles_ex", load_library().llmint8_read_outlier_tiles_ex(
