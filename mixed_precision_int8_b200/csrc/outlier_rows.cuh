@@ -17,12 +17,24 @@
 #include <cstdint>
 #include <cuda_fp16.h>
 
+#include "ptx_sm100.cuh"
+
 namespace llmint8 {
 
 constexpr int kNarrowOutliers = 16;
 
 __host__ __device__ __forceinline__ bool outliers_wide(int32_t n) { return n > kNarrowOutliers; }
 __host__ __device__ __forceinline__ int32_t pad64(int32_t n) { return (n + 63) & ~63; }
+
+// Whether the outlier columns fill at least half of the span they cover
+// (as for a low threshold, up to every column): the builders then move
+// aligned stretches of consecutive columns as 16-byte pieces. The choice
+// changes only the schedule, never a value.
+__device__ __forceinline__ bool outliers_dense(int32_t n, const int32_t *idx) {
+  if (n <= 0) return false;
+  const int32_t lo = __ldcg(idx), hi = __ldcg(idx + n - 1);
+  return hi - lo + 1 <= 2 * n;
+}
 
 // Element (row, t) of XO and (t, j) of WO.
 __device__ __forceinline__ int64_t xo_index(int64_t row, int32_t t, int32_t n, int32_t ldk) {
@@ -31,6 +43,90 @@ __device__ __forceinline__ int64_t xo_index(int64_t row, int32_t t, int32_t n, i
 __device__ __forceinline__ int64_t wo_index(int32_t t, int64_t j, int32_t n, int32_t o,
                                             int32_t ldk) {
   return outliers_wide(n) ? j * ldk + t : static_cast<int64_t>(t) * o + j;
+}
+
+// fp16(fp32(fp32(code) * scale) / 127) for the four signed byte codes of w.
+__device__ __forceinline__ uint2 dequant4(uint32_t w, float scale) {
+  uint16_t r[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int32_t code = static_cast<int32_t>(static_cast<int8_t>((w >> (8 * e)) & 0xFFu));
+    r[e] = __half_as_ushort(
+        __float2half_rn(__fdiv_rn(static_cast<float>(code) * scale, 127.0f)));
+  }
+  return make_uint2(static_cast<uint32_t>(r[0]) | (static_cast<uint32_t>(r[1]) << 16),
+                    static_cast<uint32_t>(r[2]) | (static_cast<uint32_t>(r[3]) << 16));
+}
+
+// The wide layout from the int8 codes (the value rule of build_wo_rows).
+// Work items are (j, g): 16 consecutive outlier positions t = 16g .. 16g+15
+// of row j, g fastest, so a warp reads one stretch of row j of wq and
+// writes 32 consecutive 32-byte pieces of row j of WO. Where those 16
+// positions are 16 consecutive, 16-aligned columns of X (every outlier
+// column in a dense stretch, as for a zero threshold) the codes come in
+// one 16-byte load; otherwise in 16 byte gathers. Positions from |O| up to
+// pad64(|O|) are written as zeros. Four items in flight per thread.
+__device__ __forceinline__ void build_wo_wide_codes(int32_t n, const int32_t *__restrict__ idx,
+                                                    const int8_t *__restrict__ wq,
+                                                    const float *__restrict__ aw, int32_t h,
+                                                    int32_t o, int32_t ldk,
+                                                    uint16_t *__restrict__ WO, int64_t first,
+                                                    int64_t stride) {
+  constexpr int UI = 4;
+  const int64_t G = pad64(n) >> 4;
+  const int64_t items = static_cast<int64_t>(o) * G;
+  // (j, g) of item `first`, and the step of `stride` items in those terms
+  int64_t j = first / G, g = first - (first / G) * G;
+  const int64_t dj = stride / G, dg = stride - (stride / G) * G;
+  for (int64_t q0 = first; q0 < items; q0 += UI * stride) {
+    uint4 code[UI];
+    float scale[UI];
+    int64_t jj[UI], tt[UI];
+#pragma unroll
+    for (int u = 0; u < UI; ++u) {
+      jj[u] = j;
+      tt[u] = g << 4;
+      code[u] = make_uint4(0u, 0u, 0u, 0u);
+      scale[u] = 0.0f;
+      if (q0 + u * stride < items && tt[u] < n) {
+        const int32_t t0 = static_cast<int32_t>(tt[u]);
+        const int8_t *row = wq + j * h;
+        scale[u] = __ldg(aw + j);
+        const int4 *ip = reinterpret_cast<const int4 *>(idx + t0);
+        const int4 i0 = __ldcg(ip), i3 = __ldcg(ip + 3);
+        if (t0 + 15 < n && i3.w - i0.x == 15 && (i0.x & 15) == 0) {
+          code[u] = __ldg(reinterpret_cast<const uint4 *>(row + i0.x));
+        } else {
+          const int4 i1 = __ldcg(ip + 1), i2 = __ldcg(ip + 2);
+          const int32_t c[16] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w,
+                                 i2.x, i2.y, i2.z, i2.w, i3.x, i3.y, i3.z, i3.w};
+          uint32_t b[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            if (t0 + e < n)
+              b[e >> 2] |= static_cast<uint32_t>(static_cast<uint8_t>(__ldg(row + c[e])))
+                           << (8 * (e & 3));
+          code[u] = make_uint4(b[0], b[1], b[2], b[3]);
+        }
+      }
+      g += dg;
+      j += dj;
+      if (g >= G) {
+        g -= G;
+        ++j;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < UI; ++u) {
+      if (q0 + u * stride >= items) break;
+      // codes past |O| are zero, and so are their values
+      const uint2 v0 = dequant4(code[u].x, scale[u]), v1 = dequant4(code[u].y, scale[u]);
+      const uint2 v2 = dequant4(code[u].z, scale[u]), v3 = dequant4(code[u].w, scale[u]);
+      uint4 *dst = reinterpret_cast<uint4 *>(WO + jj[u] * ldk + tt[u]);
+      dst[0] = make_uint4(v0.x, v0.y, v1.x, v1.y);
+      dst[1] = make_uint4(v2.x, v2.y, v3.x, v3.y);
+    }
+  }
 }
 
 // Step 2, W side, for every outlier column: WO[t][j] = fp16(fp32(fp32(
@@ -87,12 +183,19 @@ __device__ __noinline__ void build_wo_rows(int32_t n, const int32_t *__restrict_
     }
     return;
   }
-  // wide: the items are (t, j) with t < pad64(n) and j < o, stored at
-  // WO[j*ldk + t]. Each thread keeps one t (its index loaded once) and walks
-  // j; a warp covers 32 consecutive t of one row j, so the gathers from wq
-  // and the stores coalesce. With fewer threads than t values (a CTA
-  // building every row alone) each thread takes several t in turn.
   const int32_t T = pad64(n);
+  if (w16 == nullptr && outliers_dense(n, idx)) {
+    build_wo_wide_codes(n, idx, wq, aw, h, o, ldk, WO, first, stride);
+    // the wide tiles are read by TMA (the async proxy)
+    fence_proxy_async_global();
+    return;
+  }
+  // wide, scattered outlier columns (or from the fp16 weight): the items
+  // are (t, j) with t < pad64(n) and j < o, stored at WO[j*ldk + t]. Each
+  // thread keeps one t (its index loaded once) and walks j; a warp covers
+  // 32 consecutive t of one row j, so the stores coalesce. With fewer
+  // threads than t values (a CTA building every row alone) each thread
+  // takes several t in turn.
   constexpr int UW = 8;  // gathers in flight per thread
   auto column = [&](int32_t t, int64_t jbeg, int64_t jstep) {
     const bool tl = t < n;
@@ -136,6 +239,7 @@ __device__ __noinline__ void build_wo_rows(int32_t n, const int32_t *__restrict_
   } else {
     for (int64_t t = first; t < T; t += stride) column(static_cast<int32_t>(t), 0, 1);
   }
+  fence_proxy_async_global();
 }
 
 }  // namespace llmint8

@@ -623,8 +623,8 @@ __global__ void __launch_bounds__(kFixThreads) k_act_fixup(const FixupParams p) 
         const uint32_t mag = hv & 0x7FFFu;
         if (mag < thresh_bits) mo = mag;
       }
-    } else {
-    // four gathers in flight per lane (many outlier columns: up to h)
+    } else if (!outliers_dense(n, idx)) {
+    // four gathers in flight per lane (many scattered outlier columns)
     for (int32_t t0 = lane; t0 < n; t0 += 4 * 32) {
       int32_t jj[4];
       uint32_t hv[4];
@@ -648,6 +648,68 @@ __global__ void __launch_bounds__(kFixThreads) k_act_fixup(const FixupParams p) 
         }
       }
     }
+    } else {
+      // a dense outlier set (up to every column): groups of 8 consecutive
+      // positions t per lane, two groups in flight. A group whose 8 columns
+      // are 8 consecutive, 8-aligned columns of X moves as one 16-byte load,
+      // one 16-byte XO store and one 8-byte code store; any other group as
+      // 8 gathers.
+      int8_t *qr = Xq + row * h;
+      const int32_t ngroups = (n + 7) >> 3;
+      for (int32_t g0 = lane; g0 < ngroups; g0 += 2 * 32) {
+        int4 ia[2], ib[2];
+        uint4 v[2];
+        bool dense[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int32_t t0 = (g0 + 32 * u) << 3;
+          dense[u] = false;
+          v[u] = make_uint4(0u, 0u, 0u, 0u);
+          ia[u] = make_int4(0, 0, 0, 0);
+          ib[u] = ia[u];
+          if (t0 < n) {
+            ia[u] = __ldcg(reinterpret_cast<const int4 *>(idx + t0));
+            ib[u] = __ldcg(reinterpret_cast<const int4 *>(idx + t0) + 1);
+            dense[u] = t0 + 7 < n && ib[u].w - ia[u].x == 7 && (ia[u].x & 7) == 0;
+            if (dense[u]) {
+              v[u] = __ldg(reinterpret_cast<const uint4 *>(xr + ia[u].x));
+            } else {
+              const int32_t c[8] = {ia[u].x, ia[u].y, ia[u].z, ia[u].w,
+                                    ib[u].x, ib[u].y, ib[u].z, ib[u].w};
+              uint32_t wv[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                if (t0 + e < n) wv[e >> 1] |= static_cast<uint32_t>(xr[c[e]]) << (16 * (e & 1));
+              v[u] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            }
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int32_t t0 = (g0 + 32 * u) << 3;
+          if (t0 >= n) continue;
+          // positions past |O| hold zero, below every threshold
+          const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t lo = w[e] & 0x7FFFu, hi = (w[e] >> 16) & 0x7FFFu;
+            if (lo < thresh_bits) mo = max(mo, lo);
+            if (hi < thresh_bits) mo = max(mo, hi);
+          }
+          if (XO) *reinterpret_cast<uint4 *>(XO + row * p.ldk + t0) = v[u];
+          // the outlier columns' codes (a row sent to recomputation below is
+          // requantised whole, outlier columns zero again)
+          if (dense[u]) {
+            *reinterpret_cast<uint2 *>(qr + ia[u].x) = make_uint2(0u, 0u);
+          } else {
+            const int32_t c[8] = {ia[u].x, ia[u].y, ia[u].z, ia[u].w,
+                                  ib[u].x, ib[u].y, ib[u].z, ib[u].w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              if (t0 + e < n) qr[c[e]] = 0;
+          }
+        }
+      }
     }
     if (XO && outliers_wide(n))  // zero padding of the wide layout
       for (int32_t t = n + lane; t < pad64(n); t += 32) XO[row * p.ldk + t] = 0;

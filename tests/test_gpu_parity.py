@@ -497,6 +497,11 @@ WIDE_CASES = [
     (129, 1040, 784, tuple(range(3, 1040, 13)), 6.0),    # |O| = 80: a partial k-block
     (256, 512, 2048, (), 0.0),                           # every column out: |O| = 512
     (8, 1024, 512, tuple(range(5, 1024, 16)), 6.0),      # |O| = 64, decode and prefill
+    # |O| = 97, filling over half of its span (the builders' dense schedule):
+    # an aligned stretch (whole 8- and 16-column groups), a consecutive but
+    # unaligned run, scattered columns and a partial group
+    (200, 1024, 512, tuple(range(16, 80)) + tuple(range(83, 102)) + tuple(range(104, 200, 7)),
+     6.0),
 ]
 
 
