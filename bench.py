@@ -72,8 +72,10 @@ SOAK_MIN_S = 0.5
 # scale granularity flags -> LLMINT8_SCALE_VECTORWISE (0) / TENSORWISE (1)
 SCALE_MODES = {"row": 0, "column": 0, "tensor": 1}
 KERNEL_SOURCES = ["mixed_precision_int8_b200/csrc/gemm_sm100.cuh",
+                  "mixed_precision_int8_b200/csrc/gemm_pair_sm100.cuh",
                   "mixed_precision_int8_b200/csrc/decode_sm100.cuh",
                   "mixed_precision_int8_b200/csrc/quant_kernels.cuh",
+                  "mixed_precision_int8_b200/csrc/outlier_rows.cuh",
                   "mixed_precision_int8_b200/csrc/ptx_sm100.cuh",
                   "mixed_precision_int8_b200/csrc/llmint8_api.cu"]
 
@@ -509,14 +511,17 @@ def bench_workload(name, args, world, rank, local, K, Wm, headline: bool):
                 "kernel": kernel, "algorithmic_bytes": algo_bytes,
                 "peak_source": f"hbm_gbs ({peaks['source']})"}
     else:
-        kernel = "k_gemm_i8_fused"
+        kernel = ("k_gemm_i8_pair"
+                  if binding.llmint8_prefill_kernel(s, h, o) == binding.PATH_PREFILL_PAIR
+                  else "k_gemm_i8_fused")
         peak = 2.0 * peaks["bf16_tflops"]
         achieved = ops / (gemm_ms_avg * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak, "kernel": kernel,
                 "peak_source": "bf16_tflops x 2 (nominal int8/bf16 dense "
                                f"ratio 4.5/2.25), {peaks['source']}"}
-    roof["traffic"] = recorded_traffic(wl.name, kernel)
+    # the committed DRAM counters are for the workload's own threshold
+    roof["traffic"] = recorded_traffic(wl.name, kernel) if alpha_override is None else None
     roof["kernel_ms"] = gemm_ms_avg
     roof["kernel_timing"] = ("CUDA events recorded by the library around "
                              "this kernel, averaged over a second pass of the "

@@ -109,14 +109,35 @@ typedef struct {
     const uint16_t *w16_dev;
 } llmint8_weight;
 
+/* llmint8_matmul_opts.path */
+#define LLMINT8_PATH_AUTO 0
+#define LLMINT8_PATH_PREFILL 1
+#define LLMINT8_PATH_DECODE 2
+#define LLMINT8_PATH_PREFILL_SINGLE 3
+#define LLMINT8_PATH_PREFILL_PAIR 4
+
+/* The kernel llmint8_matmul runs, on the current device, for an [s, h] x
+ * [h, o] call with the automatic path: LLMINT8_PATH_DECODE (s <= 16),
+ * LLMINT8_PATH_PREFILL_PAIR (the int8 weight, h*o bytes, is larger than the
+ * device's L2 and CTA pairs fit the device) or LLMINT8_PATH_PREFILL_SINGLE.
+ * A negative llmint8_status on error (LLMINT8_ERR_SHAPE for s < 0, h <= 0
+ * or o <= 0; no usable device). Enqueues nothing. */
+LLMINT8_API int32_t llmint8_prefill_kernel(int64_t s, int64_t h, int64_t o);
+
 /* Optional extras for llmint8_matmul_ex (all fields may be zero/NULL).
  *  gemm_event_start/stop: cudaEvent_t (as void*) recorded on `stream`
  *      immediately before and after the int8 GEMM kernel launch, for timing
  *      the dominant kernel from the caller.
  *  ci_dev: if non-NULL, int32 [s][o] receives the exact int32 accumulators
  *      of Step 4 (testing; costs an extra 4*s*o bytes of stores).
- *  path: 0 = automatic, 1 = force the prefill GEMM kernel, 2 = force the
- *      decode (s <= 16) kernel; 2 with s > 16 is LLMINT8_ERR_ARG.
+ *  path: LLMINT8_PATH_AUTO (0) = automatic; LLMINT8_PATH_PREFILL (1) = the
+ *      prefill GEMM, its kernel chosen automatically; LLMINT8_PATH_DECODE
+ *      (2) = the decode (s <= 16) kernel, LLMINT8_ERR_ARG with s > 16;
+ *      LLMINT8_PATH_PREFILL_SINGLE (3) = the prefill GEMM with one CTA per
+ *      128 x 256 tile; LLMINT8_PATH_PREFILL_PAIR (4) = the prefill GEMM with
+ *      a pair of CTAs (a cluster of two) per 256 x 256 tile,
+ *      LLMINT8_ERR_UNSUPPORTED where no such cluster fits the device. Every
+ *      kernel gives the same results bit for bit.
  *  launches (out): number of kernels this call enqueued.
  *  x_scale: LLMINT8_SCALE_VECTORWISE (0, the method: one absmax per row of
  *      X) or LLMINT8_SCALE_TENSORWISE (one absmax for all of X, the largest

@@ -30,6 +30,8 @@ SCALE_VECTORWISE = 0  # LLMINT8_SCALE_VECTORWISE: per row of X / column of W
 # where the prefill path builds the fp16 outlier rows of W (LLMINT8_WO_*)
 WO_SHARED, WO_BEFORE_GEMM, WO_EACH_CTA = 0, 1, 2
 SCALE_TENSORWISE = 1  # LLMINT8_SCALE_TENSORWISE: one constant per tensor
+# llmint8_matmul_opts.path (LLMINT8_PATH_*)
+PATH_AUTO, PATH_PREFILL, PATH_DECODE, PATH_PREFILL_SINGLE, PATH_PREFILL_PAIR = 0, 1, 2, 3, 4
 
 _c_i64, _c_i32, _c_f32 = ctypes.c_int64, ctypes.c_int32, ctypes.c_float
 _vp, _sz = ctypes.c_void_p, ctypes.c_size_t
@@ -101,6 +103,7 @@ def load_library():
                                            _c_i64, _vp, _vp, _vp, _vp], _c_i32),
         "llmint8_read_device_status": ([_vp, _sz, _vp, _vp], _c_i32),
         "llmint8_decode_max_rows": ([], _c_i64),
+        "llmint8_prefill_kernel": ([_c_i64, _c_i64, _c_i64], _c_i32),
         "llmint8_matmul_noalloc": ([_vp, _c_i64, ctypes.POINTER(llmint8_weight),
                                     _c_f32, _vp, _vp], _c_i32),
         "llmint8_wait_selftest": ([_vp, _sz, ctypes.c_uint64, _vp], _c_i32),
@@ -124,7 +127,8 @@ EXPORTED = ("llmint8_status_string", "llmint8_workspace_size",
             "llmint8_prepare_weight_ex", "llmint8_quantize_rows_ex",
             "llmint8_matmul_host_ex", "llmint8_workspace_size_ex",
             "llmint8_workspace_size_host_ex", "llmint8_read_outlier_tiles_ex",
-            "llmint8_noalloc_read_device_status", "llmint8_prepare_weight_cols")
+            "llmint8_noalloc_read_device_status", "llmint8_prepare_weight_cols",
+            "llmint8_prefill_kernel")
 
 
 def status_string(code: int) -> str:
@@ -213,6 +217,15 @@ def llmint8_decode_max_rows() -> int:
     return int(load_library().llmint8_decode_max_rows())
 
 
+def llmint8_prefill_kernel(s: int, h: int, o: int) -> int:
+    """PATH_* value of the kernel the automatic choice runs for [s,h] x [h,o]
+    on the current device (PATH_DECODE, PATH_PREFILL_SINGLE or
+    PATH_PREFILL_PAIR)."""
+    r = int(load_library().llmint8_prefill_kernel(int(s), int(h), int(o)))
+    _check("llmint8_prefill_kernel", r if r < 0 else 0)
+    return r
+
+
 def llmint8_prepare_weight(W: torch.Tensor, stream=None,
                            keep_fp16: bool = False,
                            w_scale: int = SCALE_VECTORWISE) -> PreparedWeight:
@@ -283,7 +296,8 @@ def llmint8_matmul(X: torch.Tensor, w: PreparedWeight, alpha: float = 6.0,
     """C = LLM.int8()(X, W): X fp16 [s,h] on the GPU -> fp16 [s,o].
 
     ci (optional, int32 [s,o]) receives the exact int32 accumulators; path
-    forces the prefill (1) or decode (2) kernel; events = (start, stop)
+    forces a kernel (PATH_*: prefill 1, decode 2, prefill with one CTA per
+    tile 3, prefill with CTA pairs 4); events = (start, stop)
     torch.cuda.Event pair recorded around the GEMM kernel; x_scale =
     SCALE_TENSORWISE quantises X with one constant for the whole tensor;
     status_host (a HostStatusWord) reports device anomalies on the next call;

@@ -16,6 +16,7 @@
 #include "llmint8.h"
 #include "quant_kernels.cuh"
 #include "gemm_sm100.cuh"
+#include "gemm_pair_sm100.cuh"
 #include "decode_sm100.cuh"
 
 namespace {
@@ -39,6 +40,8 @@ struct DeviceInfo {
   bool init = false;
   bool supported = false;
   int sm_count = 0;
+  int max_pairs = 0;  // CTA pairs of the pair GEMM that fit at once (0: none)
+  int64_t l2_bytes = 0;
 };
 constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
@@ -55,6 +58,7 @@ llmint8_status device_info(DeviceInfo **out) {
     if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return LLMINT8_ERR_CUDA;
     d.supported = (prop.major == 10 && prop.minor == 0);
     d.sm_count = prop.multiProcessorCount;
+    d.l2_bytes = prop.l2CacheSize;
     if (d.supported) {
       if (cudaFuncSetAttribute(gemm::k_gemm_i8_fused, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)gemm::SMEM_BYTES) != cudaSuccess)
@@ -65,6 +69,28 @@ llmint8_status device_info(DeviceInfo **out) {
       if (cudaFuncSetAttribute(k_act_rows, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)kActSmemOnePerSm) != cudaSuccess)
         return LLMINT8_ERR_CUDA;
+      if (cudaFuncSetAttribute(gemm2::k_gemm_i8_pair,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)gemm2::SMEM_BYTES) != cudaSuccess)
+        return LLMINT8_ERR_CUDA;
+      // clusters of two co-resident CTAs the pair GEMM can have at once
+      // (an SM left over in a GPC cannot host half of one)
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2 * (unsigned)(d.sm_count / 2));
+      cfg.blockDim = dim3(gemm::NUM_THREADS);
+      cfg.dynamicSmemBytes = gemm2::SMEM_BYTES;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, gemm2::k_gemm_i8_pair, &cfg) != cudaSuccess)
+        clusters = 0;
+      cudaGetLastError();  // a refusal only leaves the pair kernel unused
+      d.max_pairs = std::min(clusters, d.sm_count / 2);
     }
     d.init = true;
   }
@@ -240,6 +266,27 @@ cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// The same for a kernel run by clusters of two CTAs along x.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pairs(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                         cudaStream_t st, bool pdl, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
@@ -479,7 +526,8 @@ int64_t outlier_cap(const llmint8_matmul_opts *opts, int64_t h) {
 // The options every matmul form checks before it enqueues anything.
 llmint8_status check_opts(const llmint8_matmul_opts *opts, int64_t s, int64_t h) {
   if (!opts) return LLMINT8_OK;
-  if (opts->path < 0 || opts->path > 2 || (opts->path == 2 && s > kDecodeMaxRows))
+  if (opts->path < LLMINT8_PATH_AUTO || opts->path > LLMINT8_PATH_PREFILL_PAIR ||
+      (opts->path == LLMINT8_PATH_DECODE && s > kDecodeMaxRows))
     return LLMINT8_ERR_ARG;
   if (opts->x_scale != LLMINT8_SCALE_VECTORWISE && opts->x_scale != LLMINT8_SCALE_TENSORWISE)
     return LLMINT8_ERR_ARG;
@@ -504,6 +552,16 @@ llmint8_status check_opts(const llmint8_matmul_opts *opts, int64_t s, int64_t h)
 bool host_status_set(const llmint8_matmul_opts *opts) {
   return opts && opts->status_host &&
          *reinterpret_cast<volatile int32_t *>(opts->status_host) != 0;
+}
+
+// Whether the automatic choice takes the CTA-pair GEMM for a prefill call:
+// where the int8 weight is larger than L2, so that its tiles stream from
+// HBM, and the device can run CTA pairs. Same-box measurements: on the
+// OPT-175B FFN shape (604 MB of weight) the pair kernel's layer step is
+// 1.8% shorter; where the weight stays in L2 (13B, 6.7B) the one-CTA kernel
+// is faster.
+bool pair_gemm_preferred(int64_t h, int64_t o, const DeviceInfo &dev) {
+  return dev.max_pairs >= 1 && h * o > dev.l2_bytes;
 }
 
 llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w, float alpha,
@@ -543,10 +601,20 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
   int32_t *count = count_word(ws);
   int32_t *status = status_word(ws);
 
-  const bool use_decode = (path == 2) || (path == 0 && s <= kDecodeMaxRows);
+  const bool use_decode =
+      (path == LLMINT8_PATH_DECODE) || (path == LLMINT8_PATH_AUTO && s <= kDecodeMaxRows);
+  // the prefill kernel: a CTA pair per 256 x 256 tile, or one CTA per
+  // 128 x 256 tile
+  const bool use_pair = !use_decode && (path == LLMINT8_PATH_PREFILL_PAIR ||
+                                        (path != LLMINT8_PATH_PREFILL_SINGLE &&
+                                         pair_gemm_preferred(w->h, w->o, *dev)));
+  if (use_pair && dev->max_pairs < 1) return LLMINT8_ERR_UNSUPPORTED;
 
   // Tensor maps first: a failure here must leave nothing enqueued.
   CUtensorMap tmA, tmB, tmOut, tmXO, tmWO;
+  // the pair kernel's boxes of Wq and W^O hold a CTA's half of a tile's
+  // columns
+  const uint32_t b_rows = use_pair ? (uint32_t)gemm2::BNH : (uint32_t)gemm::BN;
   if (use_decode) {
     // A = Wq tiles (rows of o), B = Xq rows (s <= 16, zero-filled to 16)
     if (!make_tmap_i8(&tmA, w->wq_dev, (uint64_t)h, (uint64_t)o, decode::BOX_K, decode::BM) ||
@@ -554,13 +622,13 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
       return LLMINT8_ERR_CUDA;
   } else {
     if (!make_tmap_i8(&tmA, xq, (uint64_t)h, (uint64_t)s, gemm::BK, gemm::BM) ||
-        !make_tmap_i8(&tmB, w->wq_dev, (uint64_t)h, (uint64_t)o, gemm::BK, gemm::BN) ||
+        !make_tmap_i8(&tmB, w->wq_dev, (uint64_t)h, (uint64_t)o, gemm::BK, b_rows) ||
         !make_tmap_f16(&tmOut, out, (uint64_t)o, (uint64_t)s, gemm::OUT_BOX_COLS, 32))
       return LLMINT8_ERR_CUDA;
     // the wide outlier tiles for the tensor cores (used only when |O| > 16)
     if (ldk > 0) {
       if (!make_tmap_f16(&tmXO, xo, (uint64_t)ldk, (uint64_t)s, gemm::OK, gemm::BM) ||
-          !make_tmap_f16(&tmWO, wo, (uint64_t)ldk, (uint64_t)o, gemm::OK, gemm::BN))
+          !make_tmap_f16(&tmWO, wo, (uint64_t)ldk, (uint64_t)o, gemm::OK, b_rows))
         return LLMINT8_ERR_CUDA;
     } else {
       tmXO = tmA;
@@ -696,12 +764,19 @@ llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w
     p.done_counter = done_counter_word(ws);
     p.status_host = status_host;
     p.timeout_ns = kTimeoutNs;
-    const int64_t tiles = (int64_t)p.num_m_blocks * p.num_n_blocks;
-    const int grid = (int)(tiles < dev->sm_count ? tiles : dev->sm_count);
     p.build_wo = gemm_builds_wo ? 1 : 0;
     p.wo_wait_ns = wo_build == LLMINT8_WO_EACH_CTA ? 0 : kWoWaitNs;
-    e = launch(gemm::k_gemm_i8_fused, dim3(grid), dim3(gemm::NUM_THREADS), gemm::SMEM_BYTES, st,
-               !timed, tmA, tmB, tmOut, tmXO, tmWO, p);
+    if (use_pair) {
+      const int64_t tiles = (int64_t)((p.num_m_blocks + 1) / 2) * p.num_n_blocks;
+      const int pairs = (int)(tiles < dev->max_pairs ? tiles : dev->max_pairs);
+      e = launch_pairs(gemm2::k_gemm_i8_pair, dim3(2 * pairs), dim3(gemm::NUM_THREADS),
+                       gemm2::SMEM_BYTES, st, !timed, tmA, tmB, tmOut, tmXO, tmWO, p);
+    } else {
+      const int64_t tiles = (int64_t)p.num_m_blocks * p.num_n_blocks;
+      const int grid = (int)(tiles < dev->sm_count ? tiles : dev->sm_count);
+      e = launch(gemm::k_gemm_i8_fused, dim3(grid), dim3(gemm::NUM_THREADS), gemm::SMEM_BYTES,
+                 st, !timed, tmA, tmB, tmOut, tmXO, tmWO, p);
+    }
     if (e != cudaSuccess) return LLMINT8_ERR_CUDA;
     if (opts && opts->gemm_event_stop)
       cudaEventRecord(reinterpret_cast<cudaEvent_t>(opts->gemm_event_stop), st);
@@ -1068,6 +1143,16 @@ extern "C" llmint8_status llmint8_matmul_noalloc(const uint16_t *X_dev, int64_t 
   // leaves nothing behind for the next one
   return matmul_impl(X_dev, s, w, alpha, out_dev, ws, (size_t)LLMINT8_NOALLOC_MAX_SCRATCH_BYTES,
                      nullptr, st, false, /*reset_state=*/true);
+}
+
+extern "C" int32_t llmint8_prefill_kernel(int64_t s, int64_t h, int64_t o) {
+  if (s < 0 || h <= 0 || o <= 0) return LLMINT8_ERR_SHAPE;
+  DeviceInfo *dev = nullptr;
+  const llmint8_status rc = device_info(&dev);
+  if (rc) return rc;
+  if (s <= kDecodeMaxRows) return LLMINT8_PATH_DECODE;
+  return pair_gemm_preferred(h, o, *dev) ? LLMINT8_PATH_PREFILL_PAIR
+                                         : LLMINT8_PATH_PREFILL_SINGLE;
 }
 
 extern "C" llmint8_status llmint8_noalloc_read_device_status(int32_t *bits_out, void *stream) {

@@ -137,9 +137,10 @@ def test_matmul_rejects_nulls_alignment_alpha_and_small_workspace(lib):
     opts.path = 2
     assert lib.llmint8_matmul_ex(FAKE, 17, ctypes.byref(w), 6.0, FAKE, FAKE,
                                  big, ctypes.byref(opts), None) == -7
-    opts.path = 3
-    assert lib.llmint8_matmul_ex(FAKE, 4, ctypes.byref(w), 6.0, FAKE, FAKE,
-                                 big, ctypes.byref(opts), None) == -7
+    for bad_path in (-1, binding.PATH_PREFILL_PAIR + 1):
+        opts.path = bad_path
+        assert lib.llmint8_matmul_ex(FAKE, 4, ctypes.byref(w), 6.0, FAKE, FAKE,
+                                     big, ctypes.byref(opts), None) == -7
 
 
 @needs_no_gpu
@@ -176,6 +177,11 @@ def test_scale_mode_constants_match_the_header():
     wo = dict(re.findall(r"#define\s+LLMINT8_WO_(\w+)\s+(\d+)", text))
     assert (int(wo["SHARED"]), int(wo["BEFORE_GEMM"]), int(wo["EACH_CTA"])) == (
         binding.WO_SHARED, binding.WO_BEFORE_GEMM, binding.WO_EACH_CTA)
+    paths = dict(re.findall(r"#define\s+LLMINT8_PATH_(\w+)\s+(\d+)", text))
+    assert {k: int(v) for k, v in paths.items()} == {
+        "AUTO": binding.PATH_AUTO, "PREFILL": binding.PATH_PREFILL,
+        "DECODE": binding.PATH_DECODE, "PREFILL_SINGLE": binding.PATH_PREFILL_SINGLE,
+        "PREFILL_PAIR": binding.PATH_PREFILL_PAIR}
     bits = dict(re.findall(r"#define\s+LLMINT8_DEV_(\w+)\s+(0x[0-9a-fA-F]+)", text))
     assert int(bits["TIMEOUT_SELFTEST"], 16) == binding.DEV_TIMEOUT_SELFTEST
     assert int(bits["OUTLIER_CAP"], 16) == binding.DEV_OUTLIER_CAP
