@@ -117,9 +117,9 @@ typedef struct {
 #define LLMINT8_PATH_PREFILL_PAIR 4
 
 /* The kernel llmint8_matmul runs, on the current device, for an [s, h] x
- * [h, o] call with the automatic path: LLMINT8_PATH_DECODE (s <= 16),
- * LLMINT8_PATH_PREFILL_PAIR (the int8 weight, h*o bytes, is larger than the
- * device's L2 and CTA pairs fit the device) or LLMINT8_PATH_PREFILL_SINGLE.
+ * [h, o] call with the automatic path: LLMINT8_PATH_DECODE (s <= 16) or
+ * LLMINT8_PATH_PREFILL_SINGLE (the CTA-pair kernel runs only when asked for
+ * with LLMINT8_PATH_PREFILL_PAIR).
  * A negative llmint8_status on error (LLMINT8_ERR_SHAPE for s < 0, h <= 0
  * or o <= 0; no usable device). Enqueues nothing. */
 LLMINT8_API int32_t llmint8_prefill_kernel(int64_t s, int64_t h, int64_t o);

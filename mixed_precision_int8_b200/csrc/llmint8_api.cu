@@ -554,14 +554,17 @@ bool host_status_set(const llmint8_matmul_opts *opts) {
          *reinterpret_cast<volatile int32_t *>(opts->status_host) != 0;
 }
 
-// Whether the automatic choice takes the CTA-pair GEMM for a prefill call:
-// where the int8 weight is larger than L2, so that its tiles stream from
-// HBM, and the device can run CTA pairs. Same-box measurements: on the
-// OPT-175B FFN shape (604 MB of weight) the pair kernel's layer step is
-// 1.8% shorter; where the weight stays in L2 (13B, 6.7B) the one-CTA kernel
-// is faster.
+// Whether the automatic choice takes the CTA-pair GEMM for a prefill call.
+// It does not: measured on B200 at the OPT shapes, the pair kernel is as
+// fast as the one-CTA kernel at best (175B FFN: 796 against 786 us per
+// launch under ncu, the tensor pipes 82% busy in both, with more DRAM reads
+// of Wq, 886 against 745 MB) and slower where the weight stays in L2 (13B
+// FFN: 291 against 279 us). It stays selectable (LLMINT8_PATH_PREFILL_PAIR).
 bool pair_gemm_preferred(int64_t h, int64_t o, const DeviceInfo &dev) {
-  return dev.max_pairs >= 1 && h * o > dev.l2_bytes;
+  (void)h;
+  (void)o;
+  (void)dev;
+  return false;
 }
 
 llmint8_status matmul_impl(const uint16_t *X, int64_t s, const llmint8_weight *w, float alpha,

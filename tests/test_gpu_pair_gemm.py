@@ -104,12 +104,10 @@ def test_pair_gemm_on_the_workloads(name):
 
 
 def test_automatic_kernel_choice():
-    """Pairs where the int8 weight exceeds L2 (it streams from HBM), one CTA
-    per tile where it fits, the decode kernel for s <= 16."""
-    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    """The decode kernel for s <= 16, else the one-CTA-per-tile GEMM (the
+    pair kernel only when asked for)."""
     assert binding.llmint8_prefill_kernel(8, 12288, 49152) == binding.PATH_DECODE
     assert binding.llmint8_prefill_kernel(2048, 4096, 4096) == binding.PATH_PREFILL_SINGLE
-    big = binding.llmint8_prefill_kernel(2048, 12288, 49152)
-    assert 12288 * 49152 > l2 and big == binding.PATH_PREFILL_PAIR
+    assert binding.llmint8_prefill_kernel(2048, 12288, 49152) == binding.PATH_PREFILL_SINGLE
     with pytest.raises(binding.Llmint8Error):
         binding.llmint8_prefill_kernel(-1, 16, 16)
