@@ -11,7 +11,7 @@ columns [col0, col0 + width) of W (llmint8_prepare_weight_cols, straight from
 the full fp16 W, no copy) and runs llmint8_matmul on them produces exactly
 that block of the layer's output, bit for bit, with no communication. A
 contiguous output, when the caller wants one, is an all-gather of the blocks
-over NCCL (torch.distributed) after the layer; nothing here multicasts.
+over NCCL (torch.distributed) after the layer.
 
 Every step of the layer runs in the CUDA library; this module only chooses
 column blocks and moves the finished blocks.
