@@ -412,11 +412,12 @@ def bench_workload(name, args, world, rank, local, K, Wm, headline: bool):
     n_outliers, _, _ = binding.llmint8_read_outlier_tiles(ws, tiles=False)  # |O|
 
     def timed_steps(n, with_kernel_events: bool):
-        """n steps, each between CUDA events on the launching stream (after
-        an L2 flush outside the events, where the workload needs one). With
-        with_kernel_events the library also records events around its
-        GEMM/decode kernel, which turns off that launch's overlap with the
-        kernel before it, so the step time is taken without them."""
+        """n steps timed with CUDA events on the launching stream: where the
+        workload needs an L2 flush, each step between its own events with
+        the flush outside them; otherwise the n steps back to back between
+        one pair. With with_kernel_events the library also records events
+        around its GEMM/decode kernel, which turns off that launch's overlap
+        with the kernel before it, so the step time is taken without them."""
         starts = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
         stops = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
         g0 = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
@@ -424,16 +425,27 @@ def bench_workload(name, args, world, rank, local, K, Wm, headline: bool):
         barrier(world)
         torch.cuda.synchronize()
         t0 = time.perf_counter()
-        for k in range(n):
-            if flush is not None:
-                flush.fill_(k & 0xFF)
-            starts[k].record(stream)
-            step((g0[k], g1[k]) if with_kernel_events else None)
-            stops[k].record(stream)
+        if flush is None and not with_kernel_events:
+            # nothing to keep out of the timing: the n steps run back to
+            # back, as consecutive layers do, between one pair of events
+            starts[0].record(stream)
+            for _ in range(n):
+                step(None)
+            stops[0].record(stream)
+        else:
+            for k in range(n):
+                if flush is not None:
+                    flush.fill_(k & 0xFF)
+                starts[k].record(stream)
+                step((g0[k], g1[k]) if with_kernel_events else None)
+                stops[k].record(stream)
         torch.cuda.synchronize()
         barrier(world)
         t1 = time.perf_counter()
-        step_ms = [a.elapsed_time(b) for a, b in zip(starts, stops)]
+        if flush is None and not with_kernel_events:
+            step_ms = [starts[0].elapsed_time(stops[0]) / n] * n
+        else:
+            step_ms = [a.elapsed_time(b) for a, b in zip(starts, stops)]
         kern_ms = ([binding.event_elapsed_ms(a, b) for a, b in zip(g0, g1)]
                    if with_kernel_events else None)
         return step_ms, kern_ms, t0, t1
