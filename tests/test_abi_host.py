@@ -285,3 +285,16 @@ def test_outlier_cap_and_status_word_are_validated_on_the_host(lib):
         opts.wo_build = bad
         assert lib.llmint8_matmul_ex(FAKE, 4, ctypes.byref(w), 6.0, FAKE, FAKE, big,
                                      ctypes.byref(opts), None) == -7
+
+
+def test_prefill_kernel_query_checks_shapes_before_the_device(lib):
+    """Bad sizes are LLMINT8_ERR_SHAPE on any host; without a usable GPU a
+    valid query is an error code (CUDA or unsupported), never a kernel."""
+    assert lib.llmint8_prefill_kernel(-1, 256, 256) == -2
+    assert lib.llmint8_prefill_kernel(16, 0, 256) == -2
+    assert lib.llmint8_prefill_kernel(16, 256, 0) == -2
+    rc = lib.llmint8_prefill_kernel(2048, 4096, 4096)
+    if torch.cuda.is_available():
+        assert rc in (binding.PATH_PREFILL_SINGLE, binding.PATH_PREFILL_PAIR)
+    else:
+        assert rc < 0
